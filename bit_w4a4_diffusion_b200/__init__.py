@@ -1,0 +1,252 @@
+"""B200 (sm_100a) SVDQuant W4A4 and AWQ W4A16 linear layers.
+
+Thin ctypes binding over ``lib/libsvdq_b200.so`` (C ABI in ``include/svdq.h``).
+Every function here only marshals arguments: it checks dtypes / devices,
+allocates outputs with torch when the caller gives none, and passes raw
+pointers and the current CUDA stream to the library.  All arithmetic of the
+layer happens in the library's CUDA kernels (or, for the offline weight pack,
+in its C++ host code).  If the library is missing, importing this package
+raises: there is no fallback.
+"""
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libsvdq_b200.so")
+
+SVDQ_NVFP4 = 0
+SVDQ_INT4 = 1
+SVDQ_RANK = 32
+PRECISIONS = {"nvfp4": SVDQ_NVFP4, "int4": SVDQ_INT4}
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"svdq status {status}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                          "(run `python -m bit_w4a4_diffusion_b200.build`)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, LL, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_ulonglong
+    sig = {
+        "svdq_status_string": (ctypes.c_char_p, [I]),
+        "svdq_last_error": (ctypes.c_char_p, []),
+        "svdq_version": (I, []),
+        "svdq_set_timeout_ns": (None, [U]),
+        "svdq_get_timeout_ns": (U, []),
+        "svdq_act_scale_bytes": (LL, [I, I, I]),
+        "svdq_weight_scale_bytes": (LL, [I, I, I]),
+        "svdq_workspace_bytes": (LL, [I, I, I, I]),
+        "svdq_scales_to_rowmajor": (I, [I, I, P, P]),
+        "svdq_scales_from_rowmajor": (I, [I, I, P, P]),
+        "svdq_pack_weights": (I, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
+        "svdq_quantize_act": (I, [I, I, I, I, P, P, P, F, F, P, P, P, P]),
+        "svdq_w4a4_gemm": (I, [I, I, I, I, I, P, P, P, P, P, P, P, F, P, P, P]),
+        "svdq_w4a4_linear": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, LL, P, P]),
+        "awq_pack_weights": (I, [I, I, P, P, P, P]),
+        "awq_w4a16_linear": (I, [I, I, I, P, P, P, P, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status):
+    if status != 0:
+        msg = lib.svdq_last_error().decode(errors="replace")
+        raise SvdqError(status, msg or lib.svdq_status_string(status).decode())
+
+
+def _prec(precision):
+    return PRECISIONS[precision] if isinstance(precision, str) else int(precision)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        assert t.is_contiguous(), "tensors must be contiguous"
+        return t.data_ptr()
+    if isinstance(t, np.ndarray):
+        assert t.flags["C_CONTIGUOUS"], "arrays must be C-contiguous"
+        return t.ctypes.data
+    return int(t)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev_bf16(t, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16):
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+    return t
+
+
+# ------------------------------------------------------------------ sizes ---
+
+def act_scale_bytes(precision, M, K):
+    return int(lib.svdq_act_scale_bytes(_prec(precision), M, K))
+
+
+def weight_scale_bytes(precision, N, K):
+    return int(lib.svdq_weight_scale_bytes(_prec(precision), N, K))
+
+
+def workspace_bytes(precision, M, K, rank=SVDQ_RANK):
+    return int(lib.svdq_workspace_bytes(_prec(precision), M, K, rank))
+
+
+def set_timeout_ns(ns):
+    lib.svdq_set_timeout_ns(int(ns))
+
+
+def get_timeout_ns():
+    return int(lib.svdq_get_timeout_ns())
+
+
+def scales_to_rowmajor(tiled, rows, K):
+    tiled = np.ascontiguousarray(np.asarray(tiled, dtype=np.uint8))
+    out = np.empty((rows, K // 16), dtype=np.uint8)
+    _check(lib.svdq_scales_to_rowmajor(rows, K, _ptr(tiled), _ptr(out)))
+    return out
+
+
+def scales_from_rowmajor(rowmajor, rows, K):
+    rowmajor = np.ascontiguousarray(np.asarray(rowmajor, dtype=np.uint8))
+    out = np.empty(weight_scale_bytes(SVDQ_NVFP4, rows, K), dtype=np.uint8)
+    _check(lib.svdq_scales_from_rowmajor(rows, K, _ptr(rowmajor), _ptr(out)))
+    return out
+
+
+# ------------------------------------------------------------------ host pack
+
+def svdq_pack_weights(precision, W_bits, smooth, L1_bits, L2_bits, rank=SVDQ_RANK):
+    """Host pack.  W_bits uint16 [N,K], smooth fp32 [K], L1_bits uint16 [K,r],
+    L2_bits uint16 [r,N].  Returns a dict of host numpy arrays."""
+    p = _prec(precision)
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    smooth = np.ascontiguousarray(smooth, dtype=np.float32)
+    L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    out = {
+        "codes": np.empty((N, K // 2), np.uint8),
+        "scales": np.empty(max(weight_scale_bytes(p, N, K), 1), np.uint8),
+        "weight_scale": np.zeros(1, np.float32),
+        "inv_smooth": np.empty(K, np.float32),
+        "lora_down": np.empty((rank, K), np.uint16),
+        "lora_up": np.empty((N, 2 * rank), np.uint16),
+    }
+    _check(lib.svdq_pack_weights(p, N, K, rank, _ptr(W_bits), _ptr(smooth), _ptr(L1_bits), _ptr(L2_bits),
+                                 _ptr(out["codes"]), _ptr(out["scales"]), _ptr(out["weight_scale"]),
+                                 _ptr(out["inv_smooth"]), _ptr(out["lora_down"]), _ptr(out["lora_up"])))
+    out["N"], out["K"], out["rank"], out["precision"] = N, K, rank, p
+    return out
+
+
+def awq_pack_weights(W_bits):
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    out = {"qweight": np.empty((N, K // 2), np.uint8), "scales": np.empty((N, K // 64), np.uint16),
+           "zeros": np.empty((N, K // 128), np.uint8)}
+    _check(lib.awq_pack_weights(N, K, _ptr(W_bits), _ptr(out["qweight"]), _ptr(out["scales"]), _ptr(out["zeros"])))
+    out["N"], out["K"] = N, K
+    return out
+
+
+def bits_to_bf16(bits, device=None):
+    """uint16 bit patterns (numpy) -> torch bfloat16 tensor (optionally on a device)."""
+    t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+    return t.to(device) if device is not None else t
+
+
+def to_device(packed, device="cuda"):
+    """Copy a host pack (dict of numpy arrays) to device tensors."""
+    d = {}
+    for k, v in packed.items():
+        if isinstance(v, np.ndarray):
+            if v.dtype == np.uint16:
+                d[k] = bits_to_bf16(v, device)
+            else:
+                d[k] = torch.from_numpy(v).to(device)
+        else:
+            d[k] = v
+    if "weight_scale" in packed:
+        d["weight_scale_f"] = float(np.asarray(packed["weight_scale"]).reshape(-1)[0])
+    return d
+
+
+# ------------------------------------------------------------------ device
+
+def svdq_quantize_act(precision, x, inv_smooth, lora_down, act_scale, weight_scale=1.0, out=None, stream=None,
+                      rank=SVDQ_RANK):
+    p = _prec(precision)
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    if out is None:
+        dev = x.device
+        out = (torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+               torch.empty(act_scale_bytes(p, M, K), dtype=torch.uint8, device=dev),
+               torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev))
+    codes, scales, lora_act = out
+    _check(lib.svdq_quantize_act(p, M, K, rank, _ptr(x), _ptr(inv_smooth), _ptr(lora_down), float(act_scale),
+                                 float(weight_scale), _ptr(codes), _ptr(scales), _ptr(lora_act), _stream(stream)))
+    return codes, scales, lora_act
+
+
+def svdq_w4a4_gemm(precision, act_codes, act_scales, lora_act, w, alpha, bias=None, y=None, dev_status=None,
+                   stream=None):
+    """w: device dict from to_device(svdq_pack_weights(...))."""
+    p = _prec(precision)
+    M = act_codes.shape[0]
+    N, K, rank = w["N"], w["K"], w["rank"]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _check(lib.svdq_w4a4_gemm(p, M, N, K, rank, _ptr(act_codes), _ptr(act_scales), _ptr(lora_act),
+                              _ptr(w["codes"]), _ptr(w["scales"]), _ptr(w["lora_up"]), _ptr(bias), float(alpha),
+                              _ptr(y), _ptr(dev_status), _stream(stream)))
+    return y
+
+
+def svdq_w4a4_linear(precision, x, w, act_scale, bias=None, y=None, workspace=None, dev_status=None, stream=None):
+    p = _prec(precision)
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    N, rank = w["N"], w["rank"]
+    assert K == w["K"]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(p, M, K, rank), dtype=torch.uint8, device=x.device)
+    wscale = w["weight_scale_f"]
+    _check(lib.svdq_w4a4_linear(p, M, N, K, rank, _ptr(x), _ptr(w["inv_smooth"]), _ptr(w["lora_down"]),
+                                float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), wscale, _ptr(w["lora_up"]),
+                                _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                _stream(stream)))
+    return y
+
+
+def awq_w4a16_linear(x, w, bias=None, y=None, stream=None):
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    N = w["N"]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib.awq_w4a16_linear(M, N, K, _ptr(x), _ptr(w["qweight"]), _ptr(w["scales"]), _ptr(w["zeros"]),
+                                _ptr(bias), _ptr(y), _stream(stream)))
+    return y

@@ -1,0 +1,295 @@
+// C-ABI entry points (declared in include/svdq.h): argument checks, device
+// checks, tensor-map set-up and kernel launches.  No allocation happens here:
+// every buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+
+#include "svdq.h"
+#include "svdq_internal.h"
+
+using namespace svdq;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Returns SVDQ_OK and the SM count if the current device is an sm_100 part.
+int check_device(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    d.ok = (d.cc_major == 10 && d.cc_minor == 0);
+    d.checked = true;
+  }
+  if (!d.ok)
+    return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "this library is built for sm_100a (B200); device %d is sm_%d%d", dev,
+                d.cc_major, d.cc_minor);
+  *sms = d.sms;
+  return SVDQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
+unsigned long long svdq_timeout_ns() { return g_timeout_ns.load(std::memory_order_relaxed); }
+
+int check_cuda(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+namespace svdq {
+
+bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace svdq
+
+extern "C" {
+
+const char* svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case SVDQ_ERR_UNSUPPORTED_DEVICE: return "unsupported device";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* svdq_last_error(void) { return g_last_error; }
+
+int svdq_version(void) { return SVDQ_VERSION; }
+
+void svdq_set_timeout_ns(unsigned long long ns) { g_timeout_ns.store(ns, std::memory_order_relaxed); }
+unsigned long long svdq_get_timeout_ns(void) { return g_timeout_ns.load(std::memory_order_relaxed); }
+
+long long svdq_act_scale_bytes(int precision, int M, int K) {
+  if (M < 0 || K <= 0) return -1;
+  const int64_t mp = round_up(M > 0 ? M : 1, 256);
+  if (precision == SVDQ_NVFP4) return (K % 64) ? -1 : mp * (K / 16);
+  if (precision == SVDQ_INT4) return (K % 64) ? -1 : mp * (K / 64) * 2;
+  return -1;
+}
+
+long long svdq_weight_scale_bytes(int precision, int N, int K) { return svdq_act_scale_bytes(precision, N, K); }
+
+long long svdq_workspace_bytes(int precision, int M, int K, int rank) {
+  if (M <= 0 || K <= 0 || rank != SVDQ_RANK) return -1;
+  const long long codes = round_up((int64_t)M * (K / 2), 256);
+  const long long scales = round_up(svdq_act_scale_bytes(precision, M, K), 256);
+  const long long lora = round_up((int64_t)M * 2 * rank * 2, 256);
+  if (scales < 0) return -1;
+  return codes + scales + lora;
+}
+
+int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
+                      const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,
+                      void* lora_act, void* stream) {
+  if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
+    return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
+  if (M <= 0 || K <= 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d must be positive", M, K);
+  if (K % 256 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of 256", K);
+  if (rank != SVDQ_RANK) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank=%d; this build supports rank %d", rank, SVDQ_RANK);
+  if (!x || !inv_smooth || !lora_down || !act_codes || !act_scales || !lora_act)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(x) || !aligned16(inv_smooth) || !aligned16(lora_down) || !aligned16(act_codes) ||
+      !aligned16(lora_act) || !aligned16(act_scales))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (precision == SVDQ_NVFP4 && !(act_scale > 0.f && weight_scale > 0.f))
+    return fail(SVDQ_ERR_INVALID_ARG, "NVFP4 tensor scales must be positive (act %g, weight %g)", act_scale,
+                weight_scale);
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  QuantActParams p{};
+  p.M = M;
+  p.K = K;
+  p.M_pad = (int)round_up(M, 256);
+  p.x = static_cast<const uint16_t*>(x);
+  p.inv_smooth = inv_smooth;
+  p.lora_down = static_cast<const uint16_t*>(lora_down);
+  p.act_scale = act_scale;
+  p.lora_scale = precision == SVDQ_NVFP4 ? 1.0f / (act_scale * weight_scale) : 1.0f;
+  p.act_codes = static_cast<uint8_t*>(act_codes);
+  p.act_scales = static_cast<uint8_t*>(act_scales);
+  p.lora_act = static_cast<uint16_t*>(lora_act);
+  return check_cuda(launch_quantize_act(p, precision == SVDQ_NVFP4, static_cast<cudaStream_t>(stream)),
+                    "quantize_act launch");
+}
+
+static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const void* act_scales, const void* lora_act,
+                           const void* w_codes, const void* w_scales, const void* lora_up, const void* bias,
+                           float alpha, void* y, int* dev_status, cudaStream_t stream, bool pdl, int sms) {
+  GemmTmaps t;
+  bool ok = true;
+  ok &= encode_tmap_2d(&t.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_codes, K / 2, M, K / 2, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&t.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, 256,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&t.la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_act, 2 * SVDQ_RANK, M, 2 * SVDQ_RANK * 2, 64,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
+                       256, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
+  GemmNvfp4Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.act_scales = static_cast<const uint8_t*>(act_scales);
+  p.w_scales = static_cast<const uint8_t*>(w_scales);
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.alpha = alpha;
+  p.dev_status = dev_status;
+  p.timeout_ns = svdq_timeout_ns();
+  return check_cuda(launch_gemm_nvfp4(p, t, sms, stream, pdl), "gemm_nvfp4 launch");
+}
+
+static int check_gemm_args(int precision, int M, int N, int K, int rank) {
+  if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
+    return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
+  if (M <= 0 || N <= 0 || K <= 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d N=%d K=%d must be positive", M, N, K);
+  if (K % 256 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of 256", K);
+  if (N % 128 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d must be a multiple of 128", N);
+  if (rank != SVDQ_RANK) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank=%d; this build supports rank %d", rank, SVDQ_RANK);
+  if (precision == SVDQ_INT4) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "INT4 W4A4 GEMM is not available in this build");
+  return SVDQ_OK;
+}
+
+int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                   const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                   const void* bias, float alpha, void* y, int* dev_status, void* stream) {
+  if (int s = check_gemm_args(precision, M, N, K, rank)) return s;
+  if (!act_codes || !act_scales || !lora_act || !w_codes || !w_scales || !lora_up || !y)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lora_act) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(lora_up) || !aligned16(y) || (bias && !aligned16(bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, y,
+                         dev_status, static_cast<cudaStream_t>(stream), false, sms);
+}
+
+int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
+                     const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
+                     float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
+                     long long workspace_bytes, int* dev_status, void* stream) {
+  if (int s = check_gemm_args(precision, M, N, K, rank)) return s;
+  if (!workspace) return fail(SVDQ_ERR_INVALID_ARG, "null workspace");
+  const long long need = svdq_workspace_bytes(precision, M, K, rank);
+  if (workspace_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* codes = ws;
+  uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
+  uint8_t* lora = scales + round_up(svdq_act_scale_bytes(precision, M, K), 256);
+  if (int s = svdq_quantize_act(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
+                                scales, lora, stream))
+    return s;
+  if (!w_codes || !w_scales || !lora_up || !y) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
+                         y, dev_status, static_cast<cudaStream_t>(stream), true, sms);
+}
+
+int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, const void* scales, const void* zeros,
+                     const void* bias, void* y, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d N=%d K=%d must be positive", M, N, K);
+  if (N % 16 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d must be a multiple of 16", N);
+  if (K % 128 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of 128", K);
+  if (!x || !qweight || !scales || !zeros || !y) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(y) || ((uintptr_t)scales & 1) || ((uintptr_t)bias & 1))
+    return fail(SVDQ_ERR_INVALID_ARG, "x, qweight and y must be 16-byte aligned; scales and bias 2-byte aligned");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  // Token rows are independent: process them 16 at a time (one weight pass each).
+  for (int m0 = 0; m0 < M; m0 += 16) {
+    AwqParams p{};
+    p.M = M - m0 < 16 ? M - m0 : 16;
+    p.N = N;
+    p.K = K;
+    p.x = static_cast<const uint16_t*>(x) + (size_t)m0 * K;
+    p.qweight = static_cast<const uint8_t*>(qweight);
+    p.scales = static_cast<const uint16_t*>(scales);
+    p.zeros = static_cast<const uint8_t*>(zeros);
+    p.bias = static_cast<const uint16_t*>(bias);
+    p.y = static_cast<uint16_t*>(y) + (size_t)m0 * N;
+    if (int s = check_cuda(launch_awq(p, sms, static_cast<cudaStream_t>(stream)), "awq launch")) return s;
+  }
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,299 @@
+// S1: smoothing + activation quantization + low-rank down-projection.
+//
+// Page: "Hugging Face integrates Nunchaku 4-bit diffusion inference into
+// Diffusers", section "SVDQuant and the Nunchaku engine": activation outliers
+// are migrated into the weights (x_hat = x / lambda per input channel), the
+// activations are quantized to 4 bits, and a 16-bit low-rank branch
+// x_hat * L1 runs beside them; the engine fuses that down-projection into the
+// quantize kernel so the branch costs almost no extra memory traffic.  Here
+// the same fusion is one HBM-bound pass over x:
+//
+//   x_hat = fp32(x) * inv_lambda                       (one fp32 multiply)
+//   NVFP4: per 16 along K, a = max|x_hat|, t = a / (6 s_a), sb = E4M3(t),
+//          d = float(sb) * s_a, code = E2M1(x_hat / d)   (RNE, satfinite)
+//   INT4:  per 64 along K, sc = bf16(a / 7), q = clamp(rint(x_hat / sc), -8, 7)
+//   u     = x_hat * L1 on tensor cores (mma.sync bf16, fp32 accumulate), with
+//           x_hat split into bf16 hi + lo so that u carries ~16 mantissa bits
+//   lora_act[m] = [hi(u * c) | lo(u * c)]  (bf16, 2r values per row), with
+//           c = 1 / (s_a s_w) for NVFP4 (folds the GEMM's per-tensor scale)
+//           and c = 1 for INT4.
+//
+// Mapping.  A CTA owns 16 rows; each warp walks 32-wide K blocks.  Lane
+// (g = lane / 4, c = lane % 4) loads 8 consecutive elements of rows g and g+8
+// at k = kb + 8c with 16-byte loads; these 16 values are exactly the lane's
+// mma.m16n8k16 A fragments for two K=16 steps under the k-permutation
+// logical(s, 2c + {0,1}, 2c + 8 + {0,1}) <-> kb + 8c + 4s + {0,1,2,3}; the B
+// fragments are loaded with the same permutation from L1^T, so the dot
+// products are unchanged.  A 16-group is the lane pair (c, c^1): its amax is
+// one shuffle.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+
+namespace {
+
+constexpr int S1_ROWS = 16;
+constexpr int S1_WARPS = 8;
+constexpr int S1_THREADS = S1_WARPS * 32;
+constexpr int S1_UNROLL = 4;
+
+SVDQ_DEV float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+
+SVDQ_DEV uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+SVDQ_DEV void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+SVDQ_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Exact E4M3 (non-negative) byte -> fp32 from the format fields.
+SVDQ_DEV float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xF, m = b & 7;
+  if (e == 0) return __uint2float_rn(m) * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Byte offset of scale (row, group) in the tiled NVFP4 scale layout:
+// 512-byte chunks of 128 rows x 4 groups, chunks ordered (row block, k chunk).
+SVDQ_DEV size_t sf_offset(int row, int group, int K) {
+  const int kchunks = K / 64;
+  return ((size_t)(row >> 7) * kchunks + (group >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
+}
+
+template <bool kNvfp4>
+__global__ void __launch_bounds__(S1_THREADS) quantize_act_kernel(QuantActParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int row0 = blockIdx.x * S1_ROWS + g;
+  const int row1 = row0 + 8;
+  const bool ok0 = row0 < p.M, ok1 = row1 < p.M;
+  const int K = p.K;
+  const int nblk = K / 32;
+
+  const uint16_t* __restrict__ x = p.x;
+  const uint16_t* __restrict__ l1t = p.lora_down;  // [r][K]
+  const float* __restrict__ inv_lam = p.inv_smooth;
+
+  // u accumulators: 4 n8 tiles (rank 32) x 4 fp32.
+  float acc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+
+  const float s_a = p.act_scale;
+  const float six_s = __fmul_rn(6.0f, s_a);
+
+  // INT4 needs a 64-group = two consecutive 32-blocks: a warp then walks pairs.
+  const int step = kNvfp4 ? 1 : 2;
+  for (int b0 = warp * step; b0 < nblk; b0 += S1_WARPS * step * S1_UNROLL) {
+    uint4 xa[S1_UNROLL * 2], xb[S1_UNROLL * 2];
+    // Issue all loads of this round first (memory-level parallelism).
+#pragma unroll
+    for (int u = 0; u < S1_UNROLL; ++u) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int blk = b0 + u * S1_WARPS * step + h;
+        const bool live = (h < step) && blk < nblk;
+        const int k = blk * 32 + 8 * c;
+        xa[2 * u + h] = (live && ok0) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row0 * K + k))
+                                      : make_uint4(0, 0, 0, 0);
+        xb[2 * u + h] = (live && ok1) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row1 * K + k))
+                                      : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < S1_UNROLL; ++u) {
+      const int blk_first = b0 + u * S1_WARPS * step;
+      if (blk_first >= nblk) break;
+      float v0[2][8], v1[2][8];  // x_hat for rows g, g+8; h = which 32-block
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h >= step) break;
+        const int k = (blk_first + h) * 32 + 8 * c;
+        const float4 il0 = __ldg(reinterpret_cast<const float4*>(inv_lam + k));
+        const float4 il1 = __ldg(reinterpret_cast<const float4*>(inv_lam + k + 4));
+        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+        unpack8(xa[2 * u + h], v0[h]);
+        unpack8(xb[2 * u + h], v1[h]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v0[h][i] = __fmul_rn(v0[h][i], il[i]);
+          v1[h][i] = __fmul_rn(v1[h][i], il[i]);
+        }
+      }
+
+      // ---------------- quantize ----------------
+      if constexpr (kNvfp4) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          a0 = fmaxf(a0, fabsf(v0[0][i]));
+          a1 = fmaxf(a1, fabsf(v1[0][i]));
+        }
+        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+        const uint32_t sb0 = cvt_e4m3(__fdiv_rn(a0, six_s));
+        const uint32_t sb1 = cvt_e4m3(__fdiv_rn(a1, six_s));
+        const float d0 = __fmul_rn(e4m3_value(sb0), s_a);
+        const float d1 = __fmul_rn(e4m3_value(sb1), s_a);
+        uint32_t w0 = 0, w1 = 0;
+        if (d0 != 0.f) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w0 |= cvt_e2m1x2(__fdiv_rn(v0[0][2 * i], d0), __fdiv_rn(v0[0][2 * i + 1], d0)) << (8 * i);
+        }
+        if (d1 != 0.f) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w1 |= cvt_e2m1x2(__fdiv_rn(v1[0][2 * i], d1), __fdiv_rn(v1[0][2 * i + 1], d1)) << (8 * i);
+        }
+        const int k = blk_first * 32 + 8 * c;
+        uint8_t* codes = p.act_codes;
+        if (ok0) *reinterpret_cast<uint32_t*>(codes + (size_t)row0 * (K / 2) + k / 2) = w0;
+        if (ok1) *reinterpret_cast<uint32_t*>(codes + (size_t)row1 * (K / 2) + k / 2) = w1;
+        if ((c & 1) == 0) {
+          const int grp = k >> 4;
+          p.act_scales[sf_offset(row0, grp, K)] = (uint8_t)sb0;  // rows >= M get 0 (zero input)
+          p.act_scales[sf_offset(row1, grp, K)] = (uint8_t)sb1;
+        }
+      } else {
+        // INT4: group of 64 = lanes c=0..3 over two 32-blocks.
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            a0 = fmaxf(a0, fabsf(v0[h][i]));
+            a1 = fmaxf(a1, fabsf(v1[h][i]));
+          }
+        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
+        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
+        const __nv_bfloat16 sc0 = __float2bfloat16_rn(__fdiv_rn(a0, 7.0f));
+        const __nv_bfloat16 sc1 = __float2bfloat16_rn(__fdiv_rn(a1, 7.0f));
+        const float f0 = __bfloat162float(sc0), f1 = __bfloat162float(sc1);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            int q0 = 0, q1 = 0;
+            if (f0 != 0.f) q0 = max(-8, min(7, __float2int_rn(__fdiv_rn(v0[h][i], f0))));
+            if (f1 != 0.f) q1 = max(-8, min(7, __float2int_rn(__fdiv_rn(v1[h][i], f1))));
+            w0 |= (uint32_t)(q0 & 0xF) << (4 * i);
+            w1 |= (uint32_t)(q1 & 0xF) << (4 * i);
+          }
+          const int k = (blk_first + h) * 32 + 8 * c;
+          if (ok0) *reinterpret_cast<uint32_t*>(p.act_codes + (size_t)row0 * (K / 2) + k / 2) = w0;
+          if (ok1) *reinterpret_cast<uint32_t*>(p.act_codes + (size_t)row1 * (K / 2) + k / 2) = w1;
+        }
+        if (c == 0) {
+          // INT4 activation scales: bf16, group-major [K/64][M_pad].
+          const int grp = blk_first >> 1;
+          uint16_t* sc = reinterpret_cast<uint16_t*>(p.act_scales);
+          sc[(size_t)grp * p.M_pad + row0] = __bfloat16_as_ushort(sc0);
+          sc[(size_t)grp * p.M_pad + row1] = __bfloat16_as_ushort(sc1);
+        }
+      }
+
+      // ---------------- low-rank down-projection ----------------
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h >= step) break;
+        const int k = (blk_first + h) * 32 + 8 * c;
+        uint32_t ahi[2][4], alo[2][4];
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          float h0[4], h1[4], l0[4], l1[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            h0[i] = bf16_round_f(v0[h][4 * s + i]);
+            h1[i] = bf16_round_f(v1[h][4 * s + i]);
+            l0[i] = __fsub_rn(v0[h][4 * s + i], h0[i]);
+            l1[i] = __fsub_rn(v1[h][4 * s + i], h1[i]);
+          }
+          ahi[s][0] = pack_bf16x2(h0[0], h0[1]);
+          ahi[s][1] = pack_bf16x2(h1[0], h1[1]);
+          ahi[s][2] = pack_bf16x2(h0[2], h0[3]);
+          ahi[s][3] = pack_bf16x2(h1[2], h1[3]);
+          alo[s][0] = pack_bf16x2(l0[0], l0[1]);
+          alo[s][1] = pack_bf16x2(l1[0], l1[1]);
+          alo[s][2] = pack_bf16x2(l0[2], l0[3]);
+          alo[s][3] = pack_bf16x2(l1[2], l1[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 bw = __ldg(reinterpret_cast<const uint4*>(l1t + (size_t)(8 * j + g) * K + k));
+          mma_bf16_16816(acc[j], ahi[0], bw.x, bw.y);
+          mma_bf16_16816(acc[j], alo[0], bw.x, bw.y);
+          mma_bf16_16816(acc[j], ahi[1], bw.z, bw.w);
+          mma_bf16_16816(acc[j], alo[1], bw.z, bw.w);
+        }
+      }
+    }
+  }
+
+  // Let the GEMM that consumes these outputs start its prologue.
+  pdl_launch_dependents();
+
+  // ---------------- cross-warp reduction of u, then the bf16 hi/lo fold ----
+  __shared__ float red[S1_WARPS][S1_ROWS][33];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    red[warp][g][8 * j + 2 * c] = acc[j][0];
+    red[warp][g][8 * j + 2 * c + 1] = acc[j][1];
+    red[warp][g + 8][8 * j + 2 * c] = acc[j][2];
+    red[warp][g + 8][8 * j + 2 * c + 1] = acc[j][3];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < S1_ROWS * 32; idx += S1_THREADS) {
+    const int r = idx >> 5, col = idx & 31;
+    float u = 0.f;
+#pragma unroll
+    for (int w = 0; w < S1_WARPS; ++w) u = __fadd_rn(u, red[w][r][col]);
+    const int row = blockIdx.x * S1_ROWS + r;
+    if (row < p.M) {
+      const float uf = __fmul_rn(u, p.lora_scale);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(uf);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(uf, __bfloat162float(hi)));
+      uint16_t* la = p.lora_act + (size_t)row * 64;
+      la[col] = __bfloat16_as_ushort(hi);
+      la[32 + col] = __bfloat16_as_ushort(lo);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream) {
+  const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
+  dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS);
+  if (nvfp4)
+    quantize_act_kernel<true><<<grid, S1_THREADS, 0, stream>>>(p);
+  else
+    quantize_act_kernel<false><<<grid, S1_THREADS, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

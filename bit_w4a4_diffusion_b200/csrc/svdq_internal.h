@@ -1,0 +1,65 @@
+// Internal launch interfaces shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace svdq {
+
+// Device-status codes written by bounded waits (0 = fine).
+enum DeviceStatus : int {
+  kDevOk = 0,
+  kDevTimeoutProducer = 1,
+  kDevTimeoutMma = 2,
+  kDevTimeoutEpilogue = 3,
+  kDevTimeoutDrain = 4,
+};
+
+struct QuantActParams {
+  int M, K, M_pad;            // M_pad: rows of the scale buffer (multiple of 256)
+  const uint16_t* x;          // bf16 [M, K]
+  const float* inv_smooth;    // fp32 [K]
+  const uint16_t* lora_down;  // bf16 [r, K]  (L1 transposed)
+  float act_scale;            // NVFP4 per-tensor activation scale s_a
+  float lora_scale;           // multiplier folded into lora_act (1/(s_a s_w) or 1)
+  uint8_t* act_codes;         // [M, K/2]
+  uint8_t* act_scales;        // NVFP4: tiled e4m3; INT4: bf16 [K/64][M_pad]
+  uint16_t* lora_act;         // bf16 [M, 2r]  (hi | lo)
+};
+
+cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream);
+
+struct GemmNvfp4Params {
+  int M, N, K;
+  const uint8_t* act_scales;  // tiled e4m3, rows padded to 256
+  const uint8_t* w_scales;    // tiled e4m3, rows padded to 256
+  const uint16_t* bias;       // bf16 [N] or null
+  float alpha;                // s_a * s_w
+  int* dev_status;            // may be null
+  unsigned long long timeout_ns;
+};
+
+struct GemmTmaps {
+  CUtensorMap a, b, la, lb, y;
+};
+
+cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                              bool pdl);
+
+struct AwqParams {
+  int M, N, K;
+  const uint16_t* x;       // bf16 [M, K]
+  const uint8_t* qweight;  // [N, K/2]
+  const uint16_t* scales;  // bf16 [N, K/64]
+  const uint8_t* zeros;    // [N, K/128] two 4-bit zeros per byte
+  const uint16_t* bias;    // bf16 [N] or null
+  uint16_t* y;             // bf16 [M, N]
+};
+
+cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream);
+
+// Tensor-map encoding through the driver entry point (no libcuda link needed).
+bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+}  // namespace svdq

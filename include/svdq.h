@@ -1,0 +1,176 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 / AWQ W4A16 linear layers.
+ *
+ * The layer (pages: "Hugging Face integrates Nunchaku 4-bit diffusion
+ * inference into Diffusers", section "SVDQuant and the Nunchaku engine";
+ * "Nunchaku Lite" Diffusers docs, "Supported quantization types" table):
+ *
+ *   y = (x diag(lambda)^-1) L1 L2 + Q(x diag(lambda)^-1) Q(R)^T + b,
+ *   R = W diag(lambda) - (L1 L2)^T,
+ *
+ * with a 16-bit rank-r branch L1 [K,r], L2 [r,N] (r = 32) and a 4-bit
+ * residual: NVFP4 (E2M1 codes, an E4M3 scale per 16 elements, an fp32
+ * per-tensor scale) or INT4 (signed, a bf16 scale per 64 elements).
+ *
+ * Conventions for every call:
+ *  - All integers are element counts.  Matrices are row-major; x is [M,K],
+ *    W is [N,K] (nn.Linear layout), y is [M,N].  bf16 data is passed as its
+ *    16-bit patterns.
+ *  - "device" pointers are CUDA device addresses owned by the caller (for
+ *    example torch tensors); "host" pointers are ordinary host memory owned by
+ *    the caller.  The library never allocates, frees or retains a pointer.
+ *  - Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Device calls are asynchronous on that stream; errors found
+ *    before launch are returned synchronously, nothing is launched then.
+ *  - Return value: an svdq_status.  svdq_last_error() gives a thread-local
+ *    message for the last failure.  No C++ exception crosses this boundary.
+ *  - `dev_status` (may be NULL) is a device int32 the GEMM kernels set to a
+ *    nonzero code when one of their bounded internal waits gives up; the
+ *    kernel then drains its copies, frees its tensor memory and exits.  The
+ *    caller reads it after synchronizing and should clear it beforehand.
+ *  - Device calls require a compute-capability 10.0 GPU (B200) as the
+ *    current device, else SVDQ_ERR_UNSUPPORTED_DEVICE.  There is no fallback.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SVDQ_VERSION 1
+#define SVDQ_RANK 32 /* the rank this build supports ("rank": 32 in the docs' config example) */
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null / misaligned pointer, bad enum, bad scale */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* a shape rule below is broken */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 */
+  SVDQ_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
+  SVDQ_ERR_DEVICE_TIMEOUT = 5      /* reported through dev_status, never returned */
+} svdq_status;
+
+/* "precision" of svdq_w4a4 in the "Supported quantization types" table:
+ * nvfp4 with group size 16, int4 with group size 64. */
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_precision;
+
+const char* svdq_status_string(int status);
+const char* svdq_last_error(void);
+int svdq_version(void);
+
+/* Upper bound, in nanoseconds, on any single internal wait of a GEMM kernel
+ * before it gives up and reports through dev_status (default 1e9).  Affects
+ * launches made after the call, from any thread. */
+void svdq_set_timeout_ns(unsigned long long ns);
+unsigned long long svdq_get_timeout_ns(void);
+
+/* ------------------------------------------------------------------ layouts
+ * Codes: 4-bit values, two per byte, element 2j in the low nibble of byte j
+ * of its row.  NVFP4 codes are E2M1 (bit 3 = sign); INT4 codes are two's
+ * complement in [-7, 7].
+ *
+ * NVFP4 scales ("tiled" layout, what the block-scaled MMA consumes): E4M3
+ * bytes, rows padded with zeros to a multiple of 256.  Scale (row m, group g),
+ * g = k/16, sits at byte
+ *     ((m/128) * (K/64) + g/4) * 512 + (m%32) * 16 + ((m%128)/32) * 4 + g%4.
+ * INT4 scales: bf16, group-major [K/64][rows padded to 256], zero padded.
+ * Sizes in bytes (or -1 for an unsupported precision / K): */
+long long svdq_act_scale_bytes(int precision, int M, int K);
+long long svdq_weight_scale_bytes(int precision, int N, int K);
+
+/* Host helpers: NVFP4 scales between row-major [rows, K/16] and tiled. */
+int svdq_scales_to_rowmajor(int rows, int K, const uint8_t* tiled, uint8_t* rowmajor);
+int svdq_scales_from_rowmajor(int rows, int K, const uint8_t* rowmajor, uint8_t* tiled);
+
+/* ------------------------------------------------------------------ host pack
+ * svdq_pack_weights: offline weight preparation (host, untimed).
+ * "SVDQuant and the Nunchaku engine": outliers migrate into the weights, a
+ * 16-bit low-rank branch absorbs the hardest part, the residual is quantized
+ * to 4 bits.  Computes, in this order:
+ *   inv_smooth[k] = fp32(1 / smooth[k]);
+ *   R[n,k] = fp32( W[n,k]*smooth[k] - sum_{t ascending} L1[k,t]*L2[t,n] )
+ *            (products and sum in fp64, one rounding to fp32);
+ *   NVFP4: s_w = amax|R| / 2688 (1 if R == 0); per 16 along k:
+ *          a = max|v|, sb = E4M3_rn_sat(a / fp32(6 s_w)), d = float(sb)*s_w,
+ *          code = E2M1_rn_sat(v / d) (sign kept), all codes 0 when d == 0.
+ *   INT4:  per 64 along k: sc = bf16(a / 7), q = clamp(rint(v / sc), -8, 7).
+ * Inputs (host): W bf16 [N,K]; smooth fp32 [K] (lambda, > 0); L1 bf16 [K,r];
+ * L2 bf16 [r,N].  Outputs (host, caller-allocated):
+ *   codes      [N, K/2] bytes
+ *   scales     svdq_weight_scale_bytes(precision, N, K) bytes
+ *   weight_scale  1 float (s_w; 1.0 for INT4)
+ *   inv_smooth fp32 [K]
+ *   lora_down  bf16 [r, K]   (L1 transposed, the down-projection operand)
+ *   lora_up    bf16 [N, 2r]  (row n = [L2[:,n], L2[:,n]], the up-projection
+ *                             operand for the hi/lo split activation)
+ * Shapes: N % 128 == 0, K % 256 == 0, rank == SVDQ_RANK. */
+int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, const float* smooth,
+                      const uint16_t* L1, const uint16_t* L2, uint8_t* codes, uint8_t* scales, float* weight_scale,
+                      float* inv_smooth, uint16_t* lora_down, uint16_t* lora_up);
+
+/* ------------------------------------------------------------------ device
+ * svdq_quantize_act: smoothing + activation quantization + low-rank
+ * down-projection in one pass over x (the Nunchaku engine's fused
+ * "down-projection + quantize" kernel, "SVDQuant and the Nunchaku engine").
+ *   x_hat = fp32(x) * inv_smooth;  codes/scales as in svdq_pack_weights with
+ *   s = act_scale for NVFP4;  u = x_hat L1 (fp32 accumulate);
+ *   lora_act[m] = [hi(u*c), lo(u*c)] (bf16 pair whose sum is u*c to ~2^-16),
+ *   c = 1/(act_scale*weight_scale) for NVFP4 and 1 for INT4.
+ * Device inputs: x bf16 [M,K]; inv_smooth fp32 [K]; lora_down bf16 [r,K].
+ * Device outputs: act_codes [M, K/2]; act_scales svdq_act_scale_bytes;
+ * lora_act bf16 [M, 2r].  act_scale (NVFP4 s_a, e.g. amax|x_hat|/2688) and
+ * weight_scale must be > 0 for NVFP4 and are ignored for INT4.
+ * Shapes: M >= 1, K % 256 == 0, rank == SVDQ_RANK. */
+int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
+                      const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,
+                      void* lora_act, void* stream);
+
+/* svdq_w4a4_gemm: the 4-bit GEMM with the low-rank up-projection and bias in
+ * its epilogue (the engine's fused "up-projection + 4-bit GEMM" kernel), on
+ * already-quantized activations:
+ *   y = bf16( alpha * ( sum_k deq(a) deq(w) + lora_act . lora_up^T ) + bias )
+ * with alpha = s_a * s_w (NVFP4).  Device inputs as produced by
+ * svdq_quantize_act and svdq_pack_weights; bias bf16 [N] or NULL; output y
+ * bf16 [M,N].  Shapes: M >= 1, N % 128 == 0, K % 256 == 0. */
+int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                   const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                   const void* bias, float alpha, void* y, int* dev_status, void* stream);
+
+/* svdq_w4a4_linear: the whole layer, svdq_quantize_act then svdq_w4a4_gemm on
+ * `stream` (the GEMM is launched with programmatic dependent launch so its
+ * prologue overlaps the quantize kernel's tail).  `workspace` is a device
+ * buffer of at least svdq_workspace_bytes(precision, M, K, rank) bytes that
+ * holds the quantized activations between the two kernels; calls that share
+ * a workspace must not overlap in time. */
+long long svdq_workspace_bytes(int precision, int M, int K, int rank);
+int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
+                     const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
+                     float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
+                     long long workspace_bytes, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------------ AWQ W4A16
+ * "Nunchaku Lite" docs, "Supported quantization types" table: awq_w4a16,
+ * int4, group size 64 -- an INT4 weight-only AWQ-style kernel for the
+ * memory-bound modulation (adaptive-norm) projections.  Asymmetric uint4 with
+ * an integer zero point per 64 along K:
+ *   mx, mn = max, min of the group; rng = mx - mn (|mx| if 0, then 1 if 0);
+ *   sc = bf16(rng / 15); z = clamp(rint(-mn / sc), 0, 15);
+ *   q = clamp(rint(w / sc) + z, 0, 15);  deq = (q - z) * sc.
+ * awq_pack_weights (host): W bf16 [N,K] -> qweight [N, K/2] (two codes per
+ * byte, element 2j low nibble), scales bf16 [N, K/64], zeros [N, K/128]
+ * (group 2j in the low nibble).  K % 128 == 0.
+ * awq_w4a16_linear (device): y bf16 [M,N] = bf16(x deq^T + bias), x bf16
+ * [M,K], bias bf16 [N] or NULL.  Rows are processed 16 at a time (each group
+ * of 16 rows streams the weight once).  N % 16 == 0, K % 128 == 0. */
+int awq_pack_weights(int N, int K, const uint16_t* W, uint8_t* qweight, uint16_t* scales, uint8_t* zeros);
+int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, const void* scales, const void* zeros,
+                     const void* bias, void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVDQ_H */

@@ -1,0 +1,88 @@
+"""The library's C++ host packer against the oracle (CPU only, bit-exact).
+
+Two independent implementations of the offline weight preparation (the
+oracle's numpy code and the library's C++) must agree bit for bit on the
+residual's quantized codes, the group scales, the tensor scale and the
+inverse smoothing vector.
+"""
+import numpy as np
+import pytest
+
+import bit_w4a4_diffusion_b200 as B
+import workloads as wl
+from oracle import awq as OA
+from oracle import svdq as O
+
+
+def _nibbles(packed):
+    lo = packed & 0xF
+    hi = packed >> 4
+    return np.stack([lo, hi], axis=-1).reshape(packed.shape[0], -1)
+
+
+CASES = [
+    ("tiny", {}),
+    ("qkv", dict(M=64, N=1024, K=3072)),
+    ("mlp_down", dict(M=64, N=384, K=2048)),
+    ("int4_m1024", dict(M=64, N=512, K=1024)),
+]
+
+
+@pytest.mark.parametrize("name,kw", CASES)
+def test_pack_weights_matches_oracle(name, kw):
+    c = wl.SVDQ_CASES[name]
+    if kw:
+        c = wl.scaled_case(c, **kw)
+    inp = wl.make_svdq_inputs(c)
+    pk = B.svdq_pack_weights(c.precision, inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    ref = O.pack_weights(c.precision, inp.W, inp.lam, inp.L1, inp.L2)
+    assert np.array_equal(pk["inv_smooth"], ref["inv_lam"])
+    if c.precision == "nvfp4":
+        assert pk["weight_scale"][0] == ref["s_w"]
+        assert np.array_equal(_nibbles(pk["codes"]), ref["codes"])
+        assert np.array_equal(B.scales_to_rowmajor(pk["scales"], c.N, c.K), ref["scales"])
+        # padding rows of the tiled layout are zero
+        tiled_again = B.scales_from_rowmajor(ref["scales"], c.N, c.K)
+        assert np.array_equal(tiled_again, pk["scales"])
+    else:
+        q = _nibbles(pk["codes"]).astype(np.int8)
+        q = np.where(q > 7, q - 16, q).astype(np.int8)
+        assert np.array_equal(q, ref["q"])
+        np_ = (c.N + 255) // 256 * 256
+        sc = pk["scales"].view(np.uint16).reshape(c.K // 64, np_)[:, :c.N].T
+        assert np.array_equal(wl.to_bf16(ref["sc"])[0], sc)
+    # low-rank operand layouts
+    assert np.array_equal(pk["lora_down"], inp.L1_bits.T)
+    assert np.array_equal(pk["lora_up"][:, :32], inp.L2_bits.T)
+    assert np.array_equal(pk["lora_up"][:, 32:], inp.L2_bits.T)
+
+
+def test_pack_rejects_bad_shapes():
+    W = np.zeros((100, 256), np.uint16)
+    with pytest.raises(B.SvdqError):
+        B.svdq_pack_weights("nvfp4", W, np.ones(256, np.float32), np.zeros((256, 32), np.uint16),
+                            np.zeros((32, 100), np.uint16))
+
+
+def test_scale_layout_formula_round_trip():
+    rng = np.random.default_rng(5)
+    rows, K = 300, 512
+    rm = rng.integers(0, 127, (rows, K // 16)).astype(np.uint8)
+    tiled = B.scales_from_rowmajor(rm, rows, K)
+    assert tiled.size == 512 * (K // 16)
+    # spot-check the documented offset formula
+    for (m, g) in [(0, 0), (37, 5), (129, 31), (299, 17)]:
+        off = ((m // 128) * (K // 64) + g // 4) * 512 + (m % 32) * 16 + ((m % 128) // 32) * 4 + g % 4
+        assert tiled[off] == rm[m, g]
+    assert np.array_equal(B.scales_to_rowmajor(tiled, rows, K), rm)
+
+
+@pytest.mark.parametrize("N,K", [(64, 256), (18432 // 16, 3072)])
+def test_awq_pack_matches_oracle(N, K):
+    inp = wl.make_awq_inputs(2, N=N, K=K)
+    pk = B.awq_pack_weights(inp.W_bits)
+    q, sc, z = OA.awq_quantize(inp.W)
+    assert np.array_equal(_nibbles(pk["qweight"]), q)
+    assert np.array_equal(pk["scales"], wl.to_bf16(sc)[0])
+    zz = np.stack([pk["zeros"] & 0xF, pk["zeros"] >> 4], axis=-1).reshape(N, -1)
+    assert np.array_equal(zz, z)

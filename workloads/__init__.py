@@ -9,6 +9,8 @@ offline calibration recipe that produces the layer's *inputs*:
 * a rank-r factorisation L1 [K, r], L2 [r, N] of (W diag(lambda))^T, taken
   from a seeded randomized subspace iteration in fp64 (Halko, Martinsson &
   Tropp 2011, Alg. 4.4) with all of Sigma put on L1, both rounded to bf16;
+* the static NVFP4 activation tensor scale s_a = amax|x_ij / lambda_j| / 2688
+  over the calibration batch (the batch itself), in fp32;
 * for the AWQ layer, the per-input-channel scale s_j = mean_i(|x_ij|)^0.5
   folded as W diag(s) and x / s, both rounded to bf16.
 
@@ -134,6 +136,7 @@ class SvdqInputs:
     L2: np.ndarray
     bias_bits: object = None    # uint16 [N] or None
     bias: object = None
+    act_scale: float = 1.0      # calibrated NVFP4 activation tensor scale (fp32)
     extra: dict = field(default_factory=dict)
 
 
@@ -159,7 +162,16 @@ def make_svdq_inputs(case: SvdqCase) -> SvdqInputs:
     b_bits = b_v = None
     if bias is not None:
         b_bits, b_v = to_bf16(bias)
-    return SvdqInputs(case, x_bits, x_v, W_bits, W_v, lam, L1_bits, L1_v, L2_bits, L2_v, b_bits, b_v)
+    return SvdqInputs(case, x_bits, x_v, W_bits, W_v, lam, L1_bits, L1_v, L2_bits, L2_v, b_bits, b_v,
+                      calibrated_act_scale(x_v, lam))
+
+
+def calibrated_act_scale(x, lam):
+    """Static activation tensor scale from a calibration batch: amax over
+    x_ij * (1/lambda_j) (fp32 reciprocal, fp32 product), divided by 6 * 448."""
+    inv = (np.float32(1.0) / lam.astype(np.float32)).astype(np.float32)
+    amax = np.float32(np.max(np.abs((x.astype(np.float32) * inv[None, :]).astype(np.float32))))
+    return np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
 
 
 # The five workloads (diffusion-transformer shapes).  "1% of channels" is
