@@ -1,0 +1,386 @@
+"""Benchmark: SVDQuant W4A4 NVFP4 linear layer on B200.
+
+One step = one ``svdq_w4a4_linear`` call (activation smoothing + NVFP4
+quantize + low-rank down-projection, then the block-scaled FP4 GEMM with the
+low-rank up-projection and bias) on the DiT MLP up-projection workload:
+x bf16 [4096, 3072] -> y bf16 [4096, 12288], rank 32.  TFLOPS = 2 M N K / t
+(the low-rank FLOPs are not counted).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun: every rank runs its own replica of the layer
+on its own batch (tokens are independent; no collective on the data path),
+time is the max over ranks, value = FLOPs of all ranks / that time.
+
+``--impl reference`` times the CPU oracle (the plain numpy restatement in
+oracle/) on a bounded sample of rows of the same workload.
+Prints one JSON line (rank 0).
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SVDQ W4A4 linear TFLOPS at M=4096,K=3072,N=12288 NVFP4; % of B200 FP4 peak"
+WORKLOAD = "mlp_up"
+FP4_SPEC_DENSE_TFLOPS = 9000.0      # NVIDIA B200 dense FP4 (18 PF is with 2:4 sparsity)
+FP4_PER_BF16 = 4.0                  # nominal dense FP4 : BF16 throughput ratio
+L2_BYTES = 126 * 2 ** 20
+
+
+def _measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_offline(inp):
+    """The oracle's offline weight pack and weight dequantization (untimed)."""
+    from oracle import svdq as O
+    pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
+    return pw, O.dequantized_weight("nvfp4", pw)
+
+
+def oracle_step_fn(case, inp, rows_per_step, offline):
+    """Per step: the oracle's activation quantization and fp64 layer output for
+    `rows_per_step` rows (cycling through x)."""
+    from oracle import svdq as O
+    pw, deq_w = offline
+    L1 = inp.L1.astype(np.float64)
+    L2 = inp.L2.astype(np.float64)
+    state = {"r0": 0}
+
+    def step():
+        r0 = state["r0"]
+        rows = (np.arange(rows_per_step) + r0) % case.M
+        state["r0"] = (r0 + rows_per_step) % case.M
+        act = O.quantize_activations("nvfp4", inp.x[rows], pw["inv_lam"], np.float32(inp.act_scale))
+        y = O.dequantized_act("nvfp4", act) @ deq_w.T
+        y += (act["x_hat"].astype(np.float64) @ L1) @ L2
+        if inp.bias is not None:
+            y += inp.bias[None, :]
+        return y
+
+    return step
+
+
+def time_oracle(case, inp, steps, warmup, budget_s):
+    """Returns (TFLOPS, seconds per step, rows per step)."""
+    offline = oracle_offline(inp)
+    probe = oracle_step_fn(case, inp, 32, offline)
+    probe()
+    t0 = time.perf_counter()
+    probe()
+    t_row = (time.perf_counter() - t0) / 32
+    rows = int(max(1, min(case.M, budget_s / max(steps + warmup, 1) / max(t_row, 1e-6))))
+    fn = oracle_step_fn(case, inp, rows, offline)
+    for _ in range(warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        fn()
+    dt = (time.perf_counter() - t0) / steps
+    return 2.0 * rows * case.N * case.K / dt / 1e12, dt, rows
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period_s=0.005):
+        self.samples, self.reasons, self.period = [], set(), period_s
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_w4a4_diffusion_b200 as B
+    import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    case = wl.SVDQ_CASES[WORKLOAD]
+    inp = wl.make_svdq_inputs(case)
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    s_a = float(inp.act_scale)
+    M, N, K = case.M, case.N, case.K
+    flops = 2.0 * M * N * K
+
+    # Rotate over enough independent weight / activation / output sets that
+    # a step's working set is never L2-resident from the previous use.
+    per_set = M * K * 2 + M * N * 2 + N * K // 2 + N * K // 16 + N * 128
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = []
+    x0 = B.bits_to_bf16(inp.x_bits, dev)
+    bias = B.bits_to_bf16(inp.bias_bits, dev) if inp.bias_bits is not None else None
+    for i in range(nsets):
+        w = B.to_device(pk, dev)
+        sets.append(dict(w=w, x=x0.clone(), y=torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                         ws=torch.empty(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev),
+                         codes=torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                         scales=torch.empty(B.act_scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev),
+                         lora=torch.empty((M, 64), dtype=torch.bfloat16, device=dev)))
+    stream = torch.cuda.current_stream(dev)
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk["weight_scale"][0])))
+
+    def layer(i, st=None):
+        s = sets[i % nsets]
+        B.svdq_w4a4_linear("nvfp4", s["x"], s["w"], s_a, bias=bias, y=s["y"], workspace=s["ws"],
+                           stream=st if st is not None else torch.cuda.current_stream(dev))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- timed region: K steps of the whole layer, replayed from a CUDA graph
+    # of G consecutive steps (rotating the sets) so host launch cost is off the
+    # critical path; a remainder is launched eagerly.
+    for i in range(args.warmup):
+        layer(i)
+    torch.cuda.synchronize()
+    G = nsets * max(1, 16 // nsets)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(G):
+            layer(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    reps, rem = divmod(args.steps, G)
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with sampler:
+        torch.cuda._sleep(20_000_000)          # let the host queue run ahead of the GPU
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        for i in range(rem):
+            layer(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    t_ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_per_step = t_ms / args.steps
+    value = world * flops * args.steps / (t_ms * 1e-3) / 1e12
+
+    # ---- per-kernel durations (events around each kernel, same rotation)
+    nk = max(20, min(args.steps, 400))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nk)]
+    torch.cuda._sleep(100_000_000)             # host enqueues all launches before the GPU reaches them
+    for i in range(nk):
+        s = sets[i % nsets]
+        ev[i][0].record(stream)
+        B.svdq_quantize_act("nvfp4", s["x"], s["w"]["inv_smooth"], s["w"]["lora_down"], s_a,
+                            s["w"]["weight_scale_f"], out=(s["codes"], s["scales"], s["lora"]), stream=stream)
+        ev[i][1].record(stream)
+        B.svdq_w4a4_gemm("nvfp4", s["codes"], s["scales"], s["lora"], s["w"], alpha, bias=bias, y=s["y"],
+                         stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_s1 = sum(e[0].elapsed_time(e[1]) for e in ev) / nk * 1e3    # us
+    t_s2 = sum(e[1].elapsed_time(e[2]) for e in ev) / nk * 1e3
+
+    # ---- end to end through the public API with host buffers
+    x_host = inp.x_bits.view(np.int16)
+    hx = torch.from_numpy(x_host).view(torch.bfloat16).pin_memory()
+    hy = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    ke = max(3, min(50, args.steps // 10))
+    for i in range(2):
+        s = sets[i % nsets]
+        s["x"].copy_(hx, non_blocking=True)
+        layer(i)
+        hy.copy_(s["y"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(ke):
+        s = sets[i % nsets]
+        s["x"].copy_(hx, non_blocking=True)
+        layer(i)
+        hy.copy_(s["y"], non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_value = world * flops * ke / (te_ms * 1e-3) / 1e12
+
+    peaks, peak_src = _measured_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    s2_tflops = flops / (t_s2 * 1e-6) / 1e12
+    s1_bytes = M * K * 2 + M * K // 2 + M * K // 16 + M * 64 * 2 + K * 4 + 32 * K * 2
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": f"DiT MLP up-projection, svdq_w4a4_linear NVFP4 r32: x bf16 [{M},{K}] -> "
+                               f"y bf16 [{M},{N}] (quantize + low-rank down-proj, FP4 GEMM + low-rank up-proj "
+                               f"+ bias)",
+                   "M": M, "K": K, "N": N, "rank": 32, "global_batch_tokens": M * world,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"rotating {nsets} weight/activation/output sets ({nsets * per_set / 2**20:.0f} MiB "
+                         f"> 126 MiB L2)"},
+        "pct_of_fp4_peak": {"spec_dense_9pf": round(100 * value / world / FP4_SPEC_DENSE_TFLOPS, 2),
+                            f"{peak_src}_bf16x4": round(100 * value / world / fp4_peak, 2)},
+        "roofline": {"kernel": "gemm_nvfp4 (S2)", "bound": "tensor", "achieved": round(s2_tflops, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(s2_tflops / fp4_peak, 4),
+                     "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} "
+                                    f"(nominal fp4:bf16 dense ratio)",
+                     "traffic": None},
+        "kernels": {"quantize_act_us": round(t_s1, 2), "gemm_nvfp4_us": round(t_s2, 2),
+                    "quantize_act_gbs": round(s1_bytes / (t_s1 * 1e-6) / 1e9, 1),
+                    "quantize_act_hbm_frac": round(s1_bytes / (t_s1 * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": int(M * K * 2),
+                "d2h_bytes_per_step": int(M * N * 2), "steps": ke},
+        "gpu_launches": 2 * args.steps,
+        "graph": f"{G} steps per CUDA graph, {reps} replays + {rem} eager",
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        tf, dt, rows = time_oracle(case, inp, steps=3, warmup=1, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOPS", "cores": _cpu_threads(), "kind": "oracle",
+                               "sample": f"{rows} of {M} rows per step, 3 steps (numpy fp64 oracle, weight "
+                                         f"pack and dequantization offline)",
+                               "s_per_step": round(dt, 3)}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import workloads as wl
+        case = wl.SVDQ_CASES[WORKLOAD]
+        inp = wl.make_svdq_inputs(case)
+        budget = max(30.0, min(150.0, 1.0 * (args.steps + args.warmup)))
+        tf, dt, rows = time_oracle(case, inp, args.steps, args.warmup, budget)
+        cores = _cpu_threads()
+        sample = f"{rows} of {case.M} rows per step (numpy fp64 oracle; weight pack and dequantization offline)"
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(tf, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"DiT MLP up-projection {case.M}x{case.K}->{case.N} NVFP4 r32"},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(tf, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -198,6 +198,8 @@ def svdq_quantize_act(precision, x, inv_smooth, lora_down, act_scale, weight_sca
     p = _prec(precision)
     _dev_bf16(x, "x")
     M, K = x.shape
+    if act_scale_bytes(p, M, K) < 0 or M <= 0:
+        raise SvdqError(2, f"unsupported shape M={M} K={K}")
     if out is None:
         dev = x.device
         out = (torch.empty((M, K // 2), dtype=torch.uint8, device=dev),

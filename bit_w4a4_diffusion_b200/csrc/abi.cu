@@ -195,8 +195,8 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
                        128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
                        256, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 32, 32,
-                       CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
+                       CU_TENSOR_MAP_SWIZZLE_32B);
   if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
   GemmNvfp4Params p{};
   p.M = M;

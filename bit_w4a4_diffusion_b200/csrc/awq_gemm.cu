@@ -43,9 +43,10 @@ SVDQ_DEV void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint3
 // Byte j of `lo_nib` / `hi_nib` (the low / high nibbles of four code bytes)
 // -> bf16x2 {128 + lo, 128 + hi} - {128 + z, 128 + z} = {lo - z, hi - z}.
 SVDQ_DEV uint32_t dequant_pair(uint32_t lo_nib, uint32_t hi_nib, int j, uint32_t zz) {
+  // Selector nibble n picks result byte n: byte 0 <- lo_j, byte 2 <- hi_j.
   const uint32_t sel = (uint32_t)j | ((uint32_t)(4 + j) << 8);
-  uint32_t v = __byte_perm(lo_nib, hi_nib, sel);  // byte0 = lo_j, byte1 = hi_j
-  v = (v & 0xFFu) | ((v & 0xFF00u) << 8) | 0x43004300u;
+  uint32_t v = __byte_perm(lo_nib, hi_nib, sel);
+  v = (v & 0x00FF00FFu) | 0x43004300u;
   __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&v), *reinterpret_cast<const __nv_bfloat162*>(&zz));
   return *reinterpret_cast<uint32_t*>(&r);
 }

@@ -19,6 +19,11 @@
 //   warps 2..5  epilogue (TMEM -> registers -> bf16 -> swizzled smem -> TMA store)
 // Pipeline: STAGES-deep smem ring of K=256 slices; slot 0 of every tile is the
 // low-rank slice (u' in the A slot, [L2^T|L2^T] in the B slot).
+// Tensor memory (512 columns): two 256-column fp32 accumulators at columns 0
+// and 192, overlapping in [192, 256), and the block scales in [448, 512).
+// Consecutive tiles alternate accumulators; the epilogue drains the shared 64
+// columns first and then releases the accumulator, so the next tile's MMAs
+// run while the epilogue finishes the remaining 192 columns.
 // Every mbarrier wait is bounded; on timeout the kernel records a status code,
 // drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -32,19 +37,21 @@ namespace {
 
 constexpr int BM = 128, BN = 256;
 constexpr int BK_BYTES = 128;  // 256 fp4 elements
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK_BYTES;            // 16 KB
 constexpr int B_BYTES = BN * BK_BYTES;            // 32 KB
 constexpr int SFA_BYTES = 4 * 512;                // 4 K64 chunks x 128 rows
 constexpr int SFB_BYTES = 2 * 4 * 512;            // 2 row blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int EPI_WARPS = 4;
-constexpr int EPI_CHUNK = 32;                          // columns per TMEM load / store
-constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;      // 32 rows x 64 B
+constexpr int EPI_CHUNK = 16;                          // columns per TMEM load / store
+constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;      // 32 rows x 32 B
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
 constexpr int NUM_THREADS = 64 + EPI_WARPS * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_ACC = 0, TMEM_SFA = 256, TMEM_SFB = 272;
+constexpr int ACC_STRIDE = 192;                        // accumulator b starts at column b * 192
+constexpr int ACC_OVERLAP = 2 * 256 - (ACC_STRIDE + 256); // 64 shared columns
+constexpr int TMEM_SFA = 448, TMEM_SFB = 464;
 // Limit for the exit-path waits on this CTA's own in-flight copies and MMAs,
 // which always complete; independent of the caller's timeout.
 constexpr unsigned long long kDrainLimitNs = 2000000000ull;
@@ -177,8 +184,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      const uint32_t d_tmem = tmem + TMEM_ACC;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const uint32_t d_tmem = tmem + (uint32_t)((it & 1) * ACC_STRIDE);
         if (!mbar_wait(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
           ok = false;
           break;
@@ -231,64 +239,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;
     uint32_t acc_phase = 0;
-    int chunk_seq = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    int chunk_seq = 0, it = 0;
+    constexpr int NCH = BN / EPI_CHUNK;
+    constexpr int NOVL = ACC_OVERLAP / EPI_CHUNK;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM;
       const int n0 = (tile / tiles_m) * BN;
+      const int b = it & 1;
       const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
       tc_fence_after();
-      for (int cc = 0; cc < BN / EPI_CHUNK; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + TMEM_ACC + ((uint32_t)(32 * q) << 16) + cc * EPI_CHUNK, r);
+      const uint32_t acc_col = (uint32_t)(b * ACC_STRIDE);
+      for (int i = 0; i < NCH; ++i) {
+        // The columns shared with the other accumulator go first: the last
+        // 64 of accumulator 0, the first 64 of accumulator 1.
+        const int cc = b == 0 ? (i + NCH - NOVL) % NCH : i;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + acc_col + cc * EPI_CHUNK, r);
         tmem_ld_wait();
-        if (cc == BN / EPI_CHUNK - 1) {
+        if (i == NOVL - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
         }
         const int ncol = n0 + cc * EPI_CHUNK;
-        float bias[32];
+        float bias[16];
         if (p.bias != nullptr && ncol < p.N) {
           const uint4* bp = reinterpret_cast<const uint4*>(p.bias + ncol);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 2; ++v) {
             const uint4 w = __ldg(bp + v);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              bias[8 * v + 2 * i] = __uint_as_float(ws[i] << 16);
-              bias[8 * v + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+            for (int k = 0; k < 4; ++k) {
+              bias[8 * v + 2 * k] = __uint_as_float(ws[k] << 16);
+              bias[8 * v + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
             }
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) bias[i] = 0.f;
+          for (int k = 0; k < 16; ++k) bias[k] = 0.f;
         }
-        uint32_t packed[16];
+        uint32_t packed[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * i]), bias[2 * i]);
-          const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * i + 1]), bias[2 * i + 1]);
+        for (int k = 0; k < 8; ++k) {
+          const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * k]), bias[2 * k]);
+          const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * k + 1]), bias[2 * k + 1]);
           __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-          packed[i] = *reinterpret_cast<uint32_t*>(&h);
+          packed[k] = *reinterpret_cast<uint32_t*>(&h);
         }
         uint8_t* buf = buf0 + (chunk_seq & 1) * EPI_BUF_BYTES;
         // The TMA store issued two chunks ago read this buffer; wait for it.
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
-        uint8_t* row = buf + lane * 64;
+        uint8_t* row = buf + lane * 32;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int pj = j ^ ((lane >> 1) & 3);  // 64-byte swizzle
+        for (int j = 0; j < 2; ++j) {
+          const int pj = j ^ ((lane >> 2) & 1);  // 32-byte swizzle
           *reinterpret_cast<uint4*>(row + pj * 16) =
               make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && ncol < p.N && m0 + 32 * q < p.M) {
-          tma_store_2d(&tm_y, ncol, m0 + 32 * q, smem_u32(buf));
-        }
+        if (lane == 0 && ncol < p.N && m0 + 32 * q < p.M) tma_store_2d(&tm_y, ncol, m0 + 32 * q, smem_u32(buf));
         if (lane == 0) bulk_commit();
         ++chunk_seq;
       }

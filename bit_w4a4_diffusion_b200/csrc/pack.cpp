@@ -32,8 +32,6 @@ uint16_t f32_to_bf16_rne(float f) {
   return (uint16_t)((u + 0x7FFFu + lsb) >> 16);  // finite inputs only
 }
 
-float bf16_round(float f) { return bf16_to_f32(f32_to_bf16_rne(f)); }
-
 // Non-negative finite fp32 -> E4M3 byte, round to nearest even, saturating at
 // 448 (0x7E).  Works on the fp32 fields directly.
 uint8_t e4m3_rne_sat(float t) {
@@ -169,12 +167,13 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
         for (int i = 0; i < 16; ++i) a = std::max(a, std::fabs(row[16 * g + i]));
         const uint8_t sb = e4m3_rne_sat(a / six_s);
         const float d = e4m3_to_f32(sb) * s;
+        const float rd = d != 0.f ? 1.0f / d : 0.f;
         scales[sf_offset(n, g, K)] = sb;
         for (int i = 0; i < 16; i += 2) {
           uint8_t c0 = 0, c1 = 0;
           if (d != 0.f) {
-            c0 = e2m1_rne_sat(row[16 * g + i] / d);
-            c1 = e2m1_rne_sat(row[16 * g + i + 1] / d);
+            c0 = e2m1_rne_sat(row[16 * g + i] * rd);
+            c1 = e2m1_rne_sat(row[16 * g + i + 1] * rd);
           }
           codes[(size_t)n * (K / 2) + (16 * g + i) / 2] = (uint8_t)(c0 | (c1 << 4));
         }
@@ -191,12 +190,13 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
         for (int i = 0; i < 64; ++i) a = std::max(a, std::fabs(row[64 * g + i]));
         const uint16_t scb = f32_to_bf16_rne(a / 7.0f);
         const float sc = bf16_to_f32(scb);
+        const float rs = sc != 0.f ? 1.0f / sc : 0.f;
         sc16[(size_t)g * np + n] = scb;
         for (int i = 0; i < 64; i += 2) {
           int q0 = 0, q1 = 0;
           if (sc != 0.f) {
-            q0 = std::clamp((int)std::nearbyint(row[64 * g + i] / sc), -8, 7);
-            q1 = std::clamp((int)std::nearbyint(row[64 * g + i + 1] / sc), -8, 7);
+            q0 = std::clamp((int)std::nearbyint(row[64 * g + i] * rs), -8, 7);
+            q1 = std::clamp((int)std::nearbyint(row[64 * g + i + 1] * rs), -8, 7);
           }
           codes[(size_t)n * (K / 2) + (64 * g + i) / 2] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
         }

@@ -10,8 +10,8 @@
 //
 //   x_hat = fp32(x) * inv_lambda                       (one fp32 multiply)
 //   NVFP4: per 16 along K, a = max|x_hat|, t = a / (6 s_a), sb = E4M3(t),
-//          d = float(sb) * s_a, code = E2M1(x_hat / d)   (RNE, satfinite)
-//   INT4:  per 64 along K, sc = bf16(a / 7), q = clamp(rint(x_hat / sc), -8, 7)
+//          d = float(sb) * s_a, code = E2M1(x_hat * fp32(1/d))  (RNE, satfinite)
+//   INT4:  per 64 along K, sc = bf16(a / 7), q = clamp(rint(x_hat * fp32(1/sc)), -8, 7)
 //   u     = x_hat * L1 on tensor cores (mma.sync bf16, fp32 accumulate), with
 //           x_hat split into bf16 hi + lo so that u carries ~16 mantissa bits
 //   lora_act[m] = [hi(u * c) | lo(u * c)]  (bf16, 2r values per row), with
@@ -39,7 +39,7 @@ namespace {
 constexpr int S1_ROWS = 16;
 constexpr int S1_WARPS = 8;
 constexpr int S1_THREADS = S1_WARPS * 32;
-constexpr int S1_UNROLL = 4;
+constexpr int S1_UNROLL = 2;
 
 SVDQ_DEV float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
@@ -80,7 +80,7 @@ SVDQ_DEV size_t sf_offset(int row, int group, int K) {
 }
 
 template <bool kNvfp4>
-__global__ void __launch_bounds__(S1_THREADS) quantize_act_kernel(QuantActParams p) {
+__global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int row0 = blockIdx.x * S1_ROWS + g;
@@ -115,9 +115,9 @@ __global__ void __launch_bounds__(S1_THREADS) quantize_act_kernel(QuantActParams
         const int blk = b0 + u * S1_WARPS * step + h;
         const bool live = (h < step) && blk < nblk;
         const int k = blk * 32 + 8 * c;
-        xa[2 * u + h] = (live && ok0) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row0 * K + k))
+        xa[2 * u + h] = (live && ok0) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)row0 * K + k))
                                       : make_uint4(0, 0, 0, 0);
-        xb[2 * u + h] = (live && ok1) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)row1 * K + k))
+        xb[2 * u + h] = (live && ok1) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)row1 * K + k))
                                       : make_uint4(0, 0, 0, 0);
       }
     }
@@ -156,21 +156,22 @@ __global__ void __launch_bounds__(S1_THREADS) quantize_act_kernel(QuantActParams
         const uint32_t sb1 = cvt_e4m3(__fdiv_rn(a1, six_s));
         const float d0 = __fmul_rn(e4m3_value(sb0), s_a);
         const float d1 = __fmul_rn(e4m3_value(sb1), s_a);
+        const float r0 = __frcp_rn(d0), r1 = __frcp_rn(d1);
         uint32_t w0 = 0, w1 = 0;
         if (d0 != 0.f) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            w0 |= cvt_e2m1x2(__fdiv_rn(v0[0][2 * i], d0), __fdiv_rn(v0[0][2 * i + 1], d0)) << (8 * i);
+            w0 |= cvt_e2m1x2(__fmul_rn(v0[0][2 * i], r0), __fmul_rn(v0[0][2 * i + 1], r0)) << (8 * i);
         }
         if (d1 != 0.f) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            w1 |= cvt_e2m1x2(__fdiv_rn(v1[0][2 * i], d1), __fdiv_rn(v1[0][2 * i + 1], d1)) << (8 * i);
+            w1 |= cvt_e2m1x2(__fmul_rn(v1[0][2 * i], r1), __fmul_rn(v1[0][2 * i + 1], r1)) << (8 * i);
         }
         const int k = blk_first * 32 + 8 * c;
         uint8_t* codes = p.act_codes;
-        if (ok0) *reinterpret_cast<uint32_t*>(codes + (size_t)row0 * (K / 2) + k / 2) = w0;
-        if (ok1) *reinterpret_cast<uint32_t*>(codes + (size_t)row1 * (K / 2) + k / 2) = w1;
+        if (ok0) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row0 * (K / 2) + k / 2), w0);
+        if (ok1) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row1 * (K / 2) + k / 2), w1);
         if ((c & 1) == 0) {
           const int grp = k >> 4;
           p.act_scales[sf_offset(row0, grp, K)] = (uint8_t)sb0;  // rows >= M get 0 (zero input)
@@ -193,14 +194,15 @@ __global__ void __launch_bounds__(S1_THREADS) quantize_act_kernel(QuantActParams
         const __nv_bfloat16 sc0 = __float2bfloat16_rn(__fdiv_rn(a0, 7.0f));
         const __nv_bfloat16 sc1 = __float2bfloat16_rn(__fdiv_rn(a1, 7.0f));
         const float f0 = __bfloat162float(sc0), f1 = __bfloat162float(sc1);
+        const float r0 = __frcp_rn(f0), r1 = __frcp_rn(f1);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t w0 = 0, w1 = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             int q0 = 0, q1 = 0;
-            if (f0 != 0.f) q0 = max(-8, min(7, __float2int_rn(__fdiv_rn(v0[h][i], f0))));
-            if (f1 != 0.f) q1 = max(-8, min(7, __float2int_rn(__fdiv_rn(v1[h][i], f1))));
+            if (f0 != 0.f) q0 = max(-8, min(7, __float2int_rn(__fmul_rn(v0[h][i], r0))));
+            if (f1 != 0.f) q1 = max(-8, min(7, __float2int_rn(__fmul_rn(v1[h][i], r1))));
             w0 |= (uint32_t)(q0 & 0xF) << (4 * i);
             w1 |= (uint32_t)(q1 & 0xF) << (4 * i);
           }

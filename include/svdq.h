@@ -96,8 +96,8 @@ int svdq_scales_from_rowmajor(int rows, int K, const uint8_t* rowmajor, uint8_t*
  *            (products and sum in fp64, one rounding to fp32);
  *   NVFP4: s_w = amax|R| / 2688 (1 if R == 0); per 16 along k:
  *          a = max|v|, sb = E4M3_rn_sat(a / fp32(6 s_w)), d = float(sb)*s_w,
- *          code = E2M1_rn_sat(v / d) (sign kept), all codes 0 when d == 0.
- *   INT4:  per 64 along k: sc = bf16(a / 7), q = clamp(rint(v / sc), -8, 7).
+ *          code = E2M1_rn_sat(v * fp32(1/d)) (sign kept), all codes 0 when d == 0.
+ *   INT4:  per 64 along k: sc = bf16(a / 7), q = clamp(rint(v * fp32(1/sc)), -8, 7).
  * Inputs (host): W bf16 [N,K]; smooth fp32 [K] (lambda, > 0); L1 bf16 [K,r];
  * L2 bf16 [r,N].  Outputs (host, caller-allocated):
  *   codes      [N, K/2] bytes

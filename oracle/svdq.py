@@ -96,8 +96,11 @@ def nvfp4_quantize(V, s):
     """NVFP4 quantization of the rows of V along the last axis, group 16.
 
     Per group of 16: a = max|v|; t = a / fp32(6*s); sb = E4M3(t) (RNE,
-    satfinite); d = fp32(float(sb) * s); code = E2M1(v / d) (RNE, satfinite,
-    sign kept).  A group with d == 0 gets all-zero (+0) codes.
+    satfinite); d = fp32(float(sb) * s); r = fp32(1 / d);
+    code = E2M1(fp32(v * r)) (RNE, satfinite, sign kept).  A group with
+    d == 0 gets all-zero (+0) codes.  The block scale is applied as a multiply
+    by its fp32 reciprocal (one division per block): the pages fix no
+    operation order, and this is the form a streaming quantizer uses.
 
     Returns (codes uint8 [rows, K] one code per element, scales uint8 [rows, K/16]).
     """
@@ -112,7 +115,8 @@ def nvfp4_quantize(V, s):
     sb = e4m3_encode_nonneg(t)
     d = (e4m3_decode(sb).astype(np.float32) * s).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = (G / d[:, :, None]).astype(np.float32)
+        r = (np.float32(1.0) / d).astype(np.float32)
+        ratio = (G * r[:, :, None]).astype(np.float32)
     ratio = np.where(d[:, :, None] == 0, np.float32(0.0), ratio)
     codes = e2m1_encode(ratio)
     codes = np.where(d[:, :, None] == 0, np.uint8(0), codes).astype(np.uint8)
@@ -134,8 +138,9 @@ def int4_quantize(V):
     """Symmetric signed INT4 quantization along the last axis, group 64.
 
     Per group: a = max|v|; sc = bf16(a / 7) (fp32 divide, then bf16 RNE);
-    q = clamp(rint(v / sc), -8, 7) with an fp32 divide and ties to even;
-    q = 0 where sc == 0.  Returns (q int8 [rows, K], sc float32 [rows, K/64]
+    r = fp32(1 / sc); q = clamp(rint(fp32(v * r)), -8, 7) with ties to even;
+    q = 0 where sc == 0 (the scale applied as a reciprocal multiply, as for
+    NVFP4).  Returns (q int8 [rows, K], sc float32 [rows, K/64]
     holding bf16 values).
     """
     V = np.asarray(V, dtype=np.float32)
@@ -145,7 +150,8 @@ def int4_quantize(V):
     a = np.max(np.abs(G), axis=2)
     sc = bf16_round((a / np.float32(7.0)).astype(np.float32))
     with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = (G / sc[:, :, None]).astype(np.float32)
+        r = (np.float32(1.0) / sc).astype(np.float32)
+        ratio = (G * r[:, :, None]).astype(np.float32)
     q = np.rint(np.where(sc[:, :, None] == 0, np.float32(0.0), ratio))
     q = np.clip(q, -8, 7).astype(np.int8)
     return q.reshape(rows, K), sc.astype(np.float32)
