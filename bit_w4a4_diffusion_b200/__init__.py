@@ -32,7 +32,7 @@ class SvdqError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
-                          "(run `python -m bit_w4a4_diffusion_b200.build`)")
+                          "(run `python bit_w4a4_diffusion_b200/build.py`)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, LL, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_ulonglong
     sig = {

@@ -1,7 +1,8 @@
 """Build the CUDA library ``libsvdq_b200.so`` in-tree with nvcc (sm_100a).
 
-Usage: ``python -m bit_w4a4_diffusion_b200.build`` (or ``build()`` from
-``__graft_entry__``).  Objects are rebuilt only when a source or header is
+Usage: ``python bit_w4a4_diffusion_b200/build.py [-v]`` (or ``build()`` from
+``__graft_entry__``); run it by path -- importing the package loads the
+library this script produces.  Objects are rebuilt only when a source or header is
 newer than the object.  Cross-compiles without a GPU.
 """
 import os

@@ -19,8 +19,9 @@
 //           and c = 1 for INT4.
 //
 // Mapping.  A CTA owns 16 rows; each warp walks 32-wide K blocks.  Lane
-// (g = lane / 4, c = lane % 4) loads 8 consecutive elements of rows g and g+8
-// at k = kb + 8c with 16-byte loads; these 16 values are exactly the lane's
+// (g = lane / 4, c = lane % 4) copies 8 consecutive elements of rows g and g+8
+// at k = kb + 8c (16-byte cp.async into its own shared-memory ring slots,
+// three blocks ahead of the compute); these 16 values are exactly the lane's
 // mma.m16n8k16 A fragments for two K=16 steps under the k-permutation
 // logical(s, 2c + {0,1}, 2c + 8 + {0,1}) <-> kb + 8c + 4s + {0,1,2,3}; the B
 // fragments are loaded with the same permutation from L1^T, so the dot
@@ -39,7 +40,6 @@ namespace {
 constexpr int S1_ROWS = 16;
 constexpr int S1_WARPS = 8;
 constexpr int S1_THREADS = S1_WARPS * 32;
-constexpr int S1_UNROLL = 2;
 
 SVDQ_DEV float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
@@ -79,21 +79,62 @@ SVDQ_DEV size_t sf_offset(int row, int group, int K) {
   return ((size_t)(row >> 7) * kchunks + (group >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
 }
 
+// Per-thread asynchronous prefetch: each lane copies the x and L1^T fragments
+// it will consume into its own slots of a shared-memory ring (no other thread
+// reads them, so no block-wide synchronisation is needed), PREFETCH units ahead.
+SVDQ_DEV void cp_async16(void* smem_dst, const void* gsrc, bool pred) {
+  const uint32_t d = smem_u32(smem_dst);
+  const int n = pred ? 16 : 0;  // src-size 0 -> the 16 bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n) : "memory");
+}
+SVDQ_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+SVDQ_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int S1_PREFETCH = 3;
+// Slot contents per 32-wide block: x rows g and g+8 (2 x 16 B), then the four
+// L1^T fragments of the lane (4 x 16 B).
+constexpr int S1_SLOT_U4 = 6;
+
 template <bool kNvfp4>
 __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActParams p) {
+  constexpr int STEP = kNvfp4 ? 1 : 2;  // 32-blocks per unit (INT4 group = 64)
+  extern __shared__ uint4 s1_ring[];     // [PREFETCH][STEP][SLOT_U4][THREADS]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int row0 = blockIdx.x * S1_ROWS + g;
   const int row1 = row0 + 8;
   const bool ok0 = row0 < p.M, ok1 = row1 < p.M;
   const int K = p.K;
-  const int nblk = K / 32;
+  const int nunits = K / (32 * STEP);
 
   const uint16_t* __restrict__ x = p.x;
   const uint16_t* __restrict__ l1t = p.lora_down;  // [r][K]
   const float* __restrict__ inv_lam = p.inv_smooth;
 
-  // u accumulators: 4 n8 tiles (rank 32) x 4 fp32.
+  auto slot = [&](int ring, int h, int q) -> uint4* {
+    return s1_ring + (((ring * STEP + h) * S1_SLOT_U4 + q) * S1_THREADS + threadIdx.x);
+  };
+  // Units of this warp: unit u = warp + S1_WARPS * i.
+  const int my_units = nunits > warp ? (nunits - warp + S1_WARPS - 1) / S1_WARPS : 0;
+  auto prefetch = [&](int i) {
+    if (i < my_units) {
+      const int unit = warp + S1_WARPS * i;
+      const int ring = i % S1_PREFETCH;
+#pragma unroll
+      for (int h = 0; h < STEP; ++h) {
+        const int k = (unit * STEP + h) * 32 + 8 * c;
+        cp_async16(slot(ring, h, 0), x + (size_t)(ok0 ? row0 : 0) * K + k, ok0);
+        cp_async16(slot(ring, h, 1), x + (size_t)(ok1 ? row1 : 0) * K + k, ok1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_async16(slot(ring, h, 2 + j), l1t + (size_t)(8 * j + g) * K + k, true);
+      }
+    }
+    cp_async_commit();  // always commit (possibly empty) so group counting stays uniform
+  };
+
   float acc[4][4];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
@@ -103,164 +144,148 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
   const float s_a = p.act_scale;
   const float six_s = __fmul_rn(6.0f, s_a);
 
-  // INT4 needs a 64-group = two consecutive 32-blocks: a warp then walks pairs.
-  const int step = kNvfp4 ? 1 : 2;
-  for (int b0 = warp * step; b0 < nblk; b0 += S1_WARPS * step * S1_UNROLL) {
-    uint4 xa[S1_UNROLL * 2], xb[S1_UNROLL * 2];
-    // Issue all loads of this round first (memory-level parallelism).
 #pragma unroll
-    for (int u = 0; u < S1_UNROLL; ++u) {
+  for (int i = 0; i < S1_PREFETCH - 1; ++i) prefetch(i);
+
+  for (int i = 0; i < my_units; ++i) {
+    prefetch(i + S1_PREFETCH - 1);
+    cp_async_wait<S1_PREFETCH - 1>();
+    const int unit = warp + S1_WARPS * i;
+    const int ring = i % S1_PREFETCH;
+    float v0[STEP][8], v1[STEP][8];  // x_hat for rows g, g+8
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int blk = b0 + u * S1_WARPS * step + h;
-        const bool live = (h < step) && blk < nblk;
-        const int k = blk * 32 + 8 * c;
-        xa[2 * u + h] = (live && ok0) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)row0 * K + k))
-                                      : make_uint4(0, 0, 0, 0);
-        xb[2 * u + h] = (live && ok1) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)row1 * K + k))
-                                      : make_uint4(0, 0, 0, 0);
+    for (int h = 0; h < STEP; ++h) {
+      const int k = (unit * STEP + h) * 32 + 8 * c;
+      const float4 il0 = __ldg(reinterpret_cast<const float4*>(inv_lam + k));
+      const float4 il1 = __ldg(reinterpret_cast<const float4*>(inv_lam + k + 4));
+      const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+      unpack8(*slot(ring, h, 0), v0[h]);
+      unpack8(*slot(ring, h, 1), v1[h]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        v0[h][e] = __fmul_rn(v0[h][e], il[e]);
+        v1[h][e] = __fmul_rn(v1[h][e], il[e]);
       }
     }
-#pragma unroll
-    for (int u = 0; u < S1_UNROLL; ++u) {
-      const int blk_first = b0 + u * S1_WARPS * step;
-      if (blk_first >= nblk) break;
-      float v0[2][8], v1[2][8];  // x_hat for rows g, g+8; h = which 32-block
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h >= step) break;
-        const int k = (blk_first + h) * 32 + 8 * c;
-        const float4 il0 = __ldg(reinterpret_cast<const float4*>(inv_lam + k));
-        const float4 il1 = __ldg(reinterpret_cast<const float4*>(inv_lam + k + 4));
-        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
-        unpack8(xa[2 * u + h], v0[h]);
-        unpack8(xb[2 * u + h], v1[h]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v0[h][i] = __fmul_rn(v0[h][i], il[i]);
-          v1[h][i] = __fmul_rn(v1[h][i], il[i]);
-        }
-      }
 
-      // ---------------- quantize ----------------
-      if constexpr (kNvfp4) {
-        float a0 = 0.f, a1 = 0.f;
+    // ---------------- quantize ----------------
+    if constexpr (kNvfp4) {
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          a0 = fmaxf(a0, fabsf(v0[0][i]));
-          a1 = fmaxf(a1, fabsf(v1[0][i]));
+      for (int e = 0; e < 8; ++e) {
+        a0 = fmaxf(a0, fabsf(v0[0][e]));
+        a1 = fmaxf(a1, fabsf(v1[0][e]));
+      }
+      a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+      a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+      const uint32_t sb0 = cvt_e4m3(__fdiv_rn(a0, six_s));
+      const uint32_t sb1 = cvt_e4m3(__fdiv_rn(a1, six_s));
+      const float d0 = __fmul_rn(e4m3_value(sb0), s_a);
+      const float d1 = __fmul_rn(e4m3_value(sb1), s_a);
+      const float r0 = __frcp_rn(d0), r1 = __frcp_rn(d1);
+      uint32_t w0 = 0, w1 = 0;
+      if (d0 != 0.f) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w0 |= cvt_e2m1x2(__fmul_rn(v0[0][2 * e], r0), __fmul_rn(v0[0][2 * e + 1], r0)) << (8 * e);
+      }
+      if (d1 != 0.f) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w1 |= cvt_e2m1x2(__fmul_rn(v1[0][2 * e], r1), __fmul_rn(v1[0][2 * e + 1], r1)) << (8 * e);
+      }
+      const int k = unit * 32 + 8 * c;
+      uint8_t* codes = p.act_codes;
+      if (ok0) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row0 * (K / 2) + k / 2), w0);
+      if (ok1) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row1 * (K / 2) + k / 2), w1);
+      if ((c & 1) == 0) {
+        const int grp = k >> 4;
+        p.act_scales[sf_offset(row0, grp, K)] = (uint8_t)sb0;  // rows >= M get 0 (zero input)
+        p.act_scales[sf_offset(row1, grp, K)] = (uint8_t)sb1;
+      }
+    } else {
+      // INT4: group of 64 = lanes c=0..3 over two 32-blocks.
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int h = 0; h < STEP; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          a0 = fmaxf(a0, fabsf(v0[h][e]));
+          a1 = fmaxf(a1, fabsf(v1[h][e]));
         }
-        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
-        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-        const uint32_t sb0 = cvt_e4m3(__fdiv_rn(a0, six_s));
-        const uint32_t sb1 = cvt_e4m3(__fdiv_rn(a1, six_s));
-        const float d0 = __fmul_rn(e4m3_value(sb0), s_a);
-        const float d1 = __fmul_rn(e4m3_value(sb1), s_a);
-        const float r0 = __frcp_rn(d0), r1 = __frcp_rn(d1);
+      a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
+      a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+      a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
+      a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
+      const __nv_bfloat16 sc0 = __float2bfloat16_rn(__fdiv_rn(a0, 7.0f));
+      const __nv_bfloat16 sc1 = __float2bfloat16_rn(__fdiv_rn(a1, 7.0f));
+      const float f0 = __bfloat162float(sc0), f1 = __bfloat162float(sc1);
+      const float r0 = __frcp_rn(f0), r1 = __frcp_rn(f1);
+#pragma unroll
+      for (int h = 0; h < STEP; ++h) {
         uint32_t w0 = 0, w1 = 0;
-        if (d0 != 0.f) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w0 |= cvt_e2m1x2(__fmul_rn(v0[0][2 * i], r0), __fmul_rn(v0[0][2 * i + 1], r0)) << (8 * i);
+        for (int e = 0; e < 8; ++e) {
+          int q0 = 0, q1 = 0;
+          if (f0 != 0.f) q0 = max(-8, min(7, __float2int_rn(__fmul_rn(v0[h][e], r0))));
+          if (f1 != 0.f) q1 = max(-8, min(7, __float2int_rn(__fmul_rn(v1[h][e], r1))));
+          w0 |= (uint32_t)(q0 & 0xF) << (4 * e);
+          w1 |= (uint32_t)(q1 & 0xF) << (4 * e);
         }
-        if (d1 != 0.f) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w1 |= cvt_e2m1x2(__fmul_rn(v1[0][2 * i], r1), __fmul_rn(v1[0][2 * i + 1], r1)) << (8 * i);
-        }
-        const int k = blk_first * 32 + 8 * c;
-        uint8_t* codes = p.act_codes;
-        if (ok0) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row0 * (K / 2) + k / 2), w0);
-        if (ok1) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row1 * (K / 2) + k / 2), w1);
-        if ((c & 1) == 0) {
-          const int grp = k >> 4;
-          p.act_scales[sf_offset(row0, grp, K)] = (uint8_t)sb0;  // rows >= M get 0 (zero input)
-          p.act_scales[sf_offset(row1, grp, K)] = (uint8_t)sb1;
-        }
-      } else {
-        // INT4: group of 64 = lanes c=0..3 over two 32-blocks.
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            a0 = fmaxf(a0, fabsf(v0[h][i]));
-            a1 = fmaxf(a1, fabsf(v1[h][i]));
-          }
-        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
-        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 2));
-        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
-        const __nv_bfloat16 sc0 = __float2bfloat16_rn(__fdiv_rn(a0, 7.0f));
-        const __nv_bfloat16 sc1 = __float2bfloat16_rn(__fdiv_rn(a1, 7.0f));
-        const float f0 = __bfloat162float(sc0), f1 = __bfloat162float(sc1);
-        const float r0 = __frcp_rn(f0), r1 = __frcp_rn(f1);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            int q0 = 0, q1 = 0;
-            if (f0 != 0.f) q0 = max(-8, min(7, __float2int_rn(__fmul_rn(v0[h][i], r0))));
-            if (f1 != 0.f) q1 = max(-8, min(7, __float2int_rn(__fmul_rn(v1[h][i], r1))));
-            w0 |= (uint32_t)(q0 & 0xF) << (4 * i);
-            w1 |= (uint32_t)(q1 & 0xF) << (4 * i);
-          }
-          const int k = (blk_first + h) * 32 + 8 * c;
-          if (ok0) *reinterpret_cast<uint32_t*>(p.act_codes + (size_t)row0 * (K / 2) + k / 2) = w0;
-          if (ok1) *reinterpret_cast<uint32_t*>(p.act_codes + (size_t)row1 * (K / 2) + k / 2) = w1;
-        }
-        if (c == 0) {
-          // INT4 activation scales: bf16, group-major [K/64][M_pad].
-          const int grp = blk_first >> 1;
-          uint16_t* sc = reinterpret_cast<uint16_t*>(p.act_scales);
-          sc[(size_t)grp * p.M_pad + row0] = __bfloat16_as_ushort(sc0);
-          sc[(size_t)grp * p.M_pad + row1] = __bfloat16_as_ushort(sc1);
-        }
+        const int k = (unit * STEP + h) * 32 + 8 * c;
+        if (ok0) __stcs(reinterpret_cast<unsigned int*>(p.act_codes + (size_t)row0 * (K / 2) + k / 2), w0);
+        if (ok1) __stcs(reinterpret_cast<unsigned int*>(p.act_codes + (size_t)row1 * (K / 2) + k / 2), w1);
       }
+      if (c == 0) {
+        // INT4 activation scales: bf16, group-major [K/64][M_pad].
+        uint16_t* sc = reinterpret_cast<uint16_t*>(p.act_scales);
+        sc[(size_t)unit * p.M_pad + row0] = __bfloat16_as_ushort(sc0);
+        sc[(size_t)unit * p.M_pad + row1] = __bfloat16_as_ushort(sc1);
+      }
+    }
 
-      // ---------------- low-rank down-projection ----------------
+    // ---------------- low-rank down-projection ----------------
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h >= step) break;
-        const int k = (blk_first + h) * 32 + 8 * c;
-        uint32_t ahi[2][4], alo[2][4];
+    for (int h = 0; h < STEP; ++h) {
+      uint32_t ahi[2][4], alo[2][4];
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          float h0[4], h1[4], l0[4], l1[4];
+      for (int st = 0; st < 2; ++st) {
+        float h0[4], h1[4], l0[4], l1[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            h0[i] = bf16_round_f(v0[h][4 * s + i]);
-            h1[i] = bf16_round_f(v1[h][4 * s + i]);
-            l0[i] = __fsub_rn(v0[h][4 * s + i], h0[i]);
-            l1[i] = __fsub_rn(v1[h][4 * s + i], h1[i]);
-          }
-          ahi[s][0] = pack_bf16x2(h0[0], h0[1]);
-          ahi[s][1] = pack_bf16x2(h1[0], h1[1]);
-          ahi[s][2] = pack_bf16x2(h0[2], h0[3]);
-          ahi[s][3] = pack_bf16x2(h1[2], h1[3]);
-          alo[s][0] = pack_bf16x2(l0[0], l0[1]);
-          alo[s][1] = pack_bf16x2(l1[0], l1[1]);
-          alo[s][2] = pack_bf16x2(l0[2], l0[3]);
-          alo[s][3] = pack_bf16x2(l1[2], l1[3]);
+        for (int e = 0; e < 4; ++e) {
+          h0[e] = bf16_round_f(v0[h][4 * st + e]);
+          h1[e] = bf16_round_f(v1[h][4 * st + e]);
+          l0[e] = __fsub_rn(v0[h][4 * st + e], h0[e]);
+          l1[e] = __fsub_rn(v1[h][4 * st + e], h1[e]);
         }
+        ahi[st][0] = pack_bf16x2(h0[0], h0[1]);
+        ahi[st][1] = pack_bf16x2(h1[0], h1[1]);
+        ahi[st][2] = pack_bf16x2(h0[2], h0[3]);
+        ahi[st][3] = pack_bf16x2(h1[2], h1[3]);
+        alo[st][0] = pack_bf16x2(l0[0], l0[1]);
+        alo[st][1] = pack_bf16x2(l1[0], l1[1]);
+        alo[st][2] = pack_bf16x2(l0[2], l0[3]);
+        alo[st][3] = pack_bf16x2(l1[2], l1[3]);
+      }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 bw = __ldg(reinterpret_cast<const uint4*>(l1t + (size_t)(8 * j + g) * K + k));
-          mma_bf16_16816(acc[j], ahi[0], bw.x, bw.y);
-          mma_bf16_16816(acc[j], alo[0], bw.x, bw.y);
-          mma_bf16_16816(acc[j], ahi[1], bw.z, bw.w);
-          mma_bf16_16816(acc[j], alo[1], bw.z, bw.w);
-        }
+      for (int j = 0; j < 4; ++j) {
+        const uint4 bw = *slot(ring, h, 2 + j);
+        mma_bf16_16816(acc[j], ahi[0], bw.x, bw.y);
+        mma_bf16_16816(acc[j], alo[0], bw.x, bw.y);
+        mma_bf16_16816(acc[j], ahi[1], bw.z, bw.w);
+        mma_bf16_16816(acc[j], alo[1], bw.z, bw.w);
       }
     }
   }
+  cp_async_wait<0>();
 
   // Let the GEMM that consumes these outputs start its prologue.
   pdl_launch_dependents();
 
   // ---------------- cross-warp reduction of u, then the bf16 hi/lo fold ----
-  __shared__ float red[S1_WARPS][S1_ROWS][33];
+  // (reuses the prefetch ring: every copy has landed and been consumed)
+  __syncthreads();
+  float(*red)[S1_ROWS][33] = reinterpret_cast<float(*)[S1_ROWS][33]>(s1_ring);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     red[warp][g][8 * j + 2 * c] = acc[j][0];
@@ -291,10 +316,17 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream) {
   const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
   dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS);
-  if (nvfp4)
-    quantize_act_kernel<true><<<grid, S1_THREADS, 0, stream>>>(p);
-  else
-    quantize_act_kernel<false><<<grid, S1_THREADS, 0, stream>>>(p);
+  const size_t ring_bytes = (size_t)S1_PREFETCH * (nvfp4 ? 1 : 2) * S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
+  cudaError_t e;
+  if (nvfp4) {
+    e = cudaFuncSetAttribute(quantize_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ring_bytes);
+    if (e != cudaSuccess) return e;
+    quantize_act_kernel<true><<<grid, S1_THREADS, ring_bytes, stream>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(quantize_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ring_bytes);
+    if (e != cudaSuccess) return e;
+    quantize_act_kernel<false><<<grid, S1_THREADS, ring_bytes, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 
