@@ -50,6 +50,8 @@ def _load():
         "svdq_quantize_act": (I, [I, I, I, I, P, P, P, F, F, P, P, P, P]),
         "svdq_w4a4_gemm": (I, [I, I, I, I, I, P, P, P, P, P, P, P, F, P, P, P]),
         "svdq_w4a4_linear": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, LL, P, P]),
+        "svdq_noalloc_scratch_bytes": (LL, []),
+        "svdq_w4a4_linear_noalloc": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, P]),
         "awq_pack_weights": (I, [I, I, P, P, P, P]),
         "awq_w4a16_linear": (I, [I, I, I, P, P, P, P, P, P, P]),
     }
@@ -240,6 +242,23 @@ def svdq_w4a4_linear(precision, x, w, act_scale, bias=None, y=None, workspace=No
                                 float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), wscale, _ptr(w["lora_up"]),
                                 _ptr(bias), _ptr(y), _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                 _stream(stream)))
+    return y
+
+
+def svdq_w4a4_linear_noalloc(precision, x, w, act_scale, bias=None, y=None, dev_status=None, stream=None):
+    """svdq_w4a4_linear without a workspace: the quantized activations live in
+    the library's built-in device scratch (see include/svdq.h)."""
+    p = _prec(precision)
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    N, rank = w["N"], w["rank"]
+    assert K == w["K"]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib.svdq_w4a4_linear_noalloc(p, M, N, K, rank, _ptr(x), _ptr(w["inv_smooth"]), _ptr(w["lora_down"]),
+                                        float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), w["weight_scale_f"],
+                                        _ptr(w["lora_up"]), _ptr(bias), _ptr(y), _ptr(dev_status),
+                                        _stream(stream)))
     return y
 
 

@@ -1,0 +1,80 @@
+// svdq_w4a4_linear_noalloc: the whole W4A4 layer without a caller-provided
+// workspace and without allocating any device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they run the layer:
+// code running while a CUDA graph is being captured on a stream the caller
+// does not control, plugins handed only input and output pointers by a host
+// framework that owns every allocation, or allocators that forbid extra
+// device allocations after start-up.  For them the quantized activations that
+// svdq_w4a4_linear keeps in its workspace live instead in a file-scope device
+// array of SVDQ_NOALLOC_SCRATCH_BYTES that the CUDA driver sets aside when it
+// loads this module; every GPU that loads the library holds it until the
+// process exits.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "svdq.h"
+#include "svdq_internal.h"
+
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SVDQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address must come
+// from cudaGetSymbolAddress, once per device, with that device current.
+int scratch_for_current_device(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return svdq::record_error(SVDQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return svdq::record_error(SVDQ_ERR_UNSUPPORTED_DEVICE, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return svdq::record_error(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+long long svdq_noalloc_scratch_bytes(void) { return (long long)SVDQ_NOALLOC_SCRATCH_BYTES; }
+
+int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
+                             const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
+                             float weight_scale, const void* lora_up, const void* bias, void* y, int* dev_status,
+                             void* stream) {
+  const long long need = svdq_workspace_bytes(precision, M, K, rank);
+  if (need < 0) {
+    // Let the regular entry point produce its precise shape / argument error.
+    return svdq_w4a4_linear(precision, M, N, K, rank, x, inv_smooth, lora_down, act_scale, w_codes, w_scales,
+                            weight_scale, lora_up, bias, y, nullptr, 0, dev_status, stream);
+  }
+  if (need > (long long)SVDQ_NOALLOC_SCRATCH_BYTES)
+    return svdq::record_error(SVDQ_ERR_UNSUPPORTED_SHAPE,
+                              "M=%d K=%d needs %lld bytes of scratch; the built-in scratch holds %lld bytes "
+                              "(use svdq_w4a4_linear with a workspace)",
+                              M, K, need, (long long)SVDQ_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (int s = scratch_for_current_device(&scratch)) return s;
+  // Nothing in the scratch has to start at zero: the quantize kernel writes
+  // every byte the GEMM then reads (all code rows < M, every scale row up to
+  // the 256-row padding, every low-rank row < M) before the GEMM starts.
+  return svdq_w4a4_linear(precision, M, N, K, rank, x, inv_smooth, lora_down, act_scale, w_codes, w_scales,
+                          weight_scale, lora_up, bias, y, scratch, need, dev_status, stream);
+}
+
+}  // extern "C"

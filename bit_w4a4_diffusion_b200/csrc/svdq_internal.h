@@ -58,6 +58,9 @@ struct AwqParams {
 
 cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream);
 
+// Records a message for svdq_last_error() and returns `status`.
+int record_error(int status, const char* fmt, ...);
+
 // Tensor-map encoding through the driver entry point (no libcuda link needed).
 bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);

@@ -152,6 +152,36 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
                      float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
                      long long workspace_bytes, int* dev_status, void* stream);
 
+/* ------------------------------------------------------------------ no-allocation variant
+ * svdq_w4a4_linear_noalloc: the same layer as svdq_w4a4_linear, for callers
+ * that cannot allocate device memory when they run it -- code recorded into a
+ * CUDA graph on a stream someone else captures, plugins that receive only
+ * input and output pointers from a host framework that owns all memory, or
+ * allocators that forbid allocations after start-up.  The pages have no
+ * counterpart to this entry point; it is a deployment convenience.
+ * Instead of a caller workspace it uses a file-scope device array of
+ * SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB) that the CUDA driver reserves on every
+ * GPU that loads the library, until the process exits.  It never calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *  - Limit: svdq_workspace_bytes(precision, M, K, rank) must not exceed
+ *    SVDQ_NOALLOC_SCRATCH_BYTES (e.g. M = 4096 tokens up to K = 12288);
+ *    larger shapes return SVDQ_ERR_UNSUPPORTED_SHAPE with a message.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (once per device, with that device current); make
+ *    that first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents;
+ *    nothing in it needs to start at zero.  Calls whose kernels overlap on
+ *    the GPU (different streams without ordering, or concurrent threads)
+ *    race on it: order them on one stream.
+ * Arguments, layouts and errors are those of svdq_w4a4_linear without the
+ * workspace pair. */
+#define SVDQ_NOALLOC_SCRATCH_BYTES (32ll << 20)
+long long svdq_noalloc_scratch_bytes(void);
+int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
+                             const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
+                             float weight_scale, const void* lora_up, const void* bias, void* y, int* dev_status,
+                             void* stream);
+
 /* ------------------------------------------------------------------ AWQ W4A16
  * "Nunchaku Lite" docs, "Supported quantization types" table: awq_w4a16,
  * int4, group size 64 -- an INT4 weight-only AWQ-style kernel for the
