@@ -319,6 +319,8 @@ def run_gpu(args, rank, world, local_rank):
         "graph": f"{G} steps per CUDA graph, {reps} replays + {rem} eager",
         "clocks": sampler.summary(),
     }
+    if not args.no_rows:
+        out["rows"] = measure_rows(B, wl, dev, peaks)
     if rank == 0 and not args.no_cpu_baseline:
         tf, dt, rows = time_oracle(case, inp, steps=3, warmup=1, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOPS", "cores": _cpu_threads(), "kind": "oracle",
@@ -326,6 +328,61 @@ def run_gpu(args, rank, world, local_rank):
                                          f"pack and dequantization offline)",
                                "s_per_step": round(dt, 3)}
     return out
+
+
+def _event_time_us(torch, fns, iters):
+    """Median device time (us) of fns[i % len(fns)]() over `iters` launches,
+    enqueued behind a GPU sleep so host launch cost never shows."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for i in range(3):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(50_000_000)
+    for i, (a, b) in enumerate(ev):
+        a.record()
+        fns[i % len(fns)]()
+        b.record()
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) * 1e3 for a, b in ev]))
+
+
+def measure_rows(B, wl, dev, peaks):
+    """The other hot-path rows at their workload sizes: AWQ W4A16 (HBM GB/s)
+    and the INT4 W4A4 layer over the token sweep (TOPS).  Weight sets rotate
+    so that no launch finds its weights in L2."""
+    import torch
+    rows = {}
+    awq = {}
+    for M in wl.AWQ_MS:
+        a = wl.make_awq_inputs(M)
+        pk = B.awq_pack_weights(a.W_bits)
+        nset = 6  # 6 x 30.5 MB > 126 MB L2
+        ws = [B.to_device(pk, dev) for _ in range(nset)]
+        x = B.bits_to_bf16(a.x_bits, dev)
+        ys = [torch.empty((M, a.N), dtype=torch.bfloat16, device=dev) for _ in range(nset)]
+        fns = [lambda i=i: B.awq_w4a16_linear(x, ws[i], y=ys[i]) for i in range(nset)]
+        t = _event_time_us(torch, fns, 60)
+        byts = a.N * a.K // 2 + a.N * a.K // 64 * 2 + a.N * a.K // 128 + M * a.K * 2 + M * a.N * 2
+        awq[f"M={M}"] = {"us": round(t, 2), "GB/s": round(byts / t / 1e3, 1),
+                         "hbm_frac": round(byts / t / 1e3 / peaks["hbm_gbs"], 3)}
+        del ws, ys
+    rows["awq_w4a16 N=18432 K=3072"] = awq
+    int4 = {}
+    for M in (1024, 2048, 4096, 8192):
+        c = wl.SVDQ_CASES[f"int4_m{M}"]
+        inp = wl.make_svdq_inputs(c)
+        pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+        nset = 4
+        ws = [B.to_device(pk, dev) for _ in range(nset)]
+        x = B.bits_to_bf16(inp.x_bits, dev)
+        ys = [torch.empty((M, c.N), dtype=torch.bfloat16, device=dev) for _ in range(nset)]
+        wsp = torch.empty(B.workspace_bytes("int4", M, c.K), dtype=torch.uint8, device=dev)
+        fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=ys[i], workspace=wsp) for i in range(nset)]
+        t = _event_time_us(torch, fns, 40)
+        int4[f"M={M}"] = {"us": round(t, 2), "TOPS": round(2.0 * M * c.N * c.K / t / 1e6, 1)}
+        del ws, ys
+    rows["svdq_w4a4 int4 K=N=3072 (quantize + i8 GEMM)"] = int4
+    return rows
 
 
 def main():
@@ -336,6 +393,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ row measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -226,8 +226,36 @@ static int check_gemm_args(int precision, int M, int N, int K, int rank) {
   if (K % 256 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of 256", K);
   if (N % 128 != 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d must be a multiple of 128", N);
   if (rank != SVDQ_RANK) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank=%d; this build supports rank %d", rank, SVDQ_RANK);
-  if (precision == SVDQ_INT4) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "INT4 W4A4 GEMM is not available in this build");
   return SVDQ_OK;
+}
+
+static int gemm_int4_impl(int M, int N, int K, const void* act_codes, const void* act_scales, const void* lora_act,
+                          const void* w_codes, const void* w_scales, const void* lora_up, const void* bias, void* y,
+                          int* dev_status, cudaStream_t stream, bool pdl, int sms) {
+  GemmInt4Tmaps t;
+  bool ok = true;
+  ok &= encode_tmap_2d(&t.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_codes, K / 2, M, K / 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_tmap_2d(&t.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_tmap_2d(&t.la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_act, 2 * SVDQ_RANK, M, 2 * SVDQ_RANK * 2, 64,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
+  GemmInt4Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.M_pad = (int)round_up(M, 256);
+  p.N_pad = (int)round_up(N, 256);
+  p.act_scales = static_cast<const uint16_t*>(act_scales);
+  p.w_scales = static_cast<const uint16_t*>(w_scales);
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.y = static_cast<uint16_t*>(y);
+  p.dev_status = dev_status;
+  p.timeout_ns = svdq_timeout_ns();
+  return check_cuda(launch_gemm_int4(p, t, sms, stream, pdl), "gemm_int4 launch");
 }
 
 int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
@@ -239,9 +267,12 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
   if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lora_act) || !aligned16(w_codes) ||
       !aligned16(w_scales) || !aligned16(lora_up) || !aligned16(y) || (bias && !aligned16(bias)))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
-  if (!(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
+  if (precision == SVDQ_NVFP4 && !(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (precision == SVDQ_INT4)
+    return gemm_int4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, y, dev_status,
+                          static_cast<cudaStream_t>(stream), false, sms);
   return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, y,
                          dev_status, static_cast<cudaStream_t>(stream), false, sms);
 }
@@ -269,6 +300,9 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (precision == SVDQ_INT4)
+    return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
+                          static_cast<cudaStream_t>(stream), true, sms);
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), true, sms);
 }

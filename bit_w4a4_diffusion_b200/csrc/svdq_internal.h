@@ -46,6 +46,23 @@ struct GemmTmaps {
 cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                               bool pdl);
 
+struct GemmInt4Params {
+  int M, N, K, M_pad, N_pad;
+  const uint16_t* act_scales;  // bf16 [K/64][M_pad]
+  const uint16_t* w_scales;    // bf16 [K/64][N_pad]
+  const uint16_t* bias;        // bf16 [N] or null
+  uint16_t* y;                 // bf16 [M, N]
+  int* dev_status;
+  unsigned long long timeout_ns;
+};
+
+struct GemmInt4Tmaps {
+  CUtensorMap a, b, la, lb;
+};
+
+cudaError_t launch_gemm_int4(const GemmInt4Params& p, const GemmInt4Tmaps& t, int num_sms, cudaStream_t stream,
+                             bool pdl);
+
 struct AwqParams {
   int M, N, K;
   const uint16_t* x;       // bf16 [M, K]

@@ -132,10 +132,13 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
 /* svdq_w4a4_gemm: the 4-bit GEMM with the low-rank up-projection and bias in
  * its epilogue (the engine's fused "up-projection + 4-bit GEMM" kernel), on
  * already-quantized activations:
- *   y = bf16( alpha * ( sum_k deq(a) deq(w) + lora_act . lora_up^T ) + bias )
- * with alpha = s_a * s_w (NVFP4).  Device inputs as produced by
- * svdq_quantize_act and svdq_pack_weights; bias bf16 [N] or NULL; output y
- * bf16 [M,N].  Shapes: M >= 1, N % 128 == 0, K % 256 == 0. */
+ *   NVFP4: y = bf16( alpha * ( sum_k deq(a) deq(w) + lora_act . lora_up^T ) + bias )
+ *          with alpha = s_a * s_w;
+ *   INT4:  y = bf16( sum_g sa[m,g] sw[n,g] sum_{k in g} qa qw + lora_act . lora_up^T + bias ),
+ *          the 64-group sums exact in int32 (alpha is ignored).
+ * Device inputs as produced by svdq_quantize_act and svdq_pack_weights; bias
+ * bf16 [N] or NULL; output y bf16 [M,N].
+ * Shapes: M >= 1, N % 128 == 0, K % 256 == 0. */
 int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
                    const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
                    const void* bias, float alpha, void* y, int* dev_status, void* stream);
