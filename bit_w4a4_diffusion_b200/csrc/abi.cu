@@ -169,9 +169,11 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
   if (!aligned16(x) || !aligned16(inv_smooth) || !aligned16(lora_down) || !aligned16(act_codes) ||
       !aligned16(lora_act) || !aligned16(act_scales))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
-  if (precision == SVDQ_NVFP4 && !(act_scale > 0.f && weight_scale > 0.f))
-    return fail(SVDQ_ERR_INVALID_ARG, "NVFP4 tensor scales must be positive (act %g, weight %g)", act_scale,
-                weight_scale);
+  // Scales from 2^-100 up keep every block reciprocal 1/(E4M3 * s) finite in fp32.
+  if (precision == SVDQ_NVFP4 && !(act_scale >= 0x1p-100f && weight_scale >= 0x1p-100f &&
+                                   act_scale < 0x1p100f && weight_scale < 0x1p100f))
+    return fail(SVDQ_ERR_INVALID_ARG, "NVFP4 tensor scales must lie in [2^-100, 2^100) (act %g, weight %g)",
+                act_scale, weight_scale);
   int sms = 0;
   if (int s = check_device(&sms)) return s;
   QuantActParams p{};

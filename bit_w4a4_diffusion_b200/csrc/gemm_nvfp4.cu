@@ -13,17 +13,22 @@
 // so the rank-r branch is four extra bf16 MMAs into the same TMEM accumulator
 // and the epilogue is a single fused multiply-add per element.
 //
-// Structure: persistent CTAs, one 128x256 output tile at a time, 6 warps:
+// Structure: persistent CTAs, one 128x256 output tile at a time, 9 warps:
 //   warp 0      TMA producer (A/B codes by tensor TMA, scales by bulk copy)
-//   warp 1      tcgen05 issuer (scale copies smem->TMEM, MMAs, commits)
+//   warp 1      MMA issuer (MMAs and commits only)
 //   warps 2..5  epilogue (TMEM -> registers -> bf16 -> swizzled smem -> TMA store)
+//   warps 6..8  block-scale copies smem -> TMEM (SFA, SFB rows 0-127, SFB rows
+//               128-255): each tcgen05.cp holds its issuing thread for tens of
+//               cycles, so the 12 copies of a K slice are spread over three
+//               threads that run ahead of the MMA warp into a second buffer.
 // Pipeline: STAGES-deep smem ring of K=256 slices; slot 0 of every tile is the
 // low-rank slice (u' in the A slot, [L2^T|L2^T] in the B slot).
 // Tensor memory (512 columns): two 256-column fp32 accumulators at columns 0
-// and 192, overlapping in [192, 256), and the block scales in [448, 512).
-// Consecutive tiles alternate accumulators; the epilogue drains the shared 64
-// columns first and then releases the accumulator, so the next tile's MMAs
-// run while the epilogue finishes the remaining 192 columns.
+// and 160, overlapping in [160, 256), and two 48-column block-scale buffers
+// in [416, 512) (K slices alternate buffers).  Consecutive tiles alternate
+// accumulators; the epilogue drains the shared 96 columns first and then
+// releases the accumulator, so the next tile's MMAs run while the epilogue
+// finishes the other 160 columns.
 // Every mbarrier wait is bounded; on timeout the kernel records a status code,
 // drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -47,11 +52,16 @@ constexpr int EPI_WARPS = 4;
 constexpr int EPI_CHUNK = 16;                          // columns per TMEM load / store
 constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;      // 32 rows x 32 B
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
-constexpr int NUM_THREADS = 64 + EPI_WARPS * 32;
+constexpr int SF_WARPS = 3;
+constexpr int SF_WARP0 = 2 + EPI_WARPS;                 // first scale-copy warp
+constexpr int NUM_THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_STRIDE = 192;                        // accumulator b starts at column b * 192
-constexpr int ACC_OVERLAP = 2 * 256 - (ACC_STRIDE + 256); // 64 shared columns
-constexpr int TMEM_SFA = 448, TMEM_SFB = 464;
+constexpr int ACC_STRIDE = 160;                        // accumulator b starts at column b * 160
+constexpr int ACC_OVERLAP = 2 * 256 - (ACC_STRIDE + 256); // 96 shared columns
+// Block scales of one K slice: SFA 4 MMAs x 4 columns, SFB 4 MMAs x 8 columns.
+constexpr int SF_COLS = 48;
+constexpr int TMEM_SF0 = ACC_STRIDE + 256;             // buffers at 416 and 464
+constexpr int TMEM_SFA_OFF = 0, TMEM_SFB_OFF = 16;
 // Limit for the exit-path waits on this CTA's own in-flight copies and MMAs,
 // which always complete; independent of the caller's timeout.
 constexpr unsigned long long kDrainLimitNs = 2000000000ull;
@@ -61,7 +71,10 @@ struct SmemCtl {
   uint64_t empty[STAGES];
   uint64_t acc_full;
   uint64_t acc_empty;
+  uint64_t sf_full[2];   // scale-copy warps -> MMA (copies of one K slice landed)
+  uint64_t sf_empty[2];  // MMA -> scale-copy warps (MMAs reading the buffer done)
   uint64_t drain;
+  uint64_t sf_drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -102,7 +115,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(smem_u32(&ctl->acc_full), 1);
     mbar_init(smem_u32(&ctl->acc_empty), EPI_WARPS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->sf_full[b]), SF_WARPS);
+      mbar_init(smem_u32(&ctl->sf_empty[b]), 1);
+    }
     mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->sf_drain), SF_WARPS);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,6 +203,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       int it = 0;
+      uint32_t ks = 0;  // K slices computed so far (selects the scale buffer)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const uint32_t d_tmem = tmem + (uint32_t)((it & 1) * ACC_STRIDE);
         if (!mbar_wait(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
@@ -205,18 +224,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < 4; ++j)
               mma_bf16(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
           } else {
-            const uint32_t ssfa = sb + B_BYTES;
-            const uint32_t ssfb = ssfa + SFA_BYTES;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tmem_cp_32x128_warpx4(tmem + TMEM_SFA + 4 * j, sf_desc(ssfa + 512 * j));
-              tmem_cp_32x128_warpx4(tmem + TMEM_SFB + 8 * j, sf_desc(ssfb + 512 * j));
-              tmem_cp_32x128_warpx4(tmem + TMEM_SFB + 8 * j + 4, sf_desc(ssfb + SFA_BYTES + 512 * j));
+            const uint32_t buf = ks & 1;
+            if (!mbar_wait(smem_u32(&ctl->sf_full[buf]), (ks >> 1) & 1, wctx, kDevTimeoutMma)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t sf = tmem + TMEM_SF0 + buf * SF_COLS;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               mma_nvfp4(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_NVFP4,
-                        tmem + TMEM_SFA + 4 * j, tmem + TMEM_SFB + 8 * j, 1u);
+                        sf + TMEM_SFA_OFF + 4 * j, sf + TMEM_SFB_OFF + 8 * j, 1u);
+            tc_commit(smem_u32(&ctl->sf_empty[buf]));
+            ++ks;
           }
           tc_commit(smem_u32(&ctl->empty[stage]));
           if (++stage == STAGES) {
@@ -234,76 +254,131 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
     }
+  } else if (warp >= SF_WARP0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ scale copies
+      // Warp SF_WARP0 + w copies part w of every K slice's block scales:
+      // w = 0: SFA (4 copies), w = 1 / 2: SFB rows 0-127 / 128-255 (4 each).
+      const int w = warp - SF_WARP0;
+      int stage = 0;
+      uint32_t phase = 0, ks = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kt = 0; kt < slices; ++kt) {
+          if (kt > 0) {
+            const uint32_t buf = ks & 1;
+            // The MMAs of the K slice two back read this buffer; wait for them.
+            if (ks >= 2 && !mbar_wait(smem_u32(&ctl->sf_empty[buf]), ((ks - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t ssfa = smem_u32(stage_base + stage * STAGE_BYTES) + A_BYTES + B_BYTES;
+            const uint32_t src = w == 0 ? ssfa : ssfa + SFA_BYTES * w;
+            const uint32_t dst = tmem + TMEM_SF0 + buf * SF_COLS + (w == 0 ? TMEM_SFA_OFF : TMEM_SFB_OFF + 4 * (w - 1));
+            const uint32_t col_step = w == 0 ? 4 : 8;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_cp_32x128_warpx4(dst + col_step * j, sf_desc(src + 512 * j));
+            tc_commit(smem_u32(&ctl->sf_full[buf]));
+            ++ks;
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      tc_commit(smem_u32(&ctl->sf_drain));
+      volatile int never = 0;
+      WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
+      mbar_wait(smem_u32(&ctl->sf_drain), 0, drain_ctx, kDevTimeoutDrain);
+    }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile.
+    // Columns are read from TMEM 32 at a time, the next chunk's load in flight
+    // while the current one is converted; the tile's bias is loaded once (lane
+    // l holds columns 8l..8l+7) and broadcast by shuffles.
+    const int q = warp & 3;
     uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;
     uint32_t acc_phase = 0;
     int chunk_seq = 0, it = 0;
-    constexpr int NCH = BN / EPI_CHUNK;
-    constexpr int NOVL = ACC_OVERLAP / EPI_CHUNK;
+    constexpr int LDC = 32;                    // columns per TMEM load
+    constexpr int NCH = BN / LDC;
+    constexpr int NOVL = ACC_OVERLAP / LDC;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM;
       const int n0 = (tile / tiles_m) * BN;
       const int b = it & 1;
+      uint4 bias8 = make_uint4(0, 0, 0, 0);
+      if (p.bias != nullptr && n0 + 8 * lane < p.N) bias8 = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
       const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
       tc_fence_after();
-      const uint32_t acc_col = (uint32_t)(b * ACC_STRIDE);
+      const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+      // The columns shared with the other accumulator go first: the last 64
+      // of accumulator 0, the first 64 of accumulator 1.
+      auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NOVL) % NCH : i; };
+      uint32_t rbuf[2][32];
+      tmem_ld_32x32b_x32(acc_base + chunk_col(0) * LDC, rbuf[0]);
+      tmem_ld_wait(rbuf[0]);
+#pragma unroll
       for (int i = 0; i < NCH; ++i) {
-        // The columns shared with the other accumulator go first: the last
-        // 64 of accumulator 0, the first 64 of accumulator 1.
-        const int cc = b == 0 ? (i + NCH - NOVL) % NCH : i;
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + acc_col + cc * EPI_CHUNK, r);
-        tmem_ld_wait();
+        uint32_t(&r)[32] = rbuf[i & 1];
+        if (i + 1 < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + 1) * LDC, rbuf[(i + 1) & 1]);
         if (i == NOVL - 1) {
+          // The shared columns (chunks 0 .. NOVL-1) are all in registers once
+          // this wait returns; release the accumulator to the MMA warp.
+          tmem_ld_wait(rbuf[(i + 1) & 1]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
         }
-        const int ncol = n0 + cc * EPI_CHUNK;
-        float bias[16];
-        if (p.bias != nullptr && ncol < p.N) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + ncol);
+        const int cc = chunk_col(i);
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const uint4 w = __ldg(bp + v);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int hh = 0; hh < 2; ++hh) {      // two 16-column halves per TMEM load
+          const int ncol = n0 + cc * LDC + hh * EPI_CHUNK;
+          const int src_lane = (cc * LDC + hh * EPI_CHUNK) / 8;  // lanes src_lane, src_lane + 1
+          uint32_t bw[8];
+          bw[0] = __shfl_sync(0xffffffffu, bias8.x, src_lane);
+          bw[1] = __shfl_sync(0xffffffffu, bias8.y, src_lane);
+          bw[2] = __shfl_sync(0xffffffffu, bias8.z, src_lane);
+          bw[3] = __shfl_sync(0xffffffffu, bias8.w, src_lane);
+          bw[4] = __shfl_sync(0xffffffffu, bias8.x, src_lane + 1);
+          bw[5] = __shfl_sync(0xffffffffu, bias8.y, src_lane + 1);
+          bw[6] = __shfl_sync(0xffffffffu, bias8.z, src_lane + 1);
+          bw[7] = __shfl_sync(0xffffffffu, bias8.w, src_lane + 1);
+          uint32_t packed[8];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              bias[8 * v + 2 * k] = __uint_as_float(ws[k] << 16);
-              bias[8 * v + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
-            }
+          for (int k = 0; k < 8; ++k) {
+            const float b0 = __uint_as_float(bw[k] << 16), b1 = __uint_as_float(bw[k] & 0xFFFF0000u);
+            const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[hh * 16 + 2 * k]), b0);
+            const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[hh * 16 + 2 * k + 1]), b1);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+            packed[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
-        } else {
+          uint8_t* buf = buf0 + (chunk_seq & 1) * EPI_BUF_BYTES;
+          // The TMA store issued two halves ago read this buffer; wait for it.
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          uint8_t* row = buf + lane * 32;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) bias[k] = 0.f;
+          for (int j = 0; j < 2; ++j) {
+            const int pj = j ^ ((lane >> 2) & 1);  // 32-byte swizzle
+            *reinterpret_cast<uint4*>(row + pj * 16) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && ncol < p.N && m0 + 32 * q < p.M) tma_store_2d(&tm_y, ncol, m0 + 32 * q, smem_u32(buf));
+          if (lane == 0) bulk_commit();
+          ++chunk_seq;
         }
-        uint32_t packed[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * k]), bias[2 * k]);
-          const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[2 * k + 1]), bias[2 * k + 1]);
-          __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-          packed[k] = *reinterpret_cast<uint32_t*>(&h);
-        }
-        uint8_t* buf = buf0 + (chunk_seq & 1) * EPI_BUF_BYTES;
-        // The TMA store issued two chunks ago read this buffer; wait for it.
-        if (lane == 0) bulk_wait_read<1>();
-        __syncwarp();
-        uint8_t* row = buf + lane * 32;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int pj = j ^ ((lane >> 2) & 1);  // 32-byte swizzle
-          *reinterpret_cast<uint4*>(row + pj * 16) =
-              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && ncol < p.N && m0 + 32 * q < p.M) tma_store_2d(&tm_y, ncol, m0 + 32 * q, smem_u32(buf));
-        if (lane == 0) bulk_commit();
-        ++chunk_seq;
+        if (i + 1 < NCH && i != NOVL - 1) tmem_ld_wait(rbuf[(i + 1) & 1]);
       }
       acc_phase ^= 1;
     }

@@ -160,12 +160,13 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
     const float s = amax > 0.f ? amax / 2688.0f : 1.0f;
     *weight_scale = s;
     const float six_s = 6.0f * s;
+    const float inv_six_s = 1.0f / six_s;
     parallel_rows(N, [&](int n) {
       const float* row = &R[(size_t)n * K];
       for (int g = 0; g < K / 16; ++g) {
         float a = 0.f;
         for (int i = 0; i < 16; ++i) a = std::max(a, std::fabs(row[16 * g + i]));
-        const uint8_t sb = e4m3_rne_sat(a / six_s);
+        const uint8_t sb = e4m3_rne_sat(a * inv_six_s);
         const float d = e4m3_to_f32(sb) * s;
         const float rd = d != 0.f ? 1.0f / d : 0.f;
         scales[sf_offset(n, g, K)] = sb;

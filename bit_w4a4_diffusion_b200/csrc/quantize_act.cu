@@ -9,7 +9,7 @@
 // the same fusion is one HBM-bound pass over x:
 //
 //   x_hat = fp32(x) * inv_lambda                       (one fp32 multiply)
-//   NVFP4: per 16 along K, a = max|x_hat|, t = a / (6 s_a), sb = E4M3(t),
+//   NVFP4: per 16 along K, a = max|x_hat|, t = a * fp32(1/(6 s_a)), sb = E4M3(t),
 //          d = float(sb) * s_a, code = E2M1(x_hat * fp32(1/d))  (RNE, satfinite)
 //   INT4:  per 64 along K, sc = bf16(a / 7), q = clamp(rint(x_hat * fp32(1/sc)), -8, 7)
 //   u     = x_hat * L1 on tensor cores (mma.sync bf16, fp32 accumulate), with
@@ -18,10 +18,10 @@
 //           c = 1 / (s_a s_w) for NVFP4 (folds the GEMM's per-tensor scale)
 //           and c = 1 for INT4.
 //
-// Mapping.  A CTA owns 16 rows; each warp walks 32-wide K blocks.  Lane
-// (g = lane / 4, c = lane % 4) copies 8 consecutive elements of rows g and g+8
-// at k = kb + 8c (16-byte cp.async into its own shared-memory ring slots,
-// three blocks ahead of the compute); these 16 values are exactly the lane's
+// Mapping.  A CTA owns 16 rows; its 16 warps walk interleaved 32-wide K
+// blocks.  Lane (g = lane / 4, c = lane % 4) copies 8 consecutive elements of
+// rows g and g+8 at k = kb + 8c (16-byte cp.async into its own shared-memory
+// ring slots, ahead of the compute); these 16 values are exactly the lane's
 // mma.m16n8k16 A fragments for two K=16 steps under the k-permutation
 // logical(s, 2c + {0,1}, 2c + 8 + {0,1}) <-> kb + 8c + 4s + {0,1,2,3}; the B
 // fragments are loaded with the same permutation from L1^T, so the dot
@@ -38,15 +38,8 @@ namespace svdq {
 namespace {
 
 constexpr int S1_ROWS = 16;
-constexpr int S1_WARPS = 8;
+constexpr int S1_WARPS = 16;
 constexpr int S1_THREADS = S1_WARPS * 32;
-
-SVDQ_DEV float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
-
-SVDQ_DEV uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
-  return *reinterpret_cast<uint32_t*>(&p);
-}
 
 SVDQ_DEV void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -65,11 +58,40 @@ SVDQ_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Eight fp32 (already multiplied by the block's reciprocal scale) -> eight
+// E2M1 codes in one 32-bit word, element 2i in the low nibble of byte i.
+SVDQ_DEV uint32_t cvt_e2m1x8(const float (&v)[8], float r) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(__fmul_rn(v[0], r)), "f"(__fmul_rn(v[1], r)), "f"(__fmul_rn(v[2], r)), "f"(__fmul_rn(v[3], r)),
+        "f"(__fmul_rn(v[4], r)), "f"(__fmul_rn(v[5], r)), "f"(__fmul_rn(v[6], r)), "f"(__fmul_rn(v[7], r)));
+  return out;
+}
+
+// x (fp32) -> the bf16 pair words of (hi, lo) with hi = bf16(x), lo = bf16(x - hi),
+// for two elements at a time: hi2 / lo2 hold (e0 in the low half, e1 high).
+SVDQ_DEV void split_bf16x2(float e0, float e1, uint32_t& hi2, uint32_t& lo2) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
+  const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
+  const float h0 = __uint_as_float(hb << 16), h1 = __uint_as_float(hb & 0xFFFF0000u);
+  __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(e0, h0), __fsub_rn(e1, h1));
+  hi2 = hb;
+  lo2 = *reinterpret_cast<uint32_t*>(&l);
+}
+
 // Exact E4M3 (non-negative) byte -> fp32 from the format fields.
 SVDQ_DEV float e4m3_value(uint32_t b) {
-  const uint32_t e = (b >> 3) & 0xF, m = b & 7;
-  if (e == 0) return __uint2float_rn(m) * 0.001953125f;  // m * 2^-9
-  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(b & 0xFF)));
+  float f;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"((unsigned short)(h2 & 0xFFFF)));
+  return f;  // E4M3 -> f16 -> f32 are both exact
 }
 
 // Byte offset of scale (row, group) in the tiled NVFP4 scale layout:
@@ -93,7 +115,7 @@ SVDQ_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-constexpr int S1_PREFETCH = 3;
+constexpr int S1_PREFETCH = 2;
 // Slot contents per 32-wide block: x rows g and g+8 (2 x 16 B), then the four
 // L1^T fragments of the lane (4 x 16 B).
 constexpr int S1_SLOT_U4 = 6;
@@ -142,7 +164,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
     for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
 
   const float s_a = p.act_scale;
-  const float six_s = __fmul_rn(6.0f, s_a);
+  const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, s_a));
 
 #pragma unroll
   for (int i = 0; i < S1_PREFETCH - 1; ++i) prefetch(i);
@@ -178,22 +200,18 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
       }
       a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, 1));
       a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-      const uint32_t sb0 = cvt_e4m3(__fdiv_rn(a0, six_s));
-      const uint32_t sb1 = cvt_e4m3(__fdiv_rn(a1, six_s));
-      const float d0 = __fmul_rn(e4m3_value(sb0), s_a);
-      const float d1 = __fmul_rn(e4m3_value(sb1), s_a);
-      const float r0 = __frcp_rn(d0), r1 = __frcp_rn(d1);
-      uint32_t w0 = 0, w1 = 0;
-      if (d0 != 0.f) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w0 |= cvt_e2m1x2(__fmul_rn(v0[0][2 * e], r0), __fmul_rn(v0[0][2 * e + 1], r0)) << (8 * e);
-      }
-      if (d1 != 0.f) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w1 |= cvt_e2m1x2(__fmul_rn(v1[0][2 * e], r1), __fmul_rn(v1[0][2 * e + 1], r1)) << (8 * e);
-      }
+      // The two lanes of a pair share both groups: the even lane derives row
+      // g's scale, the odd lane row g+8's, and they swap the results.
+      const bool odd = (c & 1) != 0;
+      const uint32_t sb_m = cvt_e4m3(__fmul_rn(odd ? a1 : a0, inv_six_s));
+      const float d_m = __fmul_rn(e4m3_value(sb_m), s_a);
+      const float r_m = d_m != 0.f ? __frcp_rn(d_m) : 0.f;  // 0 marks an all-zero group
+      const float r_o = __shfl_xor_sync(0xffffffffu, r_m, 1);
+      const uint32_t sb_o = __shfl_xor_sync(0xffffffffu, sb_m, 1);
+      const float r0 = odd ? r_o : r_m, r1 = odd ? r_m : r_o;
+      const uint32_t sb0 = odd ? sb_o : sb_m, sb1 = odd ? sb_m : sb_o;
+      const uint32_t w0 = r0 != 0.f ? cvt_e2m1x8(v0[0], r0) : 0u;
+      const uint32_t w1 = r1 != 0.f ? cvt_e2m1x8(v1[0], r1) : 0u;
       const int k = unit * 32 + 8 * c;
       uint8_t* codes = p.act_codes;
       if (ok0) __stcs(reinterpret_cast<unsigned int*>(codes + (size_t)row0 * (K / 2) + k / 2), w0);
@@ -250,22 +268,11 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
       uint32_t ahi[2][4], alo[2][4];
 #pragma unroll
       for (int st = 0; st < 2; ++st) {
-        float h0[4], h1[4], l0[4], l1[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          h0[e] = bf16_round_f(v0[h][4 * st + e]);
-          h1[e] = bf16_round_f(v1[h][4 * st + e]);
-          l0[e] = __fsub_rn(v0[h][4 * st + e], h0[e]);
-          l1[e] = __fsub_rn(v1[h][4 * st + e], h1[e]);
-        }
-        ahi[st][0] = pack_bf16x2(h0[0], h0[1]);
-        ahi[st][1] = pack_bf16x2(h1[0], h1[1]);
-        ahi[st][2] = pack_bf16x2(h0[2], h0[3]);
-        ahi[st][3] = pack_bf16x2(h1[2], h1[3]);
-        alo[st][0] = pack_bf16x2(l0[0], l0[1]);
-        alo[st][1] = pack_bf16x2(l1[0], l1[1]);
-        alo[st][2] = pack_bf16x2(l0[2], l0[3]);
-        alo[st][3] = pack_bf16x2(l1[2], l1[3]);
+        // A fragment registers: (row g, k 0-1), (row g+8, k 0-1), (row g, k 2-3), (row g+8, k 2-3)
+        split_bf16x2(v0[h][4 * st + 0], v0[h][4 * st + 1], ahi[st][0], alo[st][0]);
+        split_bf16x2(v1[h][4 * st + 0], v1[h][4 * st + 1], ahi[st][1], alo[st][1]);
+        split_bf16x2(v0[h][4 * st + 2], v0[h][4 * st + 3], ahi[st][2], alo[st][2]);
+        split_bf16x2(v1[h][4 * st + 2], v1[h][4 * st + 3], ahi[st][3], alo[st][3]);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {

@@ -95,7 +95,7 @@ int svdq_scales_from_rowmajor(int rows, int K, const uint8_t* rowmajor, uint8_t*
  *   R[n,k] = fp32( W[n,k]*smooth[k] - sum_{t ascending} L1[k,t]*L2[t,n] )
  *            (products and sum in fp64, one rounding to fp32);
  *   NVFP4: s_w = amax|R| / 2688 (1 if R == 0); per 16 along k:
- *          a = max|v|, sb = E4M3_rn_sat(a / fp32(6 s_w)), d = float(sb)*s_w,
+ *          a = max|v|, sb = E4M3_rn_sat(a * fp32(1/fp32(6 s_w))), d = float(sb)*s_w,
  *          code = E2M1_rn_sat(v * fp32(1/d)) (sign kept), all codes 0 when d == 0.
  *   INT4:  per 64 along k: sc = bf16(a / 7), q = clamp(rint(v * fp32(1/sc)), -8, 7).
  * Inputs (host): W bf16 [N,K]; smooth fp32 [K] (lambda, > 0); L1 bf16 [K,r];
@@ -123,7 +123,8 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
  * Device inputs: x bf16 [M,K]; inv_smooth fp32 [K]; lora_down bf16 [r,K].
  * Device outputs: act_codes [M, K/2]; act_scales svdq_act_scale_bytes;
  * lora_act bf16 [M, 2r].  act_scale (NVFP4 s_a, e.g. amax|x_hat|/2688) and
- * weight_scale must be > 0 for NVFP4 and are ignored for INT4.
+ * weight_scale must lie in [2^-100, 2^100) for NVFP4 (so that every block
+ * reciprocal is finite) and are ignored for INT4.
  * Shapes: M >= 1, K % 256 == 0, rank == SVDQ_RANK. */
 int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
                       const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,

@@ -95,12 +95,13 @@ def nvfp4_tensor_scale(v):
 def nvfp4_quantize(V, s):
     """NVFP4 quantization of the rows of V along the last axis, group 16.
 
-    Per group of 16: a = max|v|; t = a / fp32(6*s); sb = E4M3(t) (RNE,
-    satfinite); d = fp32(float(sb) * s); r = fp32(1 / d);
+    Per group of 16: a = max|v|; t = fp32(a * fp32(1 / fp32(6*s)));
+    sb = E4M3(t) (RNE, satfinite); d = fp32(float(sb) * s); r = fp32(1 / d);
     code = E2M1(fp32(v * r)) (RNE, satfinite, sign kept).  A group with
-    d == 0 gets all-zero (+0) codes.  The block scale is applied as a multiply
-    by its fp32 reciprocal (one division per block): the pages fix no
-    operation order, and this is the form a streaming quantizer uses.
+    d == 0 gets all-zero (+0) codes.  Every division by a scale is a multiply
+    by the scale's fp32 reciprocal (one division per tensor for 6*s, one per
+    block for d): the pages fix no operation order, and this is the form a
+    streaming quantizer uses.
 
     Returns (codes uint8 [rows, K] one code per element, scales uint8 [rows, K/16]).
     """
@@ -111,7 +112,8 @@ def nvfp4_quantize(V, s):
     G = V.reshape(rows, K // NVFP4_GROUP, NVFP4_GROUP)
     a = np.max(np.abs(G), axis=2)                                   # exact
     six_s = np.float32(np.float32(6.0) * s)
-    t = (a / six_s).astype(np.float32)
+    inv_six_s = np.float32(np.float32(1.0) / six_s)
+    t = (a * inv_six_s).astype(np.float32)
     sb = e4m3_encode_nonneg(t)
     d = (e4m3_decode(sb).astype(np.float32) * s).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
