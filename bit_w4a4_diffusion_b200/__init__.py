@@ -151,12 +151,14 @@ def svdq_pack_weights(precision, W_bits, smooth, L1_bits, L2_bits, rank=SVDQ_RAN
         "scales": np.empty(max(weight_scale_bytes(p, N, K), 1), np.uint8),
         "weight_scale": np.zeros(1, np.float32),
         "inv_smooth": np.empty(K, np.float32),
-        "lora_down": np.empty((rank, K), np.uint16),
+        "lora_down": np.empty((rank, K), np.uint16),     # bits: fp16 (NVFP4) or bf16 (INT4)
         "lora_up": np.empty((N, 2 * rank), np.uint16),
     }
     _check(lib.svdq_pack_weights(p, N, K, rank, _ptr(W_bits), _ptr(smooth), _ptr(L1_bits), _ptr(L2_bits),
                                  _ptr(out["codes"]), _ptr(out["scales"]), _ptr(out["weight_scale"]),
                                  _ptr(out["inv_smooth"]), _ptr(out["lora_down"]), _ptr(out["lora_up"])))
+    if p == SVDQ_NVFP4:
+        out["lora_down"] = out["lora_down"].view(np.float16)   # fp16 operand for NVFP4
     out["N"], out["K"], out["rank"], out["precision"] = N, K, rank, p
     return out
 

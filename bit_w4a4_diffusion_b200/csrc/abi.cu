@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 #include <atomic>
 #include <mutex>
@@ -184,7 +185,18 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
   p.inv_smooth = inv_smooth;
   p.lora_down = static_cast<const uint16_t*>(lora_down);
   p.act_scale = act_scale;
-  p.lora_scale = precision == SVDQ_NVFP4 ? 1.0f / (act_scale * weight_scale) : 1.0f;
+  if (precision == SVDQ_NVFP4) {
+    // x_hat enters the fp16 down-projection as x_hat * 2^-e, with 2^e the power
+    // of two that maps the calibrated range 2688 s_a into [2^12, 2^13).
+    int ex = 0;
+    frexpf(2688.0f * act_scale, &ex);  // 2688 s_a = m * 2^ex, m in [0.5, 1)
+    const int e = ex - 1 - 12;
+    p.lr_in_scale = ldexpf(1.0f, -e);
+    p.lora_scale = ldexpf(1.0f, e) / (act_scale * weight_scale);
+  } else {
+    p.lr_in_scale = 1.0f;
+    p.lora_scale = 1.0f;
+  }
   p.act_codes = static_cast<uint8_t*>(act_codes);
   p.act_scales = static_cast<uint8_t*>(act_scales);
   p.lora_act = static_cast<uint16_t*>(lora_act);

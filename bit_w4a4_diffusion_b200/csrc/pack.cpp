@@ -32,6 +32,27 @@ uint16_t f32_to_bf16_rne(float f) {
   return (uint16_t)((u + 0x7FFFu + lsb) >> 16);  // finite inputs only
 }
 
+// Finite fp32 with |v| <= 65504 -> fp16 bits, round to nearest even (the
+// subnormal range included).
+uint16_t f32_to_f16_rne(float v) {
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  const float a = std::fabs(v);
+  if (a == 0.0f) return sign;
+  int e;
+  std::frexp(a, &e);  // a = m * 2^e, m in [0.5, 1)
+  // Quantum of the fp16 grid at a: 2^(e-11) for normals, 2^-24 in the subnormal range.
+  const int qexp = std::max(e - 11, -24);
+  const float q = std::nearbyint(std::ldexp(a, -qexp));  // integer significand, RNE
+  const float r = std::ldexp(q, qexp);                     // rounded value, exact in fp32
+  if (r < 6.103515625e-05f) return (uint16_t)(sign | (uint16_t)std::ldexp(r, 24));  // subnormal
+  int re;
+  const float rm = std::frexp(r, &re);                     // r = rm * 2^re
+  const uint32_t mant = (uint32_t)std::ldexp(rm, 11) - 1024u;  // 10 stored bits
+  return (uint16_t)(sign | ((uint32_t)(re - 1 + 15) << 10) | mant);
+}
+
 // Non-negative finite fp32 -> E4M3 byte, round to nearest even, saturating at
 // 448 (0x7E).  Works on the fp32 fields directly.
 uint8_t e4m3_rne_sat(float t) {
@@ -129,8 +150,15 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
   const int r = rank;
 
   for (int k = 0; k < K; ++k) inv_smooth[k] = 1.0f / smooth[k];
+  // The down-projection operand: bf16 as given for INT4; for NVFP4 converted to
+  // fp16 (exact for |v| in [2^-17, 65504]: bf16 has 8 significand bits).
+  for (int i = 0; i < K * r; ++i)
+    if (precision == SVDQ_NVFP4 && !(std::fabs(bf16_to_f32(L1[i])) <= 65504.0f)) return SVDQ_ERR_INVALID_ARG;
   for (int t = 0; t < r; ++t)
-    for (int k = 0; k < K; ++k) lora_down[(size_t)t * K + k] = L1[(size_t)k * r + t];
+    for (int k = 0; k < K; ++k) {
+      const uint16_t v = L1[(size_t)k * r + t];
+      lora_down[(size_t)t * K + k] = precision == SVDQ_NVFP4 ? f32_to_f16_rne(bf16_to_f32(v)) : v;
+    }
   for (int n = 0; n < N; ++n)
     for (int t = 0; t < r; ++t) {
       lora_up[(size_t)n * 2 * r + t] = L2[(size_t)t * N + n];

@@ -12,8 +12,12 @@
 //   NVFP4: per 16 along K, a = max|x_hat|, t = a * fp32(1/(6 s_a)), sb = E4M3(t),
 //          d = float(sb) * s_a, code = E2M1(x_hat * fp32(1/d))  (RNE, satfinite)
 //   INT4:  per 64 along K, sc = bf16(a / 7), q = clamp(rint(x_hat * fp32(1/sc)), -8, 7)
-//   u     = x_hat * L1 on tensor cores (mma.sync bf16, fp32 accumulate), with
-//           x_hat split into bf16 hi + lo so that u carries ~16 mantissa bits
+//   u     = x_hat * L1 on tensor cores (mma.sync, fp32 accumulate):
+//           NVFP4: x_hat * 2^-e and L1 in fp16 (11-bit significands), with the
+//           power of two 2^-e chosen from s_a so that the calibrated range
+//           maps to [2^12, 2^13) and nothing overflows; u = acc * 2^e exactly;
+//           INT4 (no tensor scale to bound the range): x_hat split into a
+//           bf16 hi + lo pair so that u carries ~16 significand bits
 //   lora_act[m] = [hi(u * c) | lo(u * c)]  (bf16, 2r values per row), with
 //           c = 1 / (s_a s_w) for NVFP4 (folds the GEMM's per-tensor scale)
 //           and c = 1 for INT4.
@@ -28,6 +32,7 @@
 // products are unchanged.  A 16-group is the lane pair (c, c^1): its amax is
 // one shuffle.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -48,6 +53,19 @@ SVDQ_DEV void unpack8(const uint4& v, float (&f)[8]) {
     f[2 * i] = __uint_as_float(w[i] << 16);
     f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
+}
+
+SVDQ_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+SVDQ_DEV uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low half)
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 SVDQ_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -263,6 +281,24 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
     }
 
     // ---------------- low-rank down-projection ----------------
+    if constexpr (kNvfp4) {
+      const float xs = p.lr_in_scale;
+      uint32_t a[2][4];
+#pragma unroll
+      for (int st = 0; st < 2; ++st) {
+        // A fragment registers: (row g, k 0-1), (row g+8, k 0-1), (row g, k 2-3), (row g+8, k 2-3)
+        a[st][0] = pack_f16x2(__fmul_rn(v0[0][4 * st + 0], xs), __fmul_rn(v0[0][4 * st + 1], xs));
+        a[st][1] = pack_f16x2(__fmul_rn(v1[0][4 * st + 0], xs), __fmul_rn(v1[0][4 * st + 1], xs));
+        a[st][2] = pack_f16x2(__fmul_rn(v0[0][4 * st + 2], xs), __fmul_rn(v0[0][4 * st + 3], xs));
+        a[st][3] = pack_f16x2(__fmul_rn(v1[0][4 * st + 2], xs), __fmul_rn(v1[0][4 * st + 3], xs));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 bw = *slot(ring, 0, 2 + j);
+        mma_f16_16816(acc[j], a[0], bw.x, bw.y);
+        mma_f16_16816(acc[j], a[1], bw.z, bw.w);
+      }
+    } else {
 #pragma unroll
     for (int h = 0; h < STEP; ++h) {
       uint32_t ahi[2][4], alo[2][4];
@@ -282,6 +318,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
         mma_bf16_16816(acc[j], ahi[1], bw.z, bw.w);
         mma_bf16_16816(acc[j], alo[1], bw.z, bw.w);
       }
+    }
     }
   }
   cp_async_wait<0>();
@@ -308,7 +345,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
     for (int w = 0; w < S1_WARPS; ++w) u = __fadd_rn(u, red[w][r][col]);
     const int row = blockIdx.x * S1_ROWS + r;
     if (row < p.M) {
-      const float uf = __fmul_rn(u, p.lora_scale);
+      const float uf = __fmul_rn(u, p.lora_scale);  // lora_scale also undoes 2^-e (NVFP4)
       const __nv_bfloat16 hi = __float2bfloat16_rn(uf);
       const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(uf, __bfloat162float(hi)));
       uint16_t* la = p.lora_act + (size_t)row * 64;

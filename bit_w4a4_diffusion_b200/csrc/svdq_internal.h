@@ -19,9 +19,10 @@ struct QuantActParams {
   int M, K, M_pad;            // M_pad: rows of the scale buffer (multiple of 256)
   const uint16_t* x;          // bf16 [M, K]
   const float* inv_smooth;    // fp32 [K]
-  const uint16_t* lora_down;  // bf16 [r, K]  (L1 transposed)
+  const uint16_t* lora_down;  // [r, K] (L1 transposed): fp16 for NVFP4, bf16 for INT4
   float act_scale;            // NVFP4 per-tensor activation scale s_a
-  float lora_scale;           // multiplier folded into lora_act (1/(s_a s_w) or 1)
+  float lora_scale;           // multiplier folded into lora_act: 2^e/(s_a s_w) (NVFP4) or 1
+  float lr_in_scale;          // NVFP4: 2^-e applied to x_hat before its fp16 conversion
   uint8_t* act_codes;         // [M, K/2]
   uint8_t* act_scales;        // NVFP4: tiled e4m3; INT4: bf16 [K/64][M_pad]
   uint16_t* lora_act;         // bf16 [M, 2r]  (hi | lo)

@@ -104,7 +104,9 @@ int svdq_scales_from_rowmajor(int rows, int K, const uint8_t* rowmajor, uint8_t*
  *   scales     svdq_weight_scale_bytes(precision, N, K) bytes
  *   weight_scale  1 float (s_w; 1.0 for INT4)
  *   inv_smooth fp32 [K]
- *   lora_down  bf16 [r, K]   (L1 transposed, the down-projection operand)
+ *   lora_down  [r, K] 16-bit (L1 transposed, the down-projection operand):
+ *              fp16 for NVFP4 (|L1| must not exceed 65504, else
+ *              SVDQ_ERR_INVALID_ARG), bf16 for INT4
  *   lora_up    bf16 [N, 2r]  (row n = [L2[:,n], L2[:,n]], the up-projection
  *                             operand for the hi/lo split activation)
  * Shapes: N % 128 == 0, K % 256 == 0, rank == SVDQ_RANK. */
@@ -117,10 +119,13 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
  * down-projection in one pass over x (the Nunchaku engine's fused
  * "down-projection + quantize" kernel, "SVDQuant and the Nunchaku engine").
  *   x_hat = fp32(x) * inv_smooth;  codes/scales as in svdq_pack_weights with
- *   s = act_scale for NVFP4;  u = x_hat L1 (fp32 accumulate);
+ *   s = act_scale for NVFP4;  u = x_hat L1;
  *   lora_act[m] = [hi(u*c), lo(u*c)] (bf16 pair whose sum is u*c to ~2^-16),
  *   c = 1/(act_scale*weight_scale) for NVFP4 and 1 for INT4.
- * Device inputs: x bf16 [M,K]; inv_smooth fp32 [K]; lora_down bf16 [r,K].
+ * NVFP4 runs the down-projection on fp16 operands: x_hat * 2^-e with 2^e the
+ * power of two mapping 2688*act_scale into [2^12, 2^13), times the fp16
+ * lora_down; INT4 uses a bf16 hi+lo split of x_hat.  Both accumulate in fp32.
+ * Device inputs: x bf16 [M,K]; inv_smooth fp32 [K]; lora_down [r,K] as packed.
  * Device outputs: act_codes [M, K/2]; act_scales svdq_act_scale_bytes;
  * lora_act bf16 [M, 2r].  act_scale (NVFP4 s_a, e.g. amax|x_hat|/2688) and
  * weight_scale must lie in [2^-100, 2^100) for NVFP4 (so that every block

@@ -52,12 +52,14 @@ def _check_s1(inp, codes, scales, lora, pk, rows=None):
     if Mp > M:
         full = _lib().scales_to_rowmajor(scales.cpu().numpy(), Mp, K)
         assert np.all(full[M:] == 0)
-    # low-rank activation: hi + lo = u / alpha with u = x_hat L1
+    # low-rank activation: hi + lo = u / alpha with u = x_hat L1 (fp16 operands:
+    # 11-bit significands, fp32 accumulation)
     alpha = np.float64(np.float32(np.float32(inp.act_scale) * np.float32(pk["weight_scale"][0])))
     la = lora.float().cpu().numpy().astype(np.float64)[sel]
     u = ref["x_hat"].astype(np.float64) @ inp.L1.astype(np.float64) / alpha
     err = np.abs(la[:, :32] + la[:, 32:] - u)
-    assert np.max(err) <= 1e-5 * np.max(np.abs(u)) + 1e-30, f"low-rank activation error {np.max(err)}"
+    assert np.max(err) <= 2e-3 * np.max(np.abs(u)) + 1e-30, f"low-rank activation error {np.max(err)}"
+    assert np.linalg.norm(err) <= 5e-4 * np.linalg.norm(u) + 1e-30
     return ref
 
 

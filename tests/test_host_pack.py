@@ -51,8 +51,12 @@ def test_pack_weights_matches_oracle(name, kw):
         np_ = (c.N + 255) // 256 * 256
         sc = pk["scales"].view(np.uint16).reshape(c.K // 64, np_)[:, :c.N].T
         assert np.array_equal(wl.to_bf16(ref["sc"])[0], sc)
-    # low-rank operand layouts
-    assert np.array_equal(pk["lora_down"], inp.L1_bits.T)
+    # low-rank operand layouts (the NVFP4 down-projection operand is fp16)
+    if c.precision == "nvfp4":
+        assert pk["lora_down"].dtype == np.float16
+        assert np.array_equal(pk["lora_down"], inp.L1.T.astype(np.float16))
+    else:
+        assert np.array_equal(pk["lora_down"], inp.L1_bits.T)
     assert np.array_equal(pk["lora_up"][:, :32], inp.L2_bits.T)
     assert np.array_equal(pk["lora_up"][:, 32:], inp.L2_bits.T)
 
@@ -86,3 +90,30 @@ def test_awq_pack_matches_oracle(N, K):
     assert np.array_equal(pk["scales"], wl.to_bf16(sc)[0])
     zz = np.stack([pk["zeros"] & 0xF, pk["zeros"] >> 4], axis=-1).reshape(N, -1)
     assert np.array_equal(zz, z)
+
+
+def test_fp16_operand_rounding_matches_numpy():
+    """The packer's bf16 -> fp16 conversion of L1 (every finite bf16 value up
+    to 65504, subnormal range included) against numpy's float16 cast."""
+    bits = np.arange(0, 0x8000, dtype=np.uint32).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(vals) & (vals <= 65504.0)
+    vals = vals[keep]
+    K = 256
+    n = (len(vals) // K) * K
+    L1 = np.concatenate([vals[:n], -vals[:n]]).reshape(-1, K)[:, :K]
+    L1 = L1[: (L1.shape[0] // 32) * 32]
+    r_blocks = L1.reshape(-1, 32, K)
+    for blk in r_blocks[:: max(1, len(r_blocks) // 40)]:
+        L1b = wl.to_bf16(blk.T.astype(np.float32))[0]           # [K, 32] bits
+        pk = B.svdq_pack_weights("nvfp4", np.zeros((128, K), np.uint16), np.ones(K, np.float32), L1b,
+                                 np.zeros((32, 128), np.uint16))
+        assert np.array_equal(pk["lora_down"].view(np.uint16), blk.astype(np.float16).view(np.uint16))
+
+
+def test_pack_rejects_out_of_fp16_range_factor():
+    L1 = np.zeros((256, 32), np.float32)
+    L1[3, 5] = 70000.0
+    with pytest.raises(B.SvdqError):
+        B.svdq_pack_weights("nvfp4", np.zeros((128, 256), np.uint16), np.ones(256, np.float32),
+                            wl.to_bf16(L1)[0], np.zeros((32, 128), np.uint16))
