@@ -18,17 +18,19 @@
 //   warp 1      MMA issuer (MMAs and commits only)
 //   warps 2..5  epilogue (TMEM -> registers -> bf16 -> swizzled smem -> TMA store)
 //   warps 6..8  block-scale copies smem -> TMEM (SFA, SFB rows 0-127, SFB rows
-//               128-255): each tcgen05.cp holds its issuing thread for tens of
-//               cycles, so the 12 copies of a K slice are spread over three
-//               threads that run ahead of the MMA warp into a second buffer.
+//               128-255), running ahead of the MMA warp into a second buffer.
+//               Copies issued by the MMA thread itself would be ordered with
+//               its MMAs for free, but each one takes tens of cycles of the
+//               tensor pipe (about 40 on sm_100a, only about three per four
+//               MMAs hide); issued from other threads they overlap the MMAs.
 // Pipeline: STAGES-deep smem ring of K=256 slices; slot 0 of every tile is the
 // low-rank slice (u' in the A slot, [L2^T|L2^T] in the B slot).
 // Tensor memory (512 columns): two 256-column fp32 accumulators at columns 0
 // and 160, overlapping in [160, 256), and two 48-column block-scale buffers
 // in [416, 512) (K slices alternate buffers).  Consecutive tiles alternate
-// accumulators; the epilogue drains the shared 96 columns first and then
-// releases the accumulator, so the next tile's MMAs run while the epilogue
-// finishes the other 160 columns.
+// accumulators; the epilogue loads the 96 shared columns into registers first
+// and releases the accumulator at once, so the next tile's MMAs run while the
+// epilogue converts and stores.
 // Every mbarrier wait is bounded; on timeout the kernel records a status code,
 // drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -299,17 +301,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile.
-    // Columns are read from TMEM 32 at a time, the next chunk's load in flight
-    // while the current one is converted; the tile's bias is loaded once (lane
-    // l holds columns 8l..8l+7) and broadcast by shuffles.
+    // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile,
+    // read from TMEM 32 columns at a time into a ring of three register
+    // blocks.  The three chunks holding the columns shared with the other
+    // accumulator are loaded first, with one wait, and the accumulator is
+    // released before any of them is converted; later chunks are loaded into
+    // the block just converted, three chunks ahead.  The tile's bias is loaded
+    // once (lane l holds columns 8l..8l+7) and broadcast by shuffles.
     const int q = warp & 3;
     uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;
     uint32_t acc_phase = 0;
     int chunk_seq = 0, it = 0;
     constexpr int LDC = 32;                    // columns per TMEM load
     constexpr int NCH = BN / LDC;
-    constexpr int NOVL = ACC_OVERLAP / LDC;
+    constexpr int NSH = (ACC_OVERLAP + LDC - 1) / LDC;  // chunks holding shared columns
+    constexpr int NBUF = 3;
+    static_assert(NSH <= NBUF, "the shared chunks fit the first ring fill");
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM;
       const int n0 = (tile / tiles_m) * BN;
@@ -320,23 +327,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
       tc_fence_after();
       const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
-      // The columns shared with the other accumulator go first: the last 64
-      // of accumulator 0, the first 64 of accumulator 1.
-      auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NOVL) % NCH : i; };
-      uint32_t rbuf[2][32];
-      tmem_ld_32x32b_x32(acc_base + chunk_col(0) * LDC, rbuf[0]);
-      tmem_ld_wait(rbuf[0]);
+      // The columns shared with the other accumulator go first: the last
+      // ACC_OVERLAP of accumulator 0, the first ACC_OVERLAP of accumulator 1.
+      auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NSH) % NCH : i; };
+      uint32_t rb[NBUF][32];
+#pragma unroll
+      for (int i = 0; i < NBUF; ++i) tmem_ld_32x32b_x32(acc_base + chunk_col(i) * LDC, rb[i]);
+      tmem_ld_wait(rb[0]);
+      reg_fence(rb[1]);
+      reg_fence(rb[2]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
-        uint32_t(&r)[32] = rbuf[i & 1];
-        if (i + 1 < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + 1) * LDC, rbuf[(i + 1) & 1]);
-        if (i == NOVL - 1) {
-          // The shared columns (chunks 0 .. NOVL-1) are all in registers once
-          // this wait returns; release the accumulator to the MMA warp.
-          tmem_ld_wait(rbuf[(i + 1) & 1]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
+        uint32_t(&r)[32] = rb[i % NBUF];
+        if (i >= NBUF && i % NBUF == 0) {
+          // Chunks loaded since the last wait (i .. i+2 at most) land here.
+          tmem_ld_wait(rb[0]);
+          reg_fence(rb[1]);
+          reg_fence(rb[2]);
         }
         const int cc = chunk_col(i);
 #pragma unroll
@@ -378,7 +388,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) bulk_commit();
           ++chunk_seq;
         }
-        if (i + 1 < NCH && i != NOVL - 1) tmem_ld_wait(rbuf[(i + 1) & 1]);
+        // Refill the block just converted with the chunk three ahead; the
+        // accumulator is still this tile's until the MMA warp reuses it, and
+        // the non-shared chunks are not written by the next tile.
+        if (i + NBUF < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + NBUF) * LDC, r);
       }
       acc_phase ^= 1;
     }

@@ -224,6 +224,18 @@ SVDQ_DEV void tmem_ld_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 
+// Register-only fence: no use of r can be scheduled above this point.  Placed
+// after a tmem_ld_wait (volatile asm statements keep their order) it extends
+// that wait's ordering to another register block.
+SVDQ_DEV void reg_fence(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
 // Shared-memory matrix descriptor (tcgen05 form, version 1).
 //   layout: 0 = no swizzle, 2 = 128-byte swizzle, 4 = 64-byte swizzle.
 SVDQ_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
