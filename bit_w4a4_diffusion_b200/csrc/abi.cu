@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cmath>
 #include <cstring>
 #include <atomic>
@@ -204,6 +205,18 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
                     "quantize_act launch");
 }
 
+// NVFP4 GEMM kernel: the one-CTA-per-tile kernel unless
+// SVDQ_NVFP4_GEMM_KERNEL=pair asks for the CTA-pair kernel (read at every
+// call, so a process can compare the two).  Both give bit-identical results.
+// On B200 the single-CTA kernel is 2-6% faster at K = 3072 and the pair
+// kernel 2.6% faster at K = 12288: the pair halves the B bytes per SM, but
+// each stage's round trip then spans both SMs, which costs more than the
+// bytes saved while the load ring is latency-bound.
+static bool use_pair_gemm() {
+  const char* v = getenv("SVDQ_NVFP4_GEMM_KERNEL");
+  return v && strcmp(v, "pair") == 0;
+}
+
 static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const void* act_scales, const void* lora_act,
                            const void* w_codes, const void* w_scales, const void* lora_up, const void* bias,
                            float alpha, void* y, int* dev_status, cudaStream_t stream, bool pdl, int sms) {
@@ -230,6 +243,26 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
   p.alpha = alpha;
   p.dev_status = dev_status;
   p.timeout_ns = svdq_timeout_ns();
+  if (use_pair_gemm()) {
+    // CTA-pair kernel: half-tile boxes for B and [L2^T|L2^T], and the block
+    // scales as 2D maps of 256-byte rows (8 rows = one 2 KB chunk group).
+    GemmPairTmaps u;
+    u.a = t.a;
+    u.la = t.la;
+    u.y = t.y;
+    const uint64_t sfa_rows = (uint64_t)round_up(M, 256) * (K / 16) / 256;
+    const uint64_t sfb_rows = (uint64_t)round_up(N, 256) * (K / 16) / 256;
+    ok &= encode_tmap_2d(&u.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= encode_tmap_2d(&u.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
+                         128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= encode_tmap_2d(&u.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_scales, 256, sfa_rows, 256, 256, 8,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= encode_tmap_2d(&u.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 256, sfb_rows, 256, 256, 8,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the CTA-pair GEMM");
+    return check_cuda(launch_gemm_nvfp4_pair(p, u, stream, pdl), "gemm_nvfp4_pair launch");
+  }
   return check_cuda(launch_gemm_nvfp4(p, t, sms, stream, pdl), "gemm_nvfp4 launch");
 }
 

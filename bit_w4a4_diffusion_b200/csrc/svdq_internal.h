@@ -47,6 +47,14 @@ struct GemmTmaps {
 cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                               bool pdl);
 
+// The CTA-pair kernel: B and [L2^T|L2^T] boxes are 128 rows (half a tile),
+// block scales are read through 2D maps of 256-byte rows (box 256 x 8).
+struct GemmPairTmaps {
+  CUtensorMap a, b, la, lb, y, sfa, sfb;
+};
+
+cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl);
+
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;
   const uint16_t* act_scales;  // bf16 [K/64][M_pad]

@@ -82,8 +82,12 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("kernel", ["pair", "single"])
 @pytest.mark.parametrize("name,kw", SMALL)
-def test_linear_small_matches_oracle(name, kw):
+def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
+    """Both NVFP4 GEMM kernels: the one-CTA-per-tile kernel (the default) and
+    the CTA-pair kernel."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     B = _lib()
     c = wl.SVDQ_CASES[name]
     if kw:
@@ -131,10 +135,12 @@ def test_quantize_ties_and_signed_zero():
 FULL = ["qkv", "mlp_up", "mlp_down"]
 
 
+@pytest.mark.parametrize("kernel", ["single", "pair"])
 @pytest.mark.parametrize("name", FULL)
-def test_linear_full_size_sampled(name):
+def test_linear_full_size_sampled(name, kernel, monkeypatch):
     """Full workload shape (the launch configuration the benchmark times):
     all activation codes bit-exact, 48 sampled output rows within tolerance."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     B = _lib()
     c = wl.SVDQ_CASES[name]
     inp, pk, w, bias = _layer(c)
