@@ -46,7 +46,7 @@ GEMM_TRAFFIC = {
         "bit_w4a4_diffusion_b200/csrc/gemm_nvfp4.cu":
             "0e287ef39c67008611952698abdd2bd3d107f7addebb3afdeb4f0de9137df015",
         "bit_w4a4_diffusion_b200/csrc/ptx.cuh":
-            "07e95ebd7535f81e4eed1c4b4cb3b802ab03c061e684db09a067bb4bbe813e93",
+            "606656540d9b84a2048833a8cc34bab5e89372da375464192b196a3f4bcd39c1",
     },
 }
 
