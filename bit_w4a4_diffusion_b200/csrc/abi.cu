@@ -158,6 +158,15 @@ long long svdq_workspace_bytes(int precision, int M, int K, int rank) {
   return codes + scales + lora;
 }
 
+// NVFP4 activation quantizer: the TMA-fed kernel unless
+// SVDQ_NVFP4_QUANT_KERNEL=copy asks for the per-thread-copy kernel (read at
+// every call).  Both give bit-identical codes and scales; the low-rank
+// activations differ only by the order of their fp32 partial sums.
+static bool use_copy_quantizer() {
+  const char* v = getenv("SVDQ_NVFP4_QUANT_KERNEL");
+  return v && strcmp(v, "copy") == 0;
+}
+
 int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
                       const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,
                       void* lora_act, void* stream) {
@@ -201,6 +210,17 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
   p.act_codes = static_cast<uint8_t*>(act_codes);
   p.act_scales = static_cast<uint8_t*>(act_scales);
   p.lora_act = static_cast<uint16_t*>(lora_act);
+  if (precision == SVDQ_NVFP4 && !use_copy_quantizer()) {
+    // TMA-fed kernel: x [M, K] bf16 and L1^T [32, K] fp16 in 64 x 32 boxes.
+    CUtensorMap tx, tl;
+    bool ok = encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, (uint64_t)K * 2, 64, 32,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= encode_tmap_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, lora_down, K, SVDQ_RANK, (uint64_t)K * 2, 64, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the quantize kernel");
+    return check_cuda(launch_quantize_nvfp4(p, tx, tl, nullptr, svdq_timeout_ns(), static_cast<cudaStream_t>(stream)),
+                      "quantize_nvfp4 launch");
+  }
   return check_cuda(launch_quantize_act(p, precision == SVDQ_NVFP4, static_cast<cudaStream_t>(stream)),
                     "quantize_act launch");
 }

@@ -107,6 +107,30 @@ def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
     assert torch.equal(y, y2), "svdq_w4a4_linear differs from quantize + gemm"
 
 
+@pytest.mark.parametrize("name,kw", SMALL)
+def test_quantizers_agree(name, kw, monkeypatch):
+    """The TMA-fed NVFP4 quantizer (the default) and the per-thread-copy one
+    produce the same codes and scales bit for bit; their low-rank activations
+    differ only by the order of the fp32 partial sums (each is checked
+    against the oracle in the other tests)."""
+    B = _lib()
+    c = wl.SVDQ_CASES[name]
+    if kw:
+        c = wl.scaled_case(c, **kw)
+    inp, pk, w, bias = _layer(c)
+    outs = {}
+    for kern in ("tma", "copy"):
+        monkeypatch.setenv("SVDQ_NVFP4_QUANT_KERNEL", kern)
+        outs[kern] = _run_s1(inp, w)[1:]
+    torch.cuda.synchronize()
+    for a, b, what in zip(outs["tma"][:2], outs["copy"][:2], ("codes", "scales")):
+        assert torch.equal(a, b), f"{c.name}: {what} differ between the two quantizers"
+    la = outs["tma"][2].float().cpu().numpy()
+    lb = outs["copy"][2].float().cpu().numpy()
+    u_a, u_b = la[:, :32] + la[:, 32:], lb[:, :32] + lb[:, 32:]
+    assert np.max(np.abs(u_a - u_b)) <= 1e-5 * np.max(np.abs(u_b)) + 1e-30
+
+
 def test_quantize_ties_and_signed_zero():
     """Exact E2M1 midpoints and values that round to -0 (inv_smooth = 1)."""
     B = _lib()
