@@ -82,6 +82,18 @@ def _cpu_threads():
     return os.cpu_count() or 1
 
 
+def workload_config(M, K, N, world):
+    """The `config` object of both arms' JSON lines (identical by construction)."""
+    per_set = M * K * 2 + M * N * 2 + N * K // 2 + N * K // 16 + N * 128
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    return {"workload": f"DiT MLP up-projection, svdq_w4a4_linear NVFP4 r32: x bf16 [{M},{K}] -> "
+                        f"y bf16 [{M},{N}] (quantize + low-rank down-proj, FP4 GEMM + low-rank up-proj + bias)",
+            "M": M, "K": K, "N": N, "rank": 32, "global_batch_tokens": M * world,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"rotating {nsets} weight/activation/output sets ({nsets * per_set / 2**20:.0f} MiB "
+                  f"> 126 MiB L2)"}
+
+
 # ------------------------------------------------------------------ oracle arm
 
 def oracle_offline(inp):
@@ -323,13 +335,7 @@ def run_gpu(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-        "config": {"workload": f"DiT MLP up-projection, svdq_w4a4_linear NVFP4 r32: x bf16 [{M},{K}] -> "
-                               f"y bf16 [{M},{N}] (quantize + low-rank down-proj, FP4 GEMM + low-rank up-proj "
-                               f"+ bias)",
-                   "M": M, "K": K, "N": N, "rank": 32, "global_batch_tokens": M * world,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"rotating {nsets} weight/activation/output sets ({nsets * per_set / 2**20:.0f} MiB "
-                         f"> 126 MiB L2)"},
+        "config": workload_config(M, K, N, world),
         "pct_of_fp4_peak": {"spec_dense_9pf": round(100 * value / world / FP4_SPEC_DENSE_TFLOPS, 2),
                             f"{peak_src}_bf16x4": round(100 * value / world / fp4_peak, 2)},
         "roofline": {"kernel": "gemm_nvfp4 (S2)", "bound": "tensor", "achieved": round(s2_tflops, 1),
@@ -443,7 +449,7 @@ def main():
             "impl": "reference", "metric": METRIC, "value": round(tf, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": f"DiT MLP up-projection {case.M}x{case.K}->{case.N} NVFP4 r32"},
+            "data": "synthetic", "config": workload_config(case.M, case.K, case.N, args.gpus),
             "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(tf, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

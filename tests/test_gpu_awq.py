@@ -24,3 +24,19 @@ def test_awq_matches_oracle(M, with_bias):
     q, sc, z = OA.awq_quantize(inp.W)
     _, y64 = OA.awq_linear(inp.x, q, sc, z, inp.bias)
     assert_output_close(y.float().cpu().numpy(), y64, f"awq M={M}")
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 256, 8192), (19, 512, 1024), (1, 16, 128)])
+def test_awq_other_shapes(M, N, K):
+    """A long K, a short one with fewer 16-row blocks than SMs, and the minimal
+    shape (one 16-row block, two groups)."""
+    import bit_w4a4_diffusion_b200 as B
+    inp = wl.make_awq_inputs(M, N=N, K=K, seed=11, with_bias=True)
+    pk = B.awq_pack_weights(inp.W_bits)
+    w = B.to_device(pk)
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    y = B.awq_w4a16_linear(x, w, bias=B.bits_to_bf16(inp.bias_bits, "cuda"))
+    torch.cuda.synchronize()
+    q, sc, z = OA.awq_quantize(inp.W)
+    _, y64 = OA.awq_linear(inp.x, q, sc, z, inp.bias)
+    assert_output_close(y.float().cpu().numpy(), y64, f"awq M={M} N={N} K={K}")
