@@ -46,6 +46,8 @@ constexpr int B8_BYTES = BN * KS;            // 16 KB int8 (also [L2^T|L2^T] bf1
 constexpr int SC_BYTES = 2 * (BM + BN) * 2;  // bf16 scales of two groups, A then B
 constexpr int STAGE_BYTES = A8_BYTES + B8_BYTES + A4_BYTES + B4_BYTES + 1024;  // scales padded to 1 KB
 constexpr int UNPACK_WARPS = 4, EPI_WARPS = 8;
+constexpr int EPI_COLS = 4 * BN / EPI_WARPS;   // columns per epilogue warp (4 warps per lane quarter)
+constexpr int NHALF = EPI_COLS / 32;           // 32-column TMEM loads per warp
 constexpr int NUM_THREADS = (2 + UNPACK_WARPS + EPI_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int TMEM_PART = 0;     // two int32 partial buffers: columns 0 and 128
@@ -303,9 +305,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int e = warp - (2 + UNPACK_WARPS);  // 0..7
+    const int e = warp - (2 + UNPACK_WARPS);  // 0 .. EPI_WARPS - 1
     const int q = warp & 3;                   // TMEM lane quarter
-    const int ch = e >> 2;                    // column half: 64 columns each
+    const int ch = e >> 2;                    // column block of EPI_COLS
     const int row = 32 * q + lane;            // row of the tile this thread owns
     int stage = 0;
     uint32_t phase = 0, pcount = 0;
@@ -313,9 +315,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
-      float acc[64];
+      float2 acc[EPI_COLS / 2];   // columns (2 i, 2 i + 1) of this thread's EPI_COLS
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+      for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.f, 0.f);
       for (int kt = 0; kt < slices && ok; ++kt) {
         if (kt > 0) {
           // Acquire the slice's scales (landed by bulk copy) directly.
@@ -333,15 +335,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const float sa = __bfloat162float(__ushort_as_bfloat16(sc[h * BM + row]));
-            const uint16_t* sw = sc + 2 * BM + h * BN + 64 * ch;
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_PART + pb * BN + 64 * ch;
+            const float sa1 = __bfloat162float(__ushort_as_bfloat16(sc[h * BM + row]));
+            const float2 sa = make_float2(sa1, sa1);
+            const float2 unbias = make_float2(-12582912.0f, -12582912.0f);
+            const uint16_t* sw = sc + 2 * BM + h * BN + EPI_COLS * ch;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_PART + pb * BN + EPI_COLS * ch;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int half = 0; half < NHALF; ++half) {
               uint32_t r[32];
               tmem_ld_32x32b_x32(taddr + 32 * half, r);
               tmem_ld_wait(r);
-              if (half == 1) {
+              if (half == NHALF - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl->part_empty[pb]));
@@ -351,12 +355,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint4 w8 = *reinterpret_cast<const uint4*>(sw + 32 * half + 8 * v);
                 const uint32_t ws[4] = {w8.x, w8.y, w8.z, w8.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float swj = __uint_as_float(i & 1 ? (ws[i >> 1] & 0xFFFF0000u) : (ws[i >> 1] << 16));
-                  // |P| <= 64 * 7 * 7 < 2^22: exact int -> float through the 1.5 * 2^23 bias.
-                  const float pf = __fsub_rn(__int_as_float((int)r[8 * v + i] + 0x4B400000), 12582912.0f);
-                  const int j = 32 * half + 8 * v + i;
-                  acc[j] = __fmaf_rn(__fmul_rn(sa, pf), swj, acc[j]);
+                for (int i = 0; i < 4; ++i) {
+                  // Two columns at a time with the packed fp32x2 instructions:
+                  // |P| <= 64 * 7 * 7 < 2^22, exact int -> float through the
+                  // 1.5 * 2^23 bias; then acc += s_a * (s_w * P).
+                  const float2 sw2 = make_float2(__uint_as_float(ws[i] << 16), __uint_as_float(ws[i] & 0xFFFF0000u));
+                  const float2 pf = __fadd2_rn(make_float2(__int_as_float((int)r[8 * v + 2 * i] + 0x4B400000),
+                                                           __int_as_float((int)r[8 * v + 2 * i + 1] + 0x4B400000)),
+                                               unbias);
+                  const int j = 16 * half + 4 * v + i;
+                  acc[j] = __ffma2_rn(sa, __fmul2_rn(sw2, pf), acc[j]);
                 }
               }
             }
@@ -376,18 +384,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Low-rank accumulator (its MMAs completed before the last partial's).
       const int lb = it & 1;
       const int m = m0 + row;
-      const uint32_t laddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_LR + lb * BN + 64 * ch;
+      const uint32_t laddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_LR + lb * BN + EPI_COLS * ch;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < NHALF; ++half) {
         uint32_t l[32];
         tmem_ld_32x32b_x32(laddr + 32 * half, l);
         tmem_ld_wait(l);
-        if (half == 1) {
+        if (half == NHALF - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctl->lr_empty[lb]));
         }
-        const int nb = n0 + 64 * ch + 32 * half;
+        const int nb = n0 + EPI_COLS * ch + 32 * half;
         if (m < p.M && nb < p.N) {
           uint16_t* yrow = p.y + (size_t)m * p.N + nb;
 #pragma unroll
@@ -396,8 +404,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int j = 8 * v + 2 * i;
-              float y0 = __fadd_rn(acc[32 * half + j], __uint_as_float(l[j]));
-              float y1 = __fadd_rn(acc[32 * half + j + 1], __uint_as_float(l[j + 1]));
+              float y0 = __fadd_rn(acc[16 * half + j / 2].x, __uint_as_float(l[j]));
+              float y1 = __fadd_rn(acc[16 * half + j / 2].y, __uint_as_float(l[j + 1]));
               if (p.bias) {
                 y0 = __fadd_rn(y0, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j])));
                 y1 = __fadd_rn(y1, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j + 1])));
