@@ -57,9 +57,12 @@ struct WaitCtx {
 SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  // The abort word and the clock are read after the first failed poll and
+  // then every 64 polls (try_wait itself suspends the thread for a while, so
+  // a wait can end within a few polls; a limit shorter than one poll still
+  // takes effect at the first).
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0) {
+    if (i == 1 || (i & 63) == 0) {
       if (*ctx.abort_flag) return false;
       if (globaltimer_ns() - t0 > ctx.limit_ns) {
         *ctx.abort_flag = 1;
@@ -67,6 +70,7 @@ SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int c
         return false;
       }
     }
+    if (mbar_try_wait(bar, parity)) return true;
   }
 }
 

@@ -1,0 +1,52 @@
+"""Failure detection without a GPU fault: every mbarrier wait in the NVFP4
+GEMM kernels is bounded by the library's wait limit.  With the limit set to
+1 ns the first wait that is not already satisfied gives up; the kernel must
+report a timeout code through dev_status, drain its own copies and MMAs,
+free its tensor memory and return, leaving the context usable: the next
+call with the normal limit gives the correct result."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import svdq as O
+from tests.helpers import assert_output_close
+
+pytestmark = pytest.mark.gpu
+
+TIMEOUT_CODES = (1, 2, 3, 4)   # producer, MMA, epilogue, drain (csrc/svdq_internal.h)
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+def test_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
+    import bit_w4a4_diffusion_b200 as B
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
+    c = wl.scaled_case(wl.SVDQ_CASES["qkv"], M=640, N=2048)   # several tiles per CTA
+    inp = wl.make_svdq_inputs(c)
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    bias = B.bits_to_bf16(inp.bias_bits, "cuda") if inp.bias_bits is not None else None
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    s_a = float(inp.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, w["inv_smooth"], w["lora_down"], s_a, w["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk["weight_scale"][0])))
+    torch.cuda.synchronize()
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_gemm("nvfp4", codes, scales, lora, w, alpha, bias=bias, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+
+    status.zero_()
+    y = B.svdq_w4a4_gemm("nvfp4", codes, scales, lora, w, alpha, bias=bias, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
+    y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, inp.bias)
+    assert_output_close(y.float().cpu().numpy(), y64, f"{kernel} GEMM after a timed-out call")
