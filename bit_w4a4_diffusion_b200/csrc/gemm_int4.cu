@@ -76,9 +76,6 @@ constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 
 SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 
-SVDQ_DEV void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // Eight packed int4 (two's complement, element 2j in the low nibble of byte
 // j) -> eight int8 in element order (two 32-bit words).
@@ -290,12 +287,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             fence_proxy_async_smem();
           }
-          named_bar(1, UNPACK_WARPS * 32);
-          if (threadIdx.x == 64 && ok) mbar_arrive(smem_u32(&ctl->opnd[stage]));
-          if (!ok || ctl->abort_flag) {
+          // The stop decision is taken inside the barrier (an OR over all
+          // unpack threads), so that no unpack warp can go on to the next
+          // barrier after another one has left.
+          if (named_bar_any(1, UNPACK_WARPS * 32, !ok || ctl->abort_flag != 0)) {
             ok = false;
             break;
           }
+          if (threadIdx.x == 64) mbar_arrive(smem_u32(&ctl->opnd[stage]));
         }
         if (++stage == STAGES) {
           stage = 0;

@@ -74,6 +74,22 @@ SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int c
   }
 }
 
+// Named barrier `id` over `nthreads` threads that also returns, to every
+// participant, whether any of them passed a true `flag` (bar.red.or): a
+// decision taken this way is the same in every thread.
+SVDQ_DEV bool named_bar_any(uint32_t id, uint32_t nthreads, bool flag) {
+  uint32_t any;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(any)
+      : "r"((uint32_t)flag), "r"(id), "r"(nthreads)
+      : "memory");
+  return any != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 SVDQ_DEV void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

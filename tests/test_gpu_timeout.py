@@ -1,9 +1,9 @@
 """Failure detection without a GPU fault: every mbarrier wait in the NVFP4
-GEMM kernels is bounded by the library's wait limit.  With the limit set to
-1 ns the first wait that is not already satisfied gives up; the kernel must
-report a timeout code through dev_status, drain its own copies and MMAs,
-free its tensor memory and return, leaving the context usable: the next
-call with the normal limit gives the correct result."""
+and INT4 GEMM kernels is bounded by the library's wait limit.  With the limit
+set to 1 ns the first wait that is not already satisfied gives up; the kernel
+must report a timeout code through dev_status, drain its own copies and MMAs,
+free its tensor memory and return, leaving the context usable: the next call
+with the normal limit gives the correct result."""
 import numpy as np
 import pytest
 import torch
@@ -50,3 +50,33 @@ def test_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
     y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, inp.bias)
     assert_output_close(y.float().cpu().numpy(), y64, f"{kernel} GEMM after a timed-out call")
+
+
+def test_int4_gemm_wait_timeout_reports_and_recovers():
+    import bit_w4a4_diffusion_b200 as B
+    c = wl.scaled_case(wl.SVDQ_CASES["int4_m1024"], M=1024)
+    inp = wl.make_svdq_inputs(c)
+    pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    codes, scales, lora = B.svdq_quantize_act("int4", x, w["inv_smooth"], w["lora_down"], 1.0, 1.0)
+    torch.cuda.synchronize()
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_gemm("int4", codes, scales, lora, w, 1.0, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+
+    status.zero_()
+    y = B.svdq_w4a4_gemm("int4", codes, scales, lora, w, 1.0, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_pw = O.pack_weights("int4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("int4", inp.x, ref_pw["inv_lam"], np.float32(1.0))
+    y64 = O.linear_f64("int4", act, ref_pw, inp.L1, inp.L2, inp.bias)
+    assert_output_close(y.float().cpu().numpy(), y64, "INT4 GEMM after a timed-out call")
