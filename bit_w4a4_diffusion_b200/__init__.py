@@ -50,6 +50,11 @@ def _load():
         "svdq_quantize_act": (I, [I, I, I, I, P, P, P, F, F, P, P, P, P]),
         "svdq_w4a4_gemm": (I, [I, I, I, I, I, P, P, P, P, P, P, P, F, P, P, P]),
         "svdq_w4a4_linear": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, LL, P, P]),
+        "svdq_gelu_quant_work_bytes": (LL, [I]),
+        "svdq_w4a4_gemm_gelu_quant": (I, [I, I, I, I, P, P, P, P, P, P, P, F, P, P, F, F, P, P, P, P, LL, P, P]),
+        "svdq_mlp_workspace_bytes": (LL, [I, I, I, I]),
+        "svdq_w4a4_mlp_gelu": (I, [I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, F, P, P, F, P, P, P, P, LL, P,
+                                   P]),
         "svdq_noalloc_scratch_bytes": (LL, []),
         "svdq_w4a4_linear_noalloc": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, P]),
         "awq_pack_weights": (I, [I, I, P, P, P, P]),
@@ -261,6 +266,61 @@ def svdq_w4a4_linear_noalloc(precision, x, w, act_scale, bias=None, y=None, dev_
                                         float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), w["weight_scale_f"],
                                         _ptr(w["lora_up"]), _ptr(bias), _ptr(y), _ptr(dev_status),
                                         _stream(stream)))
+    return y
+
+
+def gelu_quant_work_bytes(M):
+    return int(lib.svdq_gelu_quant_work_bytes(M))
+
+
+def mlp_workspace_bytes(M, K, N_hidden, rank=SVDQ_RANK):
+    return int(lib.svdq_mlp_workspace_bytes(M, K, N_hidden, rank))
+
+
+def svdq_w4a4_gemm_gelu_quant(act_codes, act_scales, lora_act, w, alpha, w_next, next_act_scale, bias=None,
+                              out=None, work=None, dev_status=None, stream=None):
+    """The up layer's NVFP4 GEMM with the GELU-MLP epilogue.  w, w_next:
+    device dicts of the up layer and of the layer that consumes its GELU
+    output.  Returns that layer's (codes, scales, lora_act)."""
+    M = act_codes.shape[0]
+    N, K, rank = w["N"], w["K"], w["rank"]
+    if w_next["K"] != N:
+        raise SvdqError(2, f"next layer's K={w_next['K']} differs from N={N}")
+    dev = act_codes.device
+    if out is None:
+        out = (torch.empty((M, N // 2), dtype=torch.uint8, device=dev),
+               torch.empty(act_scale_bytes(SVDQ_NVFP4, M, N), dtype=torch.uint8, device=dev),
+               torch.empty((M, 2 * rank), dtype=torch.bfloat16, device=dev))
+    if work is None:
+        work = torch.empty(max(gelu_quant_work_bytes(M), 1), dtype=torch.uint8, device=dev)
+    codes, scales, lora = out
+    _check(lib.svdq_w4a4_gemm_gelu_quant(M, N, K, rank, _ptr(act_codes), _ptr(act_scales), _ptr(lora_act),
+                                         _ptr(w["codes"]), _ptr(w["scales"]), _ptr(w["lora_up"]), _ptr(bias),
+                                         float(alpha), _ptr(w_next["inv_smooth"]), _ptr(w_next["lora_down"]),
+                                         float(next_act_scale), w_next["weight_scale_f"], _ptr(codes), _ptr(scales),
+                                         _ptr(lora), _ptr(work), work.numel(), _ptr(dev_status), _stream(stream)))
+    return codes, scales, lora
+
+
+def svdq_w4a4_mlp_gelu(x, w_up, up_act_scale, w_down, down_act_scale, up_bias=None, down_bias=None, y=None,
+                       workspace=None, dev_status=None, stream=None):
+    """y = down(GELU(up(x))) with two NVFP4 svdq_w4a4 layers (device dicts)."""
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    N, rank = w_up["N"], w_up["rank"]
+    if w_up["K"] != K or w_down["K"] != N or w_down["N"] != K:
+        raise SvdqError(2, "layer shapes do not chain: up [K -> N], down [N -> K]")
+    if y is None:
+        y = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(mlp_workspace_bytes(M, K, N, rank), 1), dtype=torch.uint8, device=x.device)
+    _check(lib.svdq_w4a4_mlp_gelu(M, K, N, rank, _ptr(x), _ptr(w_up["inv_smooth"]), _ptr(w_up["lora_down"]),
+                                  float(up_act_scale), _ptr(w_up["codes"]), _ptr(w_up["scales"]),
+                                  w_up["weight_scale_f"], _ptr(w_up["lora_up"]), _ptr(up_bias),
+                                  _ptr(w_down["inv_smooth"]), _ptr(w_down["lora_down"]), float(down_act_scale),
+                                  _ptr(w_down["codes"]), _ptr(w_down["scales"]), w_down["weight_scale_f"],
+                                  _ptr(w_down["lora_up"]), _ptr(down_bias), _ptr(y), _ptr(workspace),
+                                  workspace.numel(), _ptr(dev_status), _stream(stream)))
     return y
 
 

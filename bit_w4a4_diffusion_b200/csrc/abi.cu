@@ -237,9 +237,11 @@ static bool use_pair_gemm() {
   return v && strcmp(v, "pair") == 0;
 }
 
+// gq != nullptr selects the GELU-MLP epilogue (single-CTA kernel; y unused).
 static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const void* act_scales, const void* lora_act,
                            const void* w_codes, const void* w_scales, const void* lora_up, const void* bias,
-                           float alpha, void* y, int* dev_status, cudaStream_t stream, bool pdl, int sms) {
+                           float alpha, void* y, int* dev_status, cudaStream_t stream, bool pdl, int sms,
+                           const GeluQuantParams* gq = nullptr) {
   GemmTmaps t;
   bool ok = true;
   ok &= encode_tmap_2d(&t.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_codes, K / 2, M, K / 2, 128, 128,
@@ -250,8 +252,11 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
                        128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
                        256, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
-                       CU_TENSOR_MAP_SWIZZLE_32B);
+  if (gq == nullptr)
+    ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
+                         CU_TENSOR_MAP_SWIZZLE_32B);
+  else
+    t.y = t.a;  // not read by the GELU-MLP epilogue
   if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
   GemmNvfp4Params p{};
   p.M = M;
@@ -263,6 +268,10 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
   p.alpha = alpha;
   p.dev_status = dev_status;
   p.timeout_ns = svdq_timeout_ns();
+  if (gq != nullptr) {
+    p.gq = *gq;
+    return check_cuda(launch_gemm_nvfp4_gelu(p, t, sms, stream, pdl), "gemm_nvfp4 (GELU-MLP epilogue) launch");
+  }
   if (use_pair_gemm()) {
     // CTA-pair kernel: half-tile boxes for B and [L2^T|L2^T], and the block
     // scales as 2D maps of 256-byte rows (8 rows = one 2 KB chunk group).
@@ -372,6 +381,159 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
                           static_cast<cudaStream_t>(stream), true, sms);
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), true, sms);
+}
+
+// ------------------------------------------------------------------ GELU-MLP fusion
+
+long long svdq_gelu_quant_work_bytes(int M) {
+  if (M <= 0) return -1;
+  const long long counters = round_up(round_up(M, 128) / 32 * 4, 256);
+  return counters + round_up((int64_t)M * SVDQ_RANK * 4, 256);
+}
+
+static bool nvfp4_scale_ok(float s) { return s >= 0x1p-100f && s < 0x1p100f; }
+
+// Zero the work buffer and the scale rows no tile of the fused GEMM writes
+// (the tiled layout pads rows to 256, the tiles cover a multiple of 128).
+static int gelu_quant_prepare(int M, int N, void* next_act_scales, void* work, cudaStream_t stream) {
+  if (int s = check_cuda(cudaMemsetAsync(work, 0, svdq_gelu_quant_work_bytes(M), stream), "work memset")) return s;
+  const int64_t covered = round_up(M, 128), padded = round_up(M, 256);
+  if (padded > covered) {
+    const int64_t block = (int64_t)(N / 64) * 512;  // one 128-row block of scales
+    uint8_t* base = static_cast<uint8_t*>(next_act_scales) + covered / 128 * block;
+    if (int s = check_cuda(cudaMemsetAsync(base, 0, (size_t)block, stream), "scale padding memset")) return s;
+  }
+  return SVDQ_OK;
+}
+
+static GeluQuantParams gelu_quant_params(int M, const float* next_inv_smooth, const void* next_lora_down,
+                                         float next_act_scale, float next_weight_scale, void* next_act_codes,
+                                         void* next_act_scales, void* next_lora_act, void* work) {
+  GeluQuantParams g{};
+  g.inv_smooth = next_inv_smooth;
+  g.l1t = static_cast<const uint16_t*>(next_lora_down);
+  g.s_d = next_act_scale;
+  // h_hat enters the fp16 down-projection as h_hat * 2^-e (the rule of
+  // svdq_quantize_act: 2688 s maps into [2^12, 2^13)).
+  int ex = 0;
+  frexpf(2688.0f * next_act_scale, &ex);
+  const int e = ex - 1 - 12;
+  g.lr_in_scale = ldexpf(1.0f, -e);
+  g.lora_scale = ldexpf(1.0f, e) / (next_act_scale * next_weight_scale);
+  g.codes = static_cast<uint8_t*>(next_act_codes);
+  g.scales = static_cast<uint8_t*>(next_act_scales);
+  g.lora_act = static_cast<uint16_t*>(next_lora_act);
+  uint8_t* w = static_cast<uint8_t*>(work);
+  g.counters = reinterpret_cast<unsigned int*>(w);
+  g.u_work = reinterpret_cast<float*>(w + round_up(round_up(M, 128) / 32 * 4, 256));
+  return g;
+}
+
+static int check_gelu_quant_args(int M, int N, int K, int rank, float alpha, const float* next_inv_smooth,
+                                 const void* next_lora_down, float next_act_scale, float next_weight_scale,
+                                 void* next_act_codes, void* next_act_scales, void* next_lora_act, void* work,
+                                 long long work_bytes) {
+  if (int s = check_gemm_args(SVDQ_NVFP4, M, N, K, rank)) return s;
+  if (N % 256 != 0)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d must be a multiple of 256 (it is the next layer's K)", N);
+  if (!next_inv_smooth || !next_lora_down || !next_act_codes || !next_act_scales || !next_lora_act || !work)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(next_inv_smooth) || !aligned16(next_lora_down) || !aligned16(next_act_codes) ||
+      !aligned16(next_act_scales) || !aligned16(next_lora_act) || !aligned16(work))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
+  if (!nvfp4_scale_ok(next_act_scale) || !nvfp4_scale_ok(next_weight_scale))
+    return fail(SVDQ_ERR_INVALID_ARG, "NVFP4 tensor scales must lie in [2^-100, 2^100) (act %g, weight %g)",
+                next_act_scale, next_weight_scale);
+  const long long need = svdq_gelu_quant_work_bytes(M);
+  if (work_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "work buffer of %lld bytes is smaller than the %lld needed", work_bytes, need);
+  return SVDQ_OK;
+}
+
+int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                              const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                              const void* bias, float alpha, const float* next_inv_smooth,
+                              const void* next_lora_down, float next_act_scale, float next_weight_scale,
+                              void* next_act_codes, void* next_act_scales, void* next_lora_act, void* work,
+                              long long work_bytes, int* dev_status, void* stream) {
+  if (int s = check_gelu_quant_args(M, N, K, rank, alpha, next_inv_smooth, next_lora_down, next_act_scale,
+                                    next_weight_scale, next_act_codes, next_act_scales, next_lora_act, work,
+                                    work_bytes))
+    return s;
+  if (!act_codes || !act_scales || !lora_act || !w_codes || !w_scales || !lora_up)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lora_act) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(lora_up) || (bias && !aligned16(bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int s = gelu_quant_prepare(M, N, next_act_scales, work, st)) return s;
+  const GeluQuantParams g = gelu_quant_params(M, next_inv_smooth, next_lora_down, next_act_scale, next_weight_scale,
+                                              next_act_codes, next_act_scales, next_lora_act, work);
+  return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, nullptr,
+                         dev_status, st, false, sms, &g);
+}
+
+long long svdq_mlp_workspace_bytes(int M, int K, int N_hidden, int rank) {
+  const long long a = svdq_workspace_bytes(SVDQ_NVFP4, M, K, rank);
+  const long long h = svdq_workspace_bytes(SVDQ_NVFP4, M, N_hidden, rank);
+  const long long w = svdq_gelu_quant_work_bytes(M);
+  if (a < 0 || h < 0 || w < 0) return -1;
+  return a + h + w;
+}
+
+int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, const float* up_inv_smooth,
+                       const void* up_lora_down, float up_act_scale, const void* up_w_codes, const void* up_w_scales,
+                       float up_weight_scale, const void* up_lora_up, const void* up_bias,
+                       const float* down_inv_smooth, const void* down_lora_down, float down_act_scale,
+                       const void* down_w_codes, const void* down_w_scales, float down_weight_scale,
+                       const void* down_lora_up, const void* down_bias, void* y, void* workspace,
+                       long long workspace_bytes, int* dev_status, void* stream) {
+  const int N = N_hidden;
+  if (int s = check_gemm_args(SVDQ_NVFP4, M, K, N, rank)) return s;  // the down layer: [M, N] -> [M, K]
+  if (!workspace) return fail(SVDQ_ERR_INVALID_ARG, "null workspace");
+  const long long need = svdq_mlp_workspace_bytes(M, K, N, rank);
+  if (need < 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d N_hidden=%d", M, K, N);
+  if (workspace_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* a_codes = ws;
+  uint8_t* a_scales = a_codes + round_up((int64_t)M * (K / 2), 256);
+  uint8_t* a_lora = a_scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, K), 256);
+  uint8_t* h_codes = a_lora + round_up((int64_t)M * 2 * rank * 2, 256);
+  uint8_t* h_scales = h_codes + round_up((int64_t)M * (N / 2), 256);
+  uint8_t* h_lora = h_scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, N), 256);
+  uint8_t* work = h_lora + round_up((int64_t)M * 2 * rank * 2, 256);
+  const float up_alpha = up_act_scale * up_weight_scale;
+  if (int s = check_gelu_quant_args(M, N, K, rank, up_alpha, down_inv_smooth, down_lora_down, down_act_scale,
+                                    down_weight_scale, h_codes, h_scales, h_lora, work,
+                                    svdq_gelu_quant_work_bytes(M)))
+    return s;
+  if (!up_w_codes || !up_w_scales || !up_lora_up || !down_w_codes || !down_w_scales || !down_lora_up || !y)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(up_w_codes) || !aligned16(up_w_scales) || !aligned16(up_lora_up) || !aligned16(down_w_codes) ||
+      !aligned16(down_w_scales) || !aligned16(down_lora_up) || !aligned16(y) || (up_bias && !aligned16(up_bias)) ||
+      (down_bias && !aligned16(down_bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The memsets go first so that quantize -> fused GEMM -> down GEMM form one
+  // chain of programmatic dependent launches.
+  if (int s = gelu_quant_prepare(M, N, h_scales, work, st)) return s;
+  if (int s = svdq_quantize_act(SVDQ_NVFP4, M, K, rank, x, up_inv_smooth, up_lora_down, up_act_scale,
+                                up_weight_scale, a_codes, a_scales, a_lora, stream))
+    return s;
+  const GeluQuantParams g = gelu_quant_params(M, down_inv_smooth, down_lora_down, down_act_scale, down_weight_scale,
+                                              h_codes, h_scales, h_lora, work);
+  if (int s = gemm_nvfp4_impl(M, N, K, a_codes, a_scales, a_lora, up_w_codes, up_w_scales, up_lora_up, up_bias,
+                              up_alpha, nullptr, dev_status, st, true, sms, &g))
+    return s;
+  return gemm_nvfp4_impl(M, K, N, h_codes, h_scales, h_lora, down_w_codes, down_w_scales, down_lora_up, down_bias,
+                         down_act_scale * down_weight_scale, y, dev_status, st, true, sms);
 }
 
 int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, const void* scales, const void* zeros,

@@ -93,6 +93,55 @@ constexpr uint32_t IDESC_BF16 =
 SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
 
+// ------------------------------------------------------- GELU-MLP epilogue helpers
+// Exact (erf) GELU: v Phi(v) = v (1 + erf(v / sqrt 2)) / 2.
+SVDQ_DEV float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+
+SVDQ_DEV uint32_t half2_bits(float lo, float hi) {
+  uint32_t out;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(out) : "f"(lo), "f"(hi));
+  return out;  // lo in the low half
+}
+
+SVDQ_DEV void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+SVDQ_DEV uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// D (fp32) += A (16 x 16 fp16, row) * B (16 x 8 fp16, col).
+SVDQ_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+SVDQ_DEV void red_add_f32x2(float* addr, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// Byte offset of scale (row, group) in the tiled NVFP4 scale layout.
+SVDQ_DEV size_t tiled_scale_offset(int row, int group, int K) {
+  return ((size_t)(row >> 7) * (K / 64) + (group >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
+}
+
+// 16-byte segment s (fp16 columns 8s..8s+7) of row r in a warp's 32 x 32
+// fp16 staging tile (64-byte rows; segments XOR-ed with (r / 2) mod 4 so that
+// both the row-per-lane stores and the fragment loads are conflict-free).
+SVDQ_DEV uint32_t hseg(uint32_t base, int r, int s) {
+  return base + (uint32_t)r * 64u + (uint32_t)((s ^ ((r >> 1) & 3)) << 4);
+}
+
+template <bool kGelu>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
@@ -131,7 +180,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_la);
     prefetch_tmap(&tm_lb);
-    prefetch_tmap(&tm_y);
+    if (!kGelu) prefetch_tmap(&tm_y);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -299,6 +348,178 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->sf_drain), 0, drain_ctx, kDevTimeoutDrain);
     }
+  } else if constexpr (kGelu) {
+    // ------------------------------------------------------ GELU-MLP epilogue
+    // Same TMEM schedule as the plain epilogue below.  Per 32-column chunk
+    // each lane (one row) forms h_hat = GELU(alpha D + b) * inv_lambda_down
+    // in fp32, quantizes its two 16-groups with the down layer's NVFP4 rule
+    // (16 bytes of codes, 2 scale bytes), and stages fp16(h_hat 2^-e) in a
+    // 32 x 32 shared tile from which the warp accumulates its 32 rows x 32
+    // ranks of the down layer's low-rank projection on mma.sync.  Lane (g, c)
+    // takes fp16 columns 8c..8c+3 as k-step 0 and 8c+4..8c+7 as k-step 1 (a
+    // permutation of k shared by both operands), so each of its A and B
+    // fragments is one 16-byte load.  After the tile, the partial sums go to
+    // u_work with vector reductions; the warp that completes a 32-row block's
+    // count of N tiles converts those rows to the bf16 hi/lo lora_act.
+    const int q = warp & 3;
+    const int g = lane >> 2, c = lane & 3;
+    const GeluQuantParams& gq = p.gq;
+    const uint32_t hbase = smem_u32(epi_base + (warp - 2) * 2048);
+    const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
+    const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
+    uint32_t acc_phase = 0;
+    int it = 0;
+    constexpr int LDC = 32;
+    constexpr int NCH = BN / LDC;
+    constexpr int NSH = (ACC_OVERLAP + LDC - 1) / LDC;
+    constexpr int NBUF = 3;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int m0 = (tile % tiles_m) * BM;
+      const int n0 = (tile / tiles_m) * BN;
+      const int b = it & 1;
+      const int row = m0 + 32 * q + lane;
+      const bool row_ok = row < p.M;
+      float lacc[2][4][4];
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lacc[t][j][e] = 0.f;
+      const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+      auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NSH) % NCH : i; };
+      uint32_t rb[NBUF][32];
+#pragma unroll
+      for (int i = 0; i < NBUF; ++i) tmem_ld_32x32b_x32(acc_base + chunk_col(i) * LDC, rb[i]);
+      tmem_ld_wait(rb[0]);
+      reg_fence(rb[1]);
+      reg_fence(rb[2]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        uint32_t(&r)[32] = rb[i % NBUF];
+        if (i >= NBUF && i % NBUF == 0) {
+          tmem_ld_wait(rb[0]);
+          reg_fence(rb[1]);
+          reg_fence(rb[2]);
+        }
+        const int n = n0 + chunk_col(i) * LDC;
+        // h_hat in place of the accumulator values (zero for rows past M, so
+        // their scales come out zero and they add nothing).
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const uint4 bw = p.bias != nullptr ? __ldg(reinterpret_cast<const uint4*>(p.bias + n) + k8)
+                                             : make_uint4(0, 0, 0, 0);
+          const float4 i0 = __ldg(reinterpret_cast<const float4*>(gq.inv_smooth + n) + 2 * k8);
+          const float4 i1 = __ldg(reinterpret_cast<const float4*>(gq.inv_smooth + n) + 2 * k8 + 1);
+          const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+          const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float bias_v = __uint_as_float((j & 1) ? (bb[j >> 1] & 0xFFFF0000u) : (bb[j >> 1] << 16));
+            const float v = __fmaf_rn(p.alpha, __uint_as_float(r[8 * k8 + j]), bias_v);
+            const float h = __fmul_rn(gelu_erf(v), il[j]);
+            r[8 * k8 + j] = __float_as_uint(row_ok ? h : 0.f);
+          }
+        }
+        // NVFP4 quantization of the two 16-groups (the down layer's rule).
+        uint32_t cw[4], sbs = 0;
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          float a = 0.f;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) a = fmaxf(a, fabsf(__uint_as_float(r[16 * grp + k])));
+          const uint32_t sb = cvt_e4m3(__fmul_rn(a, inv_six_s));
+          const float d = __fmul_rn(e4m3_to_f32(sb), gq.s_d);
+          uint32_t w0 = 0, w1 = 0;
+          if (d != 0.f) {
+            const float rr = __frcp_rn(d);
+            const float2 r2 = make_float2(rr, rr);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 t0 = __fmul2_rn(
+                  make_float2(__uint_as_float(r[16 * grp + 2 * k]), __uint_as_float(r[16 * grp + 2 * k + 1])), r2);
+              const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[16 * grp + 8 + 2 * k]),
+                                                       __uint_as_float(r[16 * grp + 9 + 2 * k])),
+                                           r2);
+              w0 |= cvt_e2m1x2(t0.x, t0.y) << (8 * k);
+              w1 |= cvt_e2m1x2(t1.x, t1.y) << (8 * k);
+            }
+          }
+          cw[2 * grp] = w0;
+          cw[2 * grp + 1] = w1;
+          sbs |= sb << (8 * grp);
+        }
+        if (row_ok)
+          *reinterpret_cast<uint4*>(gq.codes + (size_t)row * (p.N / 2) + n / 2) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint16_t*>(gq.scales + tiled_scale_offset(row, n / 16, p.N)) = (uint16_t)sbs;
+        // fp16(h_hat 2^-e) into the staging tile, row = lane.
+#pragma unroll
+        for (int sg = 0; sg < 4; ++sg) {
+          uint32_t hv[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 t =
+                __fmul2_rn(make_float2(__uint_as_float(r[8 * sg + 2 * k]), __uint_as_float(r[8 * sg + 2 * k + 1])), lr2);
+            hv[k] = half2_bits(t.x, t.y);
+          }
+          st_shared_v4(hseg(hbase, lane, sg), make_uint4(hv[0], hv[1], hv[2], hv[3]));
+        }
+        __syncwarp();
+        uint4 x0[2], x1[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          x0[t] = ld_shared_v4(hseg(hbase, 16 * t + g, c));
+          x1[t] = ld_shared_v4(hseg(hbase, 16 * t + 8 + g, c));
+        }
+        __syncwarp();  // every lane's loads precede the next chunk's stores
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 bq = __ldg(reinterpret_cast<const uint4*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 8 * c));
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            mma_16816(lacc[t][j], x0[t].x, x1[t].x, x0[t].y, x1[t].y, bq.x, bq.y);
+            mma_16816(lacc[t][j], x0[t].z, x1[t].z, x0[t].w, x1[t].w, bq.z, bq.w);
+          }
+        }
+        // Refill the block just converted with the chunk three ahead.
+        if (i + NBUF < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + NBUF) * LDC, r);
+      }
+      // The tile's low-rank partial: rows 16t + g (+8), ranks 8j + 2c (+1).
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r0 = m0 + 32 * q + 16 * t + g;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = 8 * j + 2 * c;
+          if (r0 < p.M) red_add_f32x2(gq.u_work + (size_t)r0 * 32 + col, lacc[t][j][0], lacc[t][j][1]);
+          if (r0 + 8 < p.M) red_add_f32x2(gq.u_work + (size_t)(r0 + 8) * 32 + col, lacc[t][j][2], lacc[t][j][3]);
+        }
+      }
+      __threadfence();
+      __syncwarp();
+      unsigned int prev = 0;
+      if (lane == 0) prev = atomicAdd(gq.counters + (m0 + 32 * q) / 32, 1u);
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev == (unsigned int)(tiles_n - 1)) {
+        // Every N tile of these 32 rows has added its partial.
+        __threadfence();
+        const int rbase = m0 + 32 * q;
+        for (int rr = 0; rr < 32 && rbase + rr < p.M; ++rr) {
+          const float uf = __fmul_rn(__ldcg(gq.u_work + (size_t)(rbase + rr) * 32 + lane), gq.lora_scale);
+          const __nv_bfloat16 hi = __float2bfloat16_rn(uf);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(uf, __bfloat162float(hi)));
+          gq.lora_act[(size_t)(rbase + rr) * 64 + lane] = __bfloat16_as_ushort(hi);
+          gq.lora_act[(size_t)(rbase + rr) * 64 + 32 + lane] = __bfloat16_as_ushort(lo);
+        }
+      }
+      acc_phase ^= 1;
+    }
   } else {
     // -------------------------------------------------------------- epilogue
     // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile,
@@ -408,12 +629,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
-                              bool pdl) {
+namespace {
+template <bool kGelu>
+cudaError_t launch_impl(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream, bool pdl) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<kGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -428,7 +650,18 @@ cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, t.a, t.b, t.la, t.lb, t.y, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel<kGelu>, t.a, t.b, t.la, t.lb, t.y, p);
+}
+}  // namespace
+
+cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                              bool pdl) {
+  return launch_impl<false>(p, t, num_sms, stream, pdl);
+}
+
+cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                                   bool pdl) {
+  return launch_impl<true>(p, t, num_sms, stream, pdl);
 }
 
 }  // namespace svdq

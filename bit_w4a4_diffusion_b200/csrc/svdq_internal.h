@@ -33,6 +33,22 @@ cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_
 cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_l1t,
                                   int* dev_status, unsigned long long timeout_ns, cudaStream_t stream);
 
+// The GELU-MLP epilogue: the up layer's output never leaves the chip; the
+// epilogue applies GELU and the down layer's smoothing, quantizer and
+// low-rank down-projection (partial sums over N tiles reduced in u_work).
+struct GeluQuantParams {
+  const float* inv_smooth;    // down layer 1/lambda, fp32 [N]
+  const uint16_t* l1t;        // down layer lora_down, fp16 [32, N]
+  float s_d;                  // down layer activation tensor scale
+  float lr_in_scale;          // 2^-e applied before the fp16 conversion
+  float lora_scale;           // 2^e / (s_d s_w_down)
+  uint8_t* codes;             // [M, N/2]
+  uint8_t* scales;            // tiled e4m3 with K = N, rows padded to 256
+  uint16_t* lora_act;         // bf16 [M, 64] (hi | lo)
+  float* u_work;              // fp32 [M, 32], zero at launch
+  unsigned int* counters;     // one per 32 rows, zero at launch
+};
+
 struct GemmNvfp4Params {
   int M, N, K;
   const uint8_t* act_scales;  // tiled e4m3, rows padded to 256
@@ -41,6 +57,7 @@ struct GemmNvfp4Params {
   float alpha;                // s_a * s_w
   int* dev_status;            // may be null
   unsigned long long timeout_ns;
+  GeluQuantParams gq;         // used by the GELU-MLP epilogue only
 };
 
 struct GemmTmaps {
@@ -49,6 +66,9 @@ struct GemmTmaps {
 
 cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                               bool pdl);
+// Same mainloop, GELU-MLP epilogue (t.y unused).
+cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                                   bool pdl);
 
 // The CTA-pair kernel: B and [L2^T|L2^T] boxes are 128 rows (half a tile),
 // block scales are read through 2D maps of 256-byte rows (box 256 x 8).

@@ -191,6 +191,59 @@ int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const
                              float weight_scale, const void* lora_up, const void* bias, void* y, int* dev_status,
                              void* stream);
 
+/* ------------------------------------------------------------------ GELU-MLP fusion
+ * "Nunchaku Lite" docs, section "Fused kernels": the original engine runs a
+ * diffusion transformer's MLP (up projection, GELU, down projection) with a
+ * fused GELU kernel.
+ *
+ * svdq_w4a4_gemm_gelu_quant: the up layer's NVFP4 GEMM (svdq_w4a4_gemm's
+ * arguments up to alpha) whose output
+ *   v = alpha * ( sum_k deq(a) deq(w) + lora_act . lora_up^T ) + bias      (fp32)
+ * is never stored: it goes through h = GELU(v) = v Phi(v) (the exact erf
+ * form), the NEXT layer's smoothing h_hat = h * next_inv_smooth[n] and the
+ * next layer's activation side exactly as svdq_quantize_act defines it for
+ * NVFP4 with s_a = next_act_scale: E2M1 codes with an E4M3 scale per 16
+ * (written to next_act_codes [M, N/2] and next_act_scales,
+ * svdq_act_scale_bytes(SVDQ_NVFP4, M, N) bytes, padding rows zero) and the
+ * low-rank activation next_lora_act bf16 [M, 2r] = [hi | lo] of
+ * (h_hat L1_next) / (next_act_scale * next_weight_scale), computed on fp16
+ * operands (h_hat * 2^-e with 2^e as in svdq_quantize_act, and
+ * next_lora_down [r, N] as packed) with fp32 accumulation.  The sum over N of
+ * the low-rank partials uses fp32 atomic adds, so next_lora_act can differ
+ * between runs in its last bits; codes and scales are deterministic.
+ * `work` is device scratch of svdq_gelu_quant_work_bytes(M) bytes that the
+ * call zeroes on `stream` before use; calls sharing it must not overlap.
+ * The outputs feed svdq_w4a4_gemm of the next layer directly.
+ * Shapes: M >= 1, N % 256 == 0 (N is the next layer's K), K % 256 == 0,
+ * rank == SVDQ_RANK.  NVFP4 only; scales in [2^-100, 2^100). */
+long long svdq_gelu_quant_work_bytes(int M);
+int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                              const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                              const void* bias, float alpha, const float* next_inv_smooth,
+                              const void* next_lora_down, float next_act_scale, float next_weight_scale,
+                              void* next_act_codes, void* next_act_scales, void* next_lora_act, void* work,
+                              long long work_bytes, int* dev_status, void* stream);
+
+/* svdq_w4a4_mlp_gelu: the MLP block y = down(GELU(up(x))) with two NVFP4
+ * svdq_w4a4 layers, up: [M, K] -> [M, N_hidden], down: [M, N_hidden] ->
+ * [M, K]: svdq_quantize_act of x for the up layer, then
+ * svdq_w4a4_gemm_gelu_quant, then the down layer's svdq_w4a4_gemm, all on
+ * `stream` (the GEMMs with programmatic dependent launch).  Each layer's
+ * arguments are those of svdq_w4a4_linear (inv_smooth, lora_down, act_scale,
+ * w_codes, w_scales, weight_scale, lora_up, bias as packed).  x and y are
+ * bf16 [M, K]; `workspace` is device memory of at least
+ * svdq_mlp_workspace_bytes(M, K, N_hidden, rank) bytes holding both layers'
+ * quantized activations and the fused GEMM's work buffer; calls sharing it
+ * must not overlap.  Shapes: K % 256 == 0, N_hidden % 256 == 0. */
+long long svdq_mlp_workspace_bytes(int M, int K, int N_hidden, int rank);
+int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, const float* up_inv_smooth,
+                       const void* up_lora_down, float up_act_scale, const void* up_w_codes, const void* up_w_scales,
+                       float up_weight_scale, const void* up_lora_up, const void* up_bias,
+                       const float* down_inv_smooth, const void* down_lora_down, float down_act_scale,
+                       const void* down_w_codes, const void* down_w_scales, float down_weight_scale,
+                       const void* down_lora_up, const void* down_bias, void* y, void* workspace,
+                       long long workspace_bytes, int* dev_status, void* stream);
+
 /* ------------------------------------------------------------------ AWQ W4A16
  * "Nunchaku Lite" docs, "Supported quantization types" table: awq_w4a16,
  * int4, group size 64 -- an INT4 weight-only AWQ-style kernel for the

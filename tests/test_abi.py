@@ -87,3 +87,38 @@ def test_awq_validation():
     assert B.lib.awq_w4a16_linear(4, 100, 256, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == 2
     assert B.lib.awq_w4a16_linear(4, 128, 100, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == 2
     assert B.lib.awq_w4a16_linear(4, 128, 256, None, FAKE, FAKE, FAKE, None, FAKE, None) == 1
+
+
+def test_gelu_mlp_sizes():
+    # counters (one uint32 per 32 rows of the 128-row tiles) + fp32 [M, 32], each rounded to 256 bytes
+    assert B.gelu_quant_work_bytes(4096) == 512 + 4096 * 32 * 4
+    assert B.gelu_quant_work_bytes(300) == 256 + 300 * 128 + (-300 * 128) % 256
+    assert B.gelu_quant_work_bytes(0) == -1
+    assert B.mlp_workspace_bytes(4096, 3072, 12288) == (B.workspace_bytes("nvfp4", 4096, 3072) +
+                                                         B.workspace_bytes("nvfp4", 4096, 12288) +
+                                                         B.gelu_quant_work_bytes(4096))
+
+
+@pytest.mark.parametrize("M,N,K,rank,status", [
+    (64, 384, 256, 32, 2),      # N (the next layer's K) not a multiple of 256
+    (64, 256, 200, 32, 2),      # K not a multiple of 256
+    (0, 256, 256, 32, 2),       # M = 0
+    (64, 256, 256, 8, 2),       # unsupported rank
+])
+def test_gemm_gelu_quant_validation(M, N, K, rank, status):
+    P = ctypes.c_void_p
+    args = [M, N, K, rank] + [P(FAKE)] * 7 + [ctypes.c_float(1.0), P(FAKE), P(FAKE), ctypes.c_float(1.0),
+                                               ctypes.c_float(1.0)] + [P(FAKE)] * 4 + [1 << 30, None, None]
+    assert B.lib.svdq_w4a4_gemm_gelu_quant(*args) == status
+
+
+def test_gemm_gelu_quant_rejects_small_work_and_bad_scale():
+    P = ctypes.c_void_p
+    base = [64, 256, 256, 32] + [P(FAKE)] * 7 + [ctypes.c_float(1.0), P(FAKE), P(FAKE)]
+    tail = [P(FAKE)] * 4
+    ok_scales = [ctypes.c_float(1.0), ctypes.c_float(1.0)]
+    assert B.lib.svdq_w4a4_gemm_gelu_quant(*(base + ok_scales + tail + [16, None, None])) == 1
+    assert b"work buffer" in B.lib.svdq_last_error()
+    assert B.lib.svdq_w4a4_gemm_gelu_quant(*(base + [ctypes.c_float(0.0), ctypes.c_float(1.0)] + tail +
+                                             [1 << 30, None, None])) == 1
+    assert b"tensor scales" in B.lib.svdq_last_error()

@@ -1,0 +1,209 @@
+"""GPU parity of the GELU-MLP fusion against the CPU oracle.
+
+The fused up-projection epilogue decides the next layer's NVFP4 codes and
+scales from its own fp32 GEMM output, which differs from the oracle's fp64
+value by rounding.  Codes and scales are therefore checked with
+``helpers.check_nvfp4_near_boundary``: every decision must be a correct
+rounding of a value within a stated error of the exact one, and the
+decisions that differ from the oracle's own must be rare.  The low-rank
+activation and the MLP output are compared within tolerances.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import mlp as OM
+from oracle import svdq as O
+from tests.helpers import check_nvfp4_near_boundary, nibbles, output_errors
+
+pytestmark = pytest.mark.gpu
+
+# Error bound on the fused epilogue's h_hat, per element.  The GEMM output v
+# differs from the oracle's exact value mainly through the low-rank branch:
+# its down-projection runs on fp16 operands, so each x_hat * 2^-e carries a
+# relative rounding error of at most 2^-11, which bounds the error of
+# x_hat L1 L2 by 2^-11 |x_hat| |L1| |L2| (elementwise absolute values); the
+# rest (the bf16 hi/lo split of u, fp32 accumulation) is a few 1e-6 of
+# rms(v).  GELU' is at most 1.13 in magnitude, and GELU and the smoothing
+# product add a few fp32 ulps of h_hat.
+V_ACC_ERR = 1e-5         # of rms(v)
+GELU_SLOPE = 1.13
+H_REL_ERR = 4e-6         # of |h_hat|
+MAX_FLIPPED = 2e-3       # fraction of codes allowed to differ from the oracle's
+
+# The MLP output inherits those flips: a hidden code that takes the
+# neighbouring E2M1 value moves its element by up to a third of the group's
+# max |h_hat| (the step from 4 to 6 at scale max/6), and that element's
+# column of the down layer's weight carries it into every output.  At the
+# 0.06% of flipped codes seen on the workloads below this gives a relative L2
+# difference of about 6e-3 and single outputs off by up to 0.12 rms(y) against
+# the oracle evaluated on its own codes; the bounds leave room for the allowed
+# fraction.  Exactness of the down layer itself is covered by the layer tests.
+MLP_REL_L2_TOL = 1.5e-2
+MLP_MAX_ABS_TOL = 0.5    # in units of rms(y_ref)
+
+
+def _assert_mlp_close(y_gpu, y_ref, what):
+    rel, excess = output_errors(y_gpu, y_ref)
+    assert np.all(np.isfinite(y_gpu)), f"{what}: non-finite outputs"
+    assert rel <= MLP_REL_L2_TOL, f"{what}: relative L2 error {rel:.3e} > {MLP_REL_L2_TOL}"
+    assert excess <= MLP_MAX_ABS_TOL, f"{what}: max-abs excess {excess:.3e} rms > {MLP_MAX_ABS_TOL}"
+
+
+def _lib():
+    import bit_w4a4_diffusion_b200 as B
+    return B
+
+
+def _mlp_case(M, K, N, seed_shift=0):
+    up = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M, K=K, N=N), bias_std=0.1)
+    down = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M, K=N, N=K), bias_std=0.05)
+    return up, down
+
+
+def _setup(up_case, down_case):
+    B = _lib()
+    iu = wl.make_svdq_inputs(up_case)
+    idn = wl.make_svdq_inputs(down_case)
+    pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
+    pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
+    return iu, idn, pk_u, pk_d, B.to_device(pk_u), B.to_device(pk_d)
+
+
+def _h_delta(v, x_hat, L1, L2, inv_lam_d):
+    rms = np.sqrt(np.mean(v ** 2))
+    lowrank = 2.0 ** -11 * (np.abs(x_hat.astype(np.float64)) @ np.abs(L1.astype(np.float64))) @ \
+        np.abs(L2.astype(np.float64))
+    dv = lowrank + V_ACC_ERR * rms
+    inv = inv_lam_d.astype(np.float64)[None, :]
+    return GELU_SLOPE * dv * inv + H_REL_ERR * np.abs(OM.gelu(v) * inv)
+
+
+def _check_hidden(iu, idn, pk_u, pk_d, codes, scales, lora, rows=None):
+    """The fused epilogue's outputs for `rows` (all if None) against the oracle."""
+    B = _lib()
+    M, N = iu.case.M, iu.case.N
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    ref_u = O.pack_weights("nvfp4", iu.W, iu.lam, iu.L1, iu.L2)
+    act_u = O.quantize_activations("nvfp4", iu.x[sel], ref_u["inv_lam"], np.float32(iu.act_scale))
+    v = OM.up_output_f64(act_u, ref_u, iu.L1, iu.L2, iu.bias)
+    inv_d = O.inverse_smoothing(idn.lam)
+    s_d = np.float32(idn.act_scale)
+    h = OM.gelu_requantize(v, inv_d, s_d)
+    got_codes = nibbles(codes.cpu().numpy())[sel]
+    got_scales = B.scales_to_rowmajor(scales.cpu().numpy(), M, N)[sel]
+    delta = _h_delta(v, act_u["x_hat"], iu.L1, iu.L2, inv_d)
+    flipped = check_nvfp4_near_boundary(h["x_hat"], s_d, got_codes, got_scales, delta)
+    assert flipped <= MAX_FLIPPED, f"{flipped:.2e} of the codes differ from the oracle's"
+    # padding rows of the tiled scale layout are zero
+    Mp = (M + 255) // 256 * 256
+    if Mp > M and rows is None:
+        full = B.scales_to_rowmajor(scales.cpu().numpy(), Mp, N)
+        assert np.all(full[M:] == 0)
+    # low-rank activation (fp16 operands, fp32 accumulation): as for the quantize kernel
+    la = lora.float().cpu().numpy().astype(np.float64)[sel]
+    u = OM.lora_act(h["x_hat"], idn.L1, s_d, np.float32(pk_d["weight_scale"][0]))
+    err = np.abs(la[:, :32] + la[:, 32:] - u)
+    assert np.max(err) <= 2e-3 * np.max(np.abs(u)) + 1e-30, f"low-rank activation error {np.max(err)}"
+    assert np.linalg.norm(err) <= 5e-4 * np.linalg.norm(u) + 1e-30
+    return v, h
+
+
+SMALL = [
+    (300, 1024, 512),     # ragged M: scale padding rows past the last tile
+    (129, 256, 256),      # one row past a tile, a single N tile
+    (1, 512, 768),        # a single token
+    (512, 768, 1024),     # several tiles in both directions
+]
+
+
+@pytest.mark.parametrize("M,K,N", SMALL)
+def test_fused_gelu_quant_matches_oracle(M, K, N):
+    B = _lib()
+    up_case, down_case = _mlp_case(M, K, N)
+    iu, idn, pk_u, pk_d, wu, wd = _setup(up_case, down_case)
+    x = B.bits_to_bf16(iu.x_bits, "cuda")
+    b_u = B.bits_to_bf16(iu.bias_bits, "cuda")
+    s_a = float(iu.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wu["inv_smooth"], wu["lora_down"], s_a, wu["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk_u["weight_scale"][0])))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hc, hs, hl = B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, alpha, wd, float(idn.act_scale), bias=b_u,
+                                             dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    v, h = _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl)
+
+    # the down layer on the fused outputs, and the one-call MLP
+    b_d = B.bits_to_bf16(idn.bias_bits, "cuda")
+    alpha_d = float(np.float32(np.float32(idn.act_scale) * np.float32(pk_d["weight_scale"][0])))
+    y = B.svdq_w4a4_gemm("nvfp4", hc, hs, hl, wd, alpha_d, bias=b_d)
+    y2 = B.svdq_w4a4_mlp_gelu(x, wu, s_a, wd, float(idn.act_scale), up_bias=b_u, down_bias=b_d,
+                              dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_d = O.pack_weights("nvfp4", idn.W, idn.lam, idn.L1, idn.L2)
+    y64 = O.linear_f64("nvfp4", h, ref_d, idn.L1, idn.L2, idn.bias)
+    _assert_mlp_close(y.float().cpu().numpy(), y64, f"MLP {M}x{K}x{N}")
+    _assert_mlp_close(y2.float().cpu().numpy(), y64, f"one-call MLP {M}x{K}x{N}")
+    # The two paths differ only through the atomic order of the low-rank sums.
+    d = (y2.float() - y.float()).abs().max().item()
+    assert d <= 1e-2 * y.float().abs().max().item()
+
+
+def test_fused_codes_are_deterministic():
+    """Codes and scales do not depend on the order of the atomic low-rank sums."""
+    B = _lib()
+    up_case, down_case = _mlp_case(384, 512, 1024)
+    iu, idn, pk_u, pk_d, wu, wd = _setup(up_case, down_case)
+    x = B.bits_to_bf16(iu.x_bits, "cuda")
+    s_a = float(iu.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wu["inv_smooth"], wu["lora_down"], s_a, wu["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk_u["weight_scale"][0])))
+    outs = [B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, alpha, wd, float(idn.act_scale)) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1])
+        # lora_act = hi + lo of the low-rank sum, whose fp32 atomic order varies
+        u0 = outs[0][2].double()[:, :32] + outs[0][2].double()[:, 32:]
+        u1 = o[2].double()[:, :32] + o[2].double()[:, 32:]
+        assert (u1 - u0).abs().max().item() <= 1e-5 * u0.abs().max().item()
+
+
+def test_fused_rejects_bad_shapes_before_launch():
+    B = _lib()
+    up_case, down_case = _mlp_case(64, 256, 384)        # N = 384 is not a multiple of 256
+    iu = wl.make_svdq_inputs(up_case)
+    pk = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
+    wu = B.to_device(pk)
+    fake_next = dict(wu, K=384)
+    x = B.bits_to_bf16(iu.x_bits, "cuda")
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wu["inv_smooth"], wu["lora_down"], 1.0, 1.0)
+    with pytest.raises(B.SvdqError):
+        B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, 1.0, fake_next, 1.0)
+
+
+def test_mlp_full_size_sampled():
+    """The DiT MLP (4096 tokens, 3072 -> 12288 -> 3072) through the one-call
+    entry point; a sample of rows checked against the oracle one by one."""
+    B = _lib()
+    up_case = dataclasses.replace(wl.SVDQ_CASES["mlp_up"], bias_std=0.1)
+    down_case = dataclasses.replace(wl.SVDQ_CASES["mlp_down"], bias_std=0.05)
+    iu, idn, pk_u, pk_d, wu, wd = _setup(up_case, down_case)
+    x = B.bits_to_bf16(iu.x_bits, "cuda")
+    b_u = B.bits_to_bf16(iu.bias_bits, "cuda")
+    b_d = B.bits_to_bf16(idn.bias_bits, "cuda")
+    s_a = float(iu.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wu["inv_smooth"], wu["lora_down"], s_a, wu["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk_u["weight_scale"][0])))
+    hc, hs, hl = B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, alpha, wd, float(idn.act_scale), bias=b_u)
+    y = B.svdq_w4a4_mlp_gelu(x, wu, s_a, wd, float(idn.act_scale), up_bias=b_u, down_bias=b_d)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 127, 128, 1000, 2047, 2048, 3001, 4094, 4095])
+    v, h = _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl, rows=rows)
+    ref_d = O.pack_weights("nvfp4", idn.W, idn.lam, idn.L1, idn.L2)
+    y64 = O.linear_f64("nvfp4", h, ref_d, idn.L1, idn.L2, idn.bias)
+    _assert_mlp_close(y.float().cpu().numpy()[rows], y64, "MLP full size (sampled rows)")
