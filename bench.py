@@ -415,7 +415,64 @@ def measure_rows(B, wl, dev, peaks):
         int4[f"M={M}"] = {"us": round(t, 2), "TOPS": round(2.0 * M * c.N * c.K / t / 1e6, 1)}
         del ws, ys
     rows["svdq_w4a4 int4 K=N=3072 (quantize + i8 GEMM)"] = int4
+    rows["mlp_gelu"] = measure_mlp(B, wl, dev)
     return rows
+
+
+def measure_mlp(B, wl, dev):
+    """The DiT MLP block x [4096, 3072] -> 12288 -> 3072, fused (the GELU
+    and the down layer's activation quantizer in the up GEMM's epilogue) and
+    unfused (up layer -> bf16 y -> GELU -> down layer; the GELU there is
+    torch's, for comparison only).  Two rotating weight sets."""
+    import dataclasses
+    import torch
+    iu = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_up"], bias_std=0.1))
+    idn = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_down"], bias_std=0.05))
+    M, K, N = iu.case.M, iu.case.K, iu.case.N
+    pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
+    pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
+    nset = 2
+    wus = [B.to_device(pk_u, dev) for _ in range(nset)]
+    wds = [B.to_device(pk_d, dev) for _ in range(nset)]
+    x = B.bits_to_bf16(iu.x_bits, dev)
+    b_u = B.bits_to_bf16(iu.bias_bits, dev)
+    b_d = B.bits_to_bf16(idn.bias_bits, dev)
+    s_u, s_d = float(iu.act_scale), float(idn.act_scale)
+    y = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(B.mlp_workspace_bytes(M, K, N), dtype=torch.uint8, device=dev)
+    fused = [lambda i=i: B.svdq_w4a4_mlp_gelu(x, wus[i], s_u, wds[i], s_d, up_bias=b_u, down_bias=b_d, y=y,
+                                              workspace=ws) for i in range(nset)]
+    y_up = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws_u = torch.empty(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(B.workspace_bytes("nvfp4", M, N), dtype=torch.uint8, device=dev)
+
+    def unfused(i):
+        B.svdq_w4a4_linear("nvfp4", x, wus[i], s_u, bias=b_u, y=y_up, workspace=ws_u)
+        g = torch.nn.functional.gelu(y_up)
+        B.svdq_w4a4_linear("nvfp4", g, wds[i], s_d, bias=b_d, y=y, workspace=ws_d)
+
+    t_f = _event_time_us(torch, fused, 40)
+    t_u = _event_time_us(torch, [lambda i=i: unfused(i) for i in range(nset)], 40)
+    # the up GEMM alone, plain epilogue vs GELU-MLP epilogue
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wus[0]["inv_smooth"], wus[0]["lora_down"], s_u,
+                                              wus[0]["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_u) * np.float32(pk_u["weight_scale"][0])))
+    hc = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    hs = torch.empty(B.act_scale_bytes("nvfp4", M, N), dtype=torch.uint8, device=dev)
+    hl = torch.empty((M, 64), dtype=torch.bfloat16, device=dev)
+    work = torch.empty(B.gelu_quant_work_bytes(M), dtype=torch.uint8, device=dev)
+    t_plain = _event_time_us(torch, [lambda i=i: B.svdq_w4a4_gemm("nvfp4", codes, scales, lora, wus[i], alpha,
+                                                                  bias=b_u, y=y_up) for i in range(nset)], 40)
+    t_gq = _event_time_us(torch, [lambda i=i: B.svdq_w4a4_gemm_gelu_quant(
+        codes, scales, lora, wus[i], alpha, wds[i], s_d, bias=b_u, out=(hc, hs, hl), work=work)
+        for i in range(nset)], 40)
+    flop = 2.0 * 2.0 * M * N * K
+    del wus, wds
+    return {"workload": f"x [{M},{K}] -> {N} -> {K}, NVFP4 r32, bias, exact GELU",
+            "fused_us": round(t_f, 2), "fused_TFLOPS": round(flop / t_f / 1e6, 1),
+            "unfused_us": round(t_u, 2), "unfused_TFLOPS": round(flop / t_u / 1e6, 1),
+            "speedup": round(t_u / t_f, 3),
+            "up_gemm_plain_us": round(t_plain, 2), "up_gemm_gelu_quant_us": round(t_gq, 2)}
 
 
 def main():

@@ -50,13 +50,28 @@ constexpr int B_BYTES = BN * BK_BYTES;            // 32 KB
 constexpr int SFA_BYTES = 4 * 512;                // 4 K64 chunks x 128 rows
 constexpr int SFB_BYTES = 2 * 4 * 512;            // 2 row blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
-constexpr int EPI_WARPS = 4;
 constexpr int EPI_CHUNK = 16;                          // columns per TMEM load / store
 constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;      // 32 rows x 32 B
-constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
-constexpr int SF_WARPS = 3;
-constexpr int SF_WARP0 = 2 + EPI_WARPS;                 // first scale-copy warp
-constexpr int NUM_THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
+constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;       // epilogue staging, 8 KB
+
+// Warp roles.  Plain epilogue (9 warps): producer 0, MMA 1, epilogue 2-5,
+// block-scale copies 6-8.  GELU-MLP epilogue (12 warps, three warpgroups):
+// epilogue 0-7, producer 8, MMA 9, block-scale copies 10-11; the last
+// warpgroup hands registers to the two epilogue warpgroups (setmaxnreg).
+template <bool kGelu>
+struct Roles {
+  static constexpr int EPI_WARPS = kGelu ? 8 : 4;
+  static constexpr int PRODUCER = kGelu ? 8 : 0;
+  static constexpr int MMA = kGelu ? 9 : 1;
+  static constexpr int SF_W0 = kGelu ? 10 : 6;
+  static constexpr int SF_WARPS = kGelu ? 2 : 3;
+  static constexpr int NUM_THREADS = (kGelu ? 12 : 9) * 32;
+};
+// Register split of the GELU-MLP kernel: launched at 168 per thread
+// (12 warps x 32 x 168 = 64512), then 224 for each epilogue thread and 56 for
+// the rest: 256 x 224 + 128 x 56 = 64512.
+constexpr int GQ_LAUNCH_REGS = 168, GQ_EPI_REGS = 224, GQ_CTL_REGS = 56;
+static_assert(256 * GQ_EPI_REGS + 128 * GQ_CTL_REGS <= 384 * GQ_LAUNCH_REGS, "register split");
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_STRIDE = 160;                        // accumulator b starts at column b * 160
 constexpr int ACC_OVERLAP = 2 * 256 - (ACC_STRIDE + 256); // 96 shared columns
@@ -81,7 +96,14 @@ struct SmemCtl {
   int abort_flag;
 };
 
-constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + sizeof(SmemCtl);
+// The GELU-MLP epilogue keeps the tile's 1/lambda (fp32) and bias (bf16)
+// columns in shared memory after the staging buffers.
+constexpr int GQ_TABLE_BYTES = BN * 4 + BN * 2;
+template <bool kGelu>
+constexpr size_t smem_bytes() {
+  return 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + (kGelu ? GQ_TABLE_BYTES : 0) + sizeof(SmemCtl);
+}
+static_assert(smem_bytes<true>() <= 232448, "shared memory per block");
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   block-scaled: a/b format E2M1 (=1) at bits 7/10, N>>3 at 17, UE4M3 scales
@@ -94,8 +116,38 @@ SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024,
 SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
 
 // ------------------------------------------------------- GELU-MLP epilogue helpers
-// Exact (erf) GELU: v Phi(v) = v (1 + erf(v / sqrt 2)) / 2.
-SVDQ_DEV float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+SVDQ_DEV float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+SVDQ_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU(v) = v Phi(v) with Phi the standard normal CDF (the exact erf form),
+// Phi(-|v|) = erfc(|v| / sqrt 2) / 2 taken from Abramowitz & Stegun,
+// "Handbook of Mathematical Functions", formula 7.1.26 (Hastings):
+//   erfc(x) ~ (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
+//   t = 1 / (1 + p x),  x >= 0,  absolute error <= 1.5e-7,
+// evaluated with the hardware reciprocal and base-2 exponential.  Taking
+// Phi(v) = erfc/2 for v < 0 and 1 - erfc/2 for v >= 0 keeps the small
+// negative tail free of cancellation.
+SVDQ_DEV float gelu(float v) {
+  const float x = fabsf(v) * 0.70710678118654752f;
+  const float t = rcp_approx(__fmaf_rn(0.3275911f, x, 1.0f));
+  float q = __fmaf_rn(1.061405429f, t, -1.453152027f);
+  q = __fmaf_rn(q, t, 1.421413741f);
+  q = __fmaf_rn(q, t, -0.284496736f);
+  q = __fmaf_rn(q, t, 0.254829592f);
+  q = __fmul_rn(q, t);
+  const float e = ex2_approx(__fmul_rn(__fmul_rn(x, x), -1.4426950408889634f));  // exp(-x^2)
+  const float half_erfc = __fmul_rn(__fmul_rn(0.5f, q), e);
+  return __fmul_rn(v, v < 0.f ? half_erfc : __fsub_rn(1.0f, half_erfc));
+}
 
 SVDQ_DEV uint32_t half2_bits(float lo, float hi) {
   uint32_t out;
@@ -106,13 +158,6 @@ SVDQ_DEV uint32_t half2_bits(float lo, float hi) {
 SVDQ_DEV void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
-}
-
-SVDQ_DEV uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
-               : "memory");
-  return v;
 }
 
 // D (fp32) += A (16 x 16 fp16, row) * B (16 x 8 fp16, col).
@@ -134,15 +179,21 @@ SVDQ_DEV size_t tiled_scale_offset(int row, int group, int K) {
   return ((size_t)(row >> 7) * (K / 64) + (group >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (group & 3);
 }
 
-// 16-byte segment s (fp16 columns 8s..8s+7) of row r in a warp's 32 x 32
-// fp16 staging tile (64-byte rows; segments XOR-ed with (r / 2) mod 4 so that
+// 16-byte segment s (fp16 columns 8s..8s+7) of row r in a warp's 32 x 16
+// fp16 staging tile (32-byte rows; segments XOR-ed with (r / 4) mod 2 so that
 // both the row-per-lane stores and the fragment loads are conflict-free).
-SVDQ_DEV uint32_t hseg(uint32_t base, int r, int s) {
-  return base + (uint32_t)r * 64u + (uint32_t)((s ^ ((r >> 1) & 3)) << 4);
+SVDQ_DEV uint32_t hseg16(uint32_t base, int r, int s) {
+  return base + (uint32_t)r * 32u + (uint32_t)((s ^ ((r >> 2) & 1)) << 4);
+}
+
+SVDQ_DEV uint2 ld_shared_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
 }
 
 template <bool kGelu>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                       const __grid_constant__ CUtensorMap tm_y, const GemmNvfp4Params p) {
@@ -150,8 +201,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kGelu ? GQ_TABLE_BYTES : 0));
 
+  using R = Roles<kGelu>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (p.M + BM - 1) / BM;
   const int tiles_n = (p.N + BN - 1) / BN;
@@ -165,24 +217,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&ctl->empty[s]), 1);
     }
     mbar_init(smem_u32(&ctl->acc_full), 1);
-    mbar_init(smem_u32(&ctl->acc_empty), EPI_WARPS);
+    mbar_init(smem_u32(&ctl->acc_empty), R::EPI_WARPS);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&ctl->sf_full[b]), SF_WARPS);
+      mbar_init(smem_u32(&ctl->sf_full[b]), R::SF_WARPS);
       mbar_init(smem_u32(&ctl->sf_empty[b]), 1);
     }
     mbar_init(smem_u32(&ctl->drain), 1);
-    mbar_init(smem_u32(&ctl->sf_drain), SF_WARPS);
+    mbar_init(smem_u32(&ctl->sf_drain), R::SF_WARPS);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == R::PRODUCER && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_la);
     prefetch_tmap(&tm_lb);
     if (!kGelu) prefetch_tmap(&tm_y);
   }
-  if (warp == 1) {
+  if (warp == R::MMA) {
     tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
     tmem_relinquish();
   }
@@ -196,7 +248,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
 
-  if (warp == 0) {
+  // ---------------------------------------------------------------- roles
+  auto role_producer = [&]() {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       int stage = 0;
@@ -247,7 +300,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (issued_mask & (1u << s))
           mbar_wait(smem_u32(&ctl->full[s]), (issued_phase >> s) & 1, drain_ctx, kDevTimeoutDrain);
     }
-  } else if (warp == 1) {
+  };
+  auto role_mma = [&]() {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
@@ -305,12 +359,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
     }
-  } else if (warp >= SF_WARP0) {
+  };
+  auto role_scale_copies = [&]() {
     if (lane == 0) {
       // ------------------------------------------------------------ scale copies
-      // Warp SF_WARP0 + w copies part w of every K slice's block scales:
-      // w = 0: SFA (4 copies), w = 1 / 2: SFB rows 0-127 / 128-255 (4 each).
-      const int w = warp - SF_WARP0;
+      // Three jobs per K slice: 0 = SFA (4 copies), 1 / 2 = SFB rows 0-127 /
+      // 128-255 (4 each); scale-copy warp w takes jobs w, w + SF_WARPS, ...
+      const int w = warp - R::SF_W0;
       int stage = 0;
       uint32_t phase = 0, ks = 0;
       bool ok = true;
@@ -329,11 +384,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_fence_after();
             const uint32_t ssfa = smem_u32(stage_base + stage * STAGE_BYTES) + A_BYTES + B_BYTES;
-            const uint32_t src = w == 0 ? ssfa : ssfa + SFA_BYTES * w;
-            const uint32_t dst = tmem + TMEM_SF0 + buf * SF_COLS + (w == 0 ? TMEM_SFA_OFF : TMEM_SFB_OFF + 4 * (w - 1));
-            const uint32_t col_step = w == 0 ? 4 : 8;
+            for (int job = w; job < 3; job += R::SF_WARPS) {
+              const uint32_t src = job == 0 ? ssfa : ssfa + SFA_BYTES * job;
+              const uint32_t dst =
+                  tmem + TMEM_SF0 + buf * SF_COLS + (job == 0 ? TMEM_SFA_OFF : TMEM_SFB_OFF + 4 * (job - 1));
+              const uint32_t col_step = job == 0 ? 4 : 8;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_cp_32x128_warpx4(dst + col_step * j, sf_desc(src + 512 * j));
+              for (int j = 0; j < 4; ++j) tmem_cp_32x128_warpx4(dst + col_step * j, sf_desc(src + 512 * j));
+            }
             tc_commit(smem_u32(&ctl->sf_full[buf]));
             ++ks;
           }
@@ -348,23 +406,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->sf_drain), 0, drain_ctx, kDevTimeoutDrain);
     }
-  } else if constexpr (kGelu) {
+  };
+  auto role_epilogue = [&]() {
+    if constexpr (kGelu) {
     // ------------------------------------------------------ GELU-MLP epilogue
-    // Same TMEM schedule as the plain epilogue below.  Per 32-column chunk
-    // each lane (one row) forms h_hat = GELU(alpha D + b) * inv_lambda_down
-    // in fp32, quantizes its two 16-groups with the down layer's NVFP4 rule
-    // (16 bytes of codes, 2 scale bytes), and stages fp16(h_hat 2^-e) in a
-    // 32 x 32 shared tile from which the warp accumulates its 32 rows x 32
-    // ranks of the down layer's low-rank projection on mma.sync.  Lane (g, c)
-    // takes fp16 columns 8c..8c+3 as k-step 0 and 8c+4..8c+7 as k-step 1 (a
-    // permutation of k shared by both operands), so each of its A and B
-    // fragments is one 16-byte load.  After the tile, the partial sums go to
-    // u_work with vector reductions; the warp that completes a 32-row block's
-    // count of N tiles converts those rows to the bf16 hi/lo lora_act.
-    const int q = warp & 3;
+    // Eight warps: warp w reads TMEM lane quarter w mod 4 (32 rows) and one
+    // half of the tile's eight 32-column chunks (w / 4 = 0: the first four in
+    // the ring order below, which include the columns shared with the other
+    // accumulator; 1: the last four).  Per chunk each lane (one row) forms
+    // h_hat = GELU(alpha D + b) * inv_lambda_down in fp32, quantizes its two
+    // 16-groups with the down layer's NVFP4 rule (16 bytes of codes, 2 scale
+    // bytes), and, 16 columns at a time, stages fp16(h_hat 2^-e) in a 32 x 16
+    // shared tile from which the warp accumulates its rows' share of the down
+    // layer's low-rank projection on mma.sync.  Lane (g, c) takes fp16
+    // columns 4c..4c+3 of the 16 as its k values (a permutation of k shared by
+    // both operands), so its A and B fragments are 8-byte loads.  The tile's
+    // 1/lambda and bias columns are staged once per tile in shared memory.
+    // After the tile the partial sums go to u_work with vector reductions; the
+    // warp that completes a 32-row block's count (two warps per N tile)
+    // converts those rows to the bf16 hi/lo lora_act.  The eight warps share
+    // named barriers 2 and 3, so every stop decision is taken by all of them.
+    constexpr int NT = R::EPI_WARPS * 32;
+    const int q = warp & 3, hf = warp >> 2;
     const int g = lane >> 2, c = lane & 3;
+    const int et = threadIdx.x;  // 0..255 over the epilogue warps
     const GeluQuantParams& gq = p.gq;
-    const uint32_t hbase = smem_u32(epi_base + (warp - 2) * 2048);
+    const uint32_t hbase = smem_u32(epi_base + warp * 1024);
+    float* tab_inv = reinterpret_cast<float*>(epi_base + EPI_BYTES);
+    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + BN * 4);
     const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
     const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
     uint32_t acc_phase = 0;
@@ -372,13 +441,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     constexpr int LDC = 32;
     constexpr int NCH = BN / LDC;
     constexpr int NSH = (ACC_OVERLAP + LDC - 1) / LDC;
+    constexpr int CPW = NCH / 2;  // chunks per warp
     constexpr int NBUF = 3;
+    static_assert(NSH <= NBUF && NBUF <= CPW, "the shared chunks fit the first ring fill of half 0");
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM;
       const int n0 = (tile / tiles_m) * BN;
       const int b = it & 1;
       const int row = m0 + 32 * q + lane;
       const bool row_ok = row < p.M;
+      // This thread's table column, fetched before the wait.
+      const float my_inv = __ldg(gq.inv_smooth + n0 + et);
+      const uint16_t my_bias = p.bias != nullptr ? __ldg(p.bias + n0 + et) : (uint16_t)0;
+      const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
+      // All epilogue threads decide together; this barrier also ends every
+      // read of the previous tile's table.
+      if (named_bar_any(2, NT, !got)) break;
+      tab_inv[et] = my_inv;
+      tab_bias[et] = my_bias;
+      asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory");
+      tc_fence_after();
       float lacc[2][4][4];
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -386,14 +468,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int e = 0; e < 4; ++e) lacc[t][j][e] = 0.f;
-      const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
       const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+      // Ring order: the shared columns first (the last ACC_OVERLAP of
+      // accumulator 0, the first ACC_OVERLAP of accumulator 1).
       auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NSH) % NCH : i; };
+      const int i0 = hf * CPW;
       uint32_t rb[NBUF][32];
 #pragma unroll
-      for (int i = 0; i < NBUF; ++i) tmem_ld_32x32b_x32(acc_base + chunk_col(i) * LDC, rb[i]);
+      for (int i = 0; i < NBUF; ++i) tmem_ld_32x32b_x32(acc_base + chunk_col(i0 + i) * LDC, rb[i]);
       tmem_ld_wait(rb[0]);
       reg_fence(rb[1]);
       reg_fence(rb[2]);
@@ -401,29 +483,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        uint32_t(&r)[32] = rb[i % NBUF];
-        if (i >= NBUF && i % NBUF == 0) {
+      for (int ii = 0; ii < CPW; ++ii) {
+        uint32_t(&r)[32] = rb[ii % NBUF];
+        if (ii >= NBUF && ii % NBUF == 0) {
           tmem_ld_wait(rb[0]);
           reg_fence(rb[1]);
           reg_fence(rb[2]);
         }
-        const int n = n0 + chunk_col(i) * LDC;
+        const int cl = chunk_col(i0 + ii) * LDC;  // column within the tile
+        const int n = n0 + cl;
         // h_hat in place of the accumulator values (zero for rows past M, so
         // their scales come out zero and they add nothing).
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8) {
-          const uint4 bw = p.bias != nullptr ? __ldg(reinterpret_cast<const uint4*>(p.bias + n) + k8)
-                                             : make_uint4(0, 0, 0, 0);
-          const float4 i0 = __ldg(reinterpret_cast<const float4*>(gq.inv_smooth + n) + 2 * k8);
-          const float4 i1 = __ldg(reinterpret_cast<const float4*>(gq.inv_smooth + n) + 2 * k8 + 1);
+          const float4 i0v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8);
+          const float4 i1v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8 + 4);
+          const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + cl + 8 * k8);
           const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-          const float il[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+          const float il[8] = {i0v.x, i0v.y, i0v.z, i0v.w, i1v.x, i1v.y, i1v.z, i1v.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float bias_v = __uint_as_float((j & 1) ? (bb[j >> 1] & 0xFFFF0000u) : (bb[j >> 1] << 16));
             const float v = __fmaf_rn(p.alpha, __uint_as_float(r[8 * k8 + j]), bias_v);
-            const float h = __fmul_rn(gelu_erf(v), il[j]);
+            const float h = __fmul_rn(gelu(v), il[j]);
             r[8 * k8 + j] = __float_as_uint(row_ok ? h : 0.f);
           }
         }
@@ -458,39 +540,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (row_ok)
           *reinterpret_cast<uint4*>(gq.codes + (size_t)row * (p.N / 2) + n / 2) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         *reinterpret_cast<uint16_t*>(gq.scales + tiled_scale_offset(row, n / 16, p.N)) = (uint16_t)sbs;
-        // fp16(h_hat 2^-e) into the staging tile, row = lane.
+        // Low-rank partial, 16 columns at a time.
 #pragma unroll
-        for (int sg = 0; sg < 4; ++sg) {
-          uint32_t hv[4];
+        for (int hh = 0; hh < 2; ++hh) {
+          uint2 bq[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 t =
-                __fmul2_rn(make_float2(__uint_as_float(r[8 * sg + 2 * k]), __uint_as_float(r[8 * sg + 2 * k + 1])), lr2);
-            hv[k] = half2_bits(t.x, t.y);
+          for (int j = 0; j < 4; ++j)
+            bq[j] = __ldg(reinterpret_cast<const uint2*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 16 * hh + 4 * c));
+#pragma unroll
+          for (int sg = 0; sg < 2; ++sg) {
+            uint32_t hv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 16 * hh + 8 * sg + 2 * k;
+              const float2 t = __fmul2_rn(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), lr2);
+              hv[k] = half2_bits(t.x, t.y);
+            }
+            st_shared_v4(hseg16(hbase, lane, sg), make_uint4(hv[0], hv[1], hv[2], hv[3]));
           }
-          st_shared_v4(hseg(hbase, lane, sg), make_uint4(hv[0], hv[1], hv[2], hv[3]));
-        }
-        __syncwarp();
-        uint4 x0[2], x1[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          x0[t] = ld_shared_v4(hseg(hbase, 16 * t + g, c));
-          x1[t] = ld_shared_v4(hseg(hbase, 16 * t + 8 + g, c));
-        }
-        __syncwarp();  // every lane's loads precede the next chunk's stores
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 bq = __ldg(reinterpret_cast<const uint4*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 8 * c));
+          __syncwarp();
+          uint2 xa[2], xb[2];
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            mma_16816(lacc[t][j], x0[t].x, x1[t].x, x0[t].y, x1[t].y, bq.x, bq.y);
-            mma_16816(lacc[t][j], x0[t].z, x1[t].z, x0[t].w, x1[t].w, bq.z, bq.w);
+            xa[t] = ld_shared_v2(hseg16(hbase, 16 * t + g, c >> 1) + (c & 1) * 8);
+            xb[t] = ld_shared_v2(hseg16(hbase, 16 * t + 8 + g, c >> 1) + (c & 1) * 8);
           }
+          __syncwarp();  // every lane's loads precede the next stores
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int t = 0; t < 2; ++t) mma_16816(lacc[t][j], xa[t].x, xb[t].x, xa[t].y, xb[t].y, bq[j].x, bq[j].y);
         }
         // Refill the block just converted with the chunk three ahead.
-        if (i + NBUF < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + NBUF) * LDC, r);
+        if (ii + NBUF < CPW) tmem_ld_32x32b_x32(acc_base + chunk_col(i0 + ii + NBUF) * LDC, r);
       }
-      // The tile's low-rank partial: rows 16t + g (+8), ranks 8j + 2c (+1).
+      // The warp's low-rank partial: rows 16t + g (+8), ranks 8j + 2c (+1).
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const int r0 = m0 + 32 * q + 16 * t + g;
@@ -506,8 +590,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       unsigned int prev = 0;
       if (lane == 0) prev = atomicAdd(gq.counters + (m0 + 32 * q) / 32, 1u);
       prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev == (unsigned int)(tiles_n - 1)) {
-        // Every N tile of these 32 rows has added its partial.
+      if (prev == (unsigned int)(2 * tiles_n - 1)) {
+        // Both halves of every N tile of these 32 rows have added their partials.
         __threadfence();
         const int rbase = m0 + 32 * q;
         for (int rr = 0; rr < 32 && rbase + rr < p.M; ++rr) {
@@ -520,7 +604,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       acc_phase ^= 1;
     }
-  } else {
+    } else {
     // -------------------------------------------------------------- epilogue
     // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile,
     // read from TMEM 32 columns at a time into a ring of three register
@@ -530,7 +614,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // the block just converted, three chunks ahead.  The tile's bias is loaded
     // once (lane l holds columns 8l..8l+7) and broadcast by shuffles.
     const int q = warp & 3;
-    uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;
+    uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;  // epilogue warps 2-5
     uint32_t acc_phase = 0;
     int chunk_seq = 0, it = 0;
     constexpr int LDC = 32;                    // columns per TMEM load
@@ -617,11 +701,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc_phase ^= 1;
     }
     if (lane == 0) bulk_wait<0>();
+    }
+  };
+
+  if constexpr (kGelu) {
+    // setmaxnreg is warpgroup-wide: the last warpgroup (producer, MMA, scale
+    // copies) gives registers to the two epilogue warpgroups.
+    if (warp >= R::EPI_WARPS) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(GQ_CTL_REGS));
+      if (warp == R::PRODUCER)
+        role_producer();
+      else if (warp == R::MMA)
+        role_mma();
+      else
+        role_scale_copies();
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(GQ_EPI_REGS));
+      role_epilogue();
+    }
+  } else {
+    if (warp == R::PRODUCER)
+      role_producer();
+    else if (warp == R::MMA)
+      role_mma();
+    else if (warp >= R::SF_W0)
+      role_scale_copies();
+    else
+      role_epilogue();
   }
+
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == R::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -635,15 +747,25 @@ cudaError_t launch_impl(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sm
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<kGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+                                         (int)smem_bytes<kGelu>());
     if (e != cudaSuccess) return e;
+    if (kGelu) {
+      // The epilogue warpgroups' setmaxnreg.inc waits until the others have
+      // released enough registers: only launch if the compiled register
+      // count makes the split add up.
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, gemm_nvfp4_kernel<kGelu>);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs * Roles<true>::NUM_THREADS < 256 * GQ_EPI_REGS + 128 * GQ_CTL_REGS)
+        return cudaErrorInvalidConfiguration;
+    }
     attr_set = true;
   }
   const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.blockDim = dim3(Roles<kGelu>::NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<kGelu>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
