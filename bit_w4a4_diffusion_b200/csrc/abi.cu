@@ -387,8 +387,7 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
 
 long long svdq_gelu_quant_work_bytes(int M) {
   if (M <= 0) return -1;
-  const long long counters = round_up(round_up(M, 128) / 32 * 4, 256);
-  return counters + round_up((int64_t)M * SVDQ_RANK * 4, 256);
+  return round_up((int64_t)M * SVDQ_RANK * 4, 256);  // fp32 low-rank sums [M, r]
 }
 
 static bool nvfp4_scale_ok(float s) { return s >= 0x1p-100f && s < 0x1p100f; }
@@ -406,27 +405,38 @@ static int gelu_quant_prepare(int M, int N, void* next_act_scales, void* work, c
   return SVDQ_OK;
 }
 
-static GeluQuantParams gelu_quant_params(int M, const float* next_inv_smooth, const void* next_lora_down,
-                                         float next_act_scale, float next_weight_scale, void* next_act_codes,
-                                         void* next_act_scales, void* next_lora_act, void* work) {
+// h_hat enters the fp16 down-projection as h_hat * 2^-e (the rule of
+// svdq_quantize_act: 2688 s maps into [2^12, 2^13)); the finalize step
+// multiplies the sums by 2^e / (s s_w).
+static int lowrank_exponent(float act_scale) {
+  int ex = 0;
+  frexpf(2688.0f * act_scale, &ex);
+  return ex - 1 - 12;
+}
+
+// The fused GEMM, then the conversion of its low-rank sums (PDL-chained).
+static int launch_gelu_quant(int M, int N, int K, const void* act_codes, const void* act_scales,
+                             const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                             const void* bias, float alpha, const float* next_inv_smooth, const void* next_lora_down,
+                             float next_act_scale, float next_weight_scale, void* next_act_codes,
+                             void* next_act_scales, void* next_lora_act, void* work, int* dev_status,
+                             cudaStream_t stream, bool pdl, int sms) {
+  const int e = lowrank_exponent(next_act_scale);
   GeluQuantParams g{};
   g.inv_smooth = next_inv_smooth;
   g.l1t = static_cast<const uint16_t*>(next_lora_down);
   g.s_d = next_act_scale;
-  // h_hat enters the fp16 down-projection as h_hat * 2^-e (the rule of
-  // svdq_quantize_act: 2688 s maps into [2^12, 2^13)).
-  int ex = 0;
-  frexpf(2688.0f * next_act_scale, &ex);
-  const int e = ex - 1 - 12;
   g.lr_in_scale = ldexpf(1.0f, -e);
-  g.lora_scale = ldexpf(1.0f, e) / (next_act_scale * next_weight_scale);
   g.codes = static_cast<uint8_t*>(next_act_codes);
   g.scales = static_cast<uint8_t*>(next_act_scales);
-  g.lora_act = static_cast<uint16_t*>(next_lora_act);
-  uint8_t* w = static_cast<uint8_t*>(work);
-  g.counters = reinterpret_cast<unsigned int*>(w);
-  g.u_work = reinterpret_cast<float*>(w + round_up(round_up(M, 128) / 32 * 4, 256));
-  return g;
+  g.u_work = static_cast<float*>(work);
+  if (int s = gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha,
+                              nullptr, dev_status, stream, pdl, sms, &g))
+    return s;
+  const float lora_scale = ldexpf(1.0f, e) / (next_act_scale * next_weight_scale);
+  return check_cuda(launch_lowrank_finalize(g.u_work, M, lora_scale, static_cast<uint16_t*>(next_lora_act), stream,
+                                            true),
+                    "low-rank finalize launch");
 }
 
 static int check_gelu_quant_args(int M, int N, int K, int rank, float alpha, const float* next_inv_smooth,
@@ -470,10 +480,9 @@ int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_cod
   if (int s = check_device(&sms)) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (int s = gelu_quant_prepare(M, N, next_act_scales, work, st)) return s;
-  const GeluQuantParams g = gelu_quant_params(M, next_inv_smooth, next_lora_down, next_act_scale, next_weight_scale,
-                                              next_act_codes, next_act_scales, next_lora_act, work);
-  return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, nullptr,
-                         dev_status, st, false, sms, &g);
+  return launch_gelu_quant(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha,
+                           next_inv_smooth, next_lora_down, next_act_scale, next_weight_scale, next_act_codes,
+                           next_act_scales, next_lora_act, work, dev_status, st, false, sms);
 }
 
 long long svdq_mlp_workspace_bytes(int M, int K, int N_hidden, int rank) {
@@ -527,10 +536,9 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
   if (int s = svdq_quantize_act(SVDQ_NVFP4, M, K, rank, x, up_inv_smooth, up_lora_down, up_act_scale,
                                 up_weight_scale, a_codes, a_scales, a_lora, stream))
     return s;
-  const GeluQuantParams g = gelu_quant_params(M, down_inv_smooth, down_lora_down, down_act_scale, down_weight_scale,
-                                              h_codes, h_scales, h_lora, work);
-  if (int s = gemm_nvfp4_impl(M, N, K, a_codes, a_scales, a_lora, up_w_codes, up_w_scales, up_lora_up, up_bias,
-                              up_alpha, nullptr, dev_status, st, true, sms, &g))
+  if (int s = launch_gelu_quant(M, N, K, a_codes, a_scales, a_lora, up_w_codes, up_w_scales, up_lora_up, up_bias,
+                                up_alpha, down_inv_smooth, down_lora_down, down_act_scale, down_weight_scale, h_codes,
+                                h_scales, h_lora, work, dev_status, st, true, sms))
     return s;
   return gemm_nvfp4_impl(M, K, N, h_codes, h_scales, h_lora, down_w_codes, down_w_scales, down_lora_up, down_bias,
                          down_act_scale * down_weight_scale, y, dev_status, st, true, sms);

@@ -68,9 +68,9 @@ struct Roles {
   static constexpr int NUM_THREADS = (kGelu ? 12 : 9) * 32;
 };
 // Register split of the GELU-MLP kernel: launched at 168 per thread
-// (12 warps x 32 x 168 = 64512), then 224 for each epilogue thread and 56 for
-// the rest: 256 x 224 + 128 x 56 = 64512.
-constexpr int GQ_LAUNCH_REGS = 168, GQ_EPI_REGS = 224, GQ_CTL_REGS = 56;
+// (12 warps x 32 x 168 = 64512), then 216 for each epilogue thread and 72 for
+// the rest: 256 x 216 + 128 x 72 = 64512.
+constexpr int GQ_LAUNCH_REGS = 168, GQ_EPI_REGS = 216, GQ_CTL_REGS = 72;
 static_assert(256 * GQ_EPI_REGS + 128 * GQ_CTL_REGS <= 384 * GQ_LAUNCH_REGS, "register split");
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_STRIDE = 160;                        // accumulator b starts at column b * 160
@@ -136,17 +136,24 @@ SVDQ_DEV float ex2_approx(float x) {
 // evaluated with the hardware reciprocal and base-2 exponential.  Taking
 // Phi(v) = erfc/2 for v < 0 and 1 - erfc/2 for v >= 0 keeps the small
 // negative tail free of cancellation.
-SVDQ_DEV float gelu(float v) {
-  const float x = fabsf(v) * 0.70710678118654752f;
-  const float t = rcp_approx(__fmaf_rn(0.3275911f, x, 1.0f));
-  float q = __fmaf_rn(1.061405429f, t, -1.453152027f);
-  q = __fmaf_rn(q, t, 1.421413741f);
-  q = __fmaf_rn(q, t, -0.284496736f);
-  q = __fmaf_rn(q, t, 0.254829592f);
-  q = __fmul_rn(q, t);
-  const float e = ex2_approx(__fmul_rn(__fmul_rn(x, x), -1.4426950408889634f));  // exp(-x^2)
-  const float half_erfc = __fmul_rn(__fmul_rn(0.5f, q), e);
-  return __fmul_rn(v, v < 0.f ? half_erfc : __fsub_rn(1.0f, half_erfc));
+// Two elements at a time on the packed fp32x2 pipe (each lane of a packed
+// operation rounds like its scalar counterpart).
+SVDQ_DEV float2 f2(float a) { return make_float2(a, a); }
+SVDQ_DEV float2 gelu2(float2 v) {
+  const float2 x = __fmul2_rn(make_float2(fabsf(v.x), fabsf(v.y)), f2(0.70710678118654752f));
+  const float2 den = __ffma2_rn(f2(0.3275911f), x, f2(1.0f));
+  const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+  float2 q = __ffma2_rn(f2(1.061405429f), t, f2(-1.453152027f));
+  q = __ffma2_rn(q, t, f2(1.421413741f));
+  q = __ffma2_rn(q, t, f2(-0.284496736f));
+  q = __ffma2_rn(q, t, f2(0.254829592f));
+  q = __fmul2_rn(q, t);
+  const float2 arg = __fmul2_rn(__fmul2_rn(x, x), f2(-1.4426950408889634f));  // -x^2 log2(e)
+  const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));         // exp(-x^2)
+  const float2 half_erfc = __fmul2_rn(__fmul2_rn(f2(0.5f), q), e);
+  const float2 upper = __fadd2_rn(f2(1.0f), make_float2(-half_erfc.x, -half_erfc.y));
+  const float2 phi = make_float2(v.x < 0.f ? half_erfc.x : upper.x, v.y < 0.f ? half_erfc.y : upper.y);
+  return __fmul2_rn(v, phi);
 }
 
 SVDQ_DEV uint32_t half2_bits(float lo, float hi) {
@@ -422,10 +429,10 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     // columns 4c..4c+3 of the 16 as its k values (a permutation of k shared by
     // both operands), so its A and B fragments are 8-byte loads.  The tile's
     // 1/lambda and bias columns are staged once per tile in shared memory.
-    // After the tile the partial sums go to u_work with vector reductions; the
-    // warp that completes a 32-row block's count (two warps per N tile)
-    // converts those rows to the bf16 hi/lo lora_act.  The eight warps share
-    // named barriers 2 and 3, so every stop decision is taken by all of them.
+    // After the tile the partial sums go to u_work with vector reductions
+    // (fire and forget: the conversion to lora_act is a separate kernel that
+    // runs after this grid).  The eight warps share named barriers 2 and 3,
+    // so every stop decision is taken by all of them.
     constexpr int NT = R::EPI_WARPS * 32;
     const int q = warp & 3, hf = warp >> 2;
     const int g = lane >> 2, c = lane & 3;
@@ -435,6 +442,7 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     float* tab_inv = reinterpret_cast<float*>(epi_base + EPI_BYTES);
     uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + BN * 4);
     const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
+    const float2 alpha2 = make_float2(p.alpha, p.alpha);
     const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
     uint32_t acc_phase = 0;
     int it = 0;
@@ -492,6 +500,14 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
         }
         const int cl = chunk_col(i0 + ii) * LDC;  // column within the tile
         const int n = n0 + cl;
+        // The chunk's low-rank B fragments (from L1 / L2), needed last.
+        uint2 bq[2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            bq[hh][j] =
+                __ldg(reinterpret_cast<const uint2*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 16 * hh + 4 * c));
         // h_hat in place of the accumulator values (zero for rows past M, so
         // their scales come out zero and they add nothing).
 #pragma unroll
@@ -502,11 +518,15 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
           const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
           const float il[8] = {i0v.x, i0v.y, i0v.z, i0v.w, i1v.x, i1v.y, i1v.z, i1v.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float bias_v = __uint_as_float((j & 1) ? (bb[j >> 1] & 0xFFFF0000u) : (bb[j >> 1] << 16));
-            const float v = __fmaf_rn(p.alpha, __uint_as_float(r[8 * k8 + j]), bias_v);
-            const float h = __fmul_rn(gelu(v), il[j]);
-            r[8 * k8 + j] = __float_as_uint(row_ok ? h : 0.f);
+          for (int j = 0; j < 4; ++j) {
+            const float2 bias2 = make_float2(__uint_as_float(bb[j] << 16), __uint_as_float(bb[j] & 0xFFFF0000u));
+            const float2 v = __ffma2_rn(alpha2,
+                                        make_float2(__uint_as_float(r[8 * k8 + 2 * j]),
+                                                    __uint_as_float(r[8 * k8 + 2 * j + 1])),
+                                        bias2);
+            const float2 h = __fmul2_rn(gelu2(v), make_float2(il[2 * j], il[2 * j + 1]));
+            r[8 * k8 + 2 * j] = __float_as_uint(row_ok ? h.x : 0.f);
+            r[8 * k8 + 2 * j + 1] = __float_as_uint(row_ok ? h.y : 0.f);
           }
         }
         // NVFP4 quantization of the two 16-groups (the down layer's rule).
@@ -543,10 +563,6 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
         // Low-rank partial, 16 columns at a time.
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint2 bq[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            bq[j] = __ldg(reinterpret_cast<const uint2*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 16 * hh + 4 * c));
 #pragma unroll
           for (int sg = 0; sg < 2; ++sg) {
             uint32_t hv[4];
@@ -569,7 +585,8 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int t = 0; t < 2; ++t) mma_16816(lacc[t][j], xa[t].x, xb[t].x, xa[t].y, xb[t].y, bq[j].x, bq[j].y);
+            for (int t = 0; t < 2; ++t)
+              mma_16816(lacc[t][j], xa[t].x, xb[t].x, xa[t].y, xb[t].y, bq[hh][j].x, bq[hh][j].y);
         }
         // Refill the block just converted with the chunk three ahead.
         if (ii + NBUF < CPW) tmem_ld_32x32b_x32(acc_base + chunk_col(i0 + ii + NBUF) * LDC, r);
@@ -583,23 +600,6 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
           const int col = 8 * j + 2 * c;
           if (r0 < p.M) red_add_f32x2(gq.u_work + (size_t)r0 * 32 + col, lacc[t][j][0], lacc[t][j][1]);
           if (r0 + 8 < p.M) red_add_f32x2(gq.u_work + (size_t)(r0 + 8) * 32 + col, lacc[t][j][2], lacc[t][j][3]);
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      unsigned int prev = 0;
-      if (lane == 0) prev = atomicAdd(gq.counters + (m0 + 32 * q) / 32, 1u);
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev == (unsigned int)(2 * tiles_n - 1)) {
-        // Both halves of every N tile of these 32 rows have added their partials.
-        __threadfence();
-        const int rbase = m0 + 32 * q;
-        for (int rr = 0; rr < 32 && rbase + rr < p.M; ++rr) {
-          const float uf = __fmul_rn(__ldcg(gq.u_work + (size_t)(rbase + rr) * 32 + lane), gq.lora_scale);
-          const __nv_bfloat16 hi = __float2bfloat16_rn(uf);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(uf, __bfloat162float(hi)));
-          gq.lora_act[(size_t)(rbase + rr) * 64 + lane] = __bfloat16_as_ushort(hi);
-          gq.lora_act[(size_t)(rbase + rr) * 64 + 32 + lane] = __bfloat16_as_ushort(lo);
         }
       }
       acc_phase ^= 1;
@@ -784,6 +784,37 @@ cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int 
 cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                                    bool pdl) {
   return launch_impl<true>(p, t, num_sms, stream, pdl);
+}
+
+namespace {
+// lora_act[m] = [hi(u c) | lo(u c)] with u the summed low-rank partials.
+__global__ void __launch_bounds__(256) lowrank_finalize_kernel(const float* __restrict__ u_work, int M, float c,
+                                                              uint16_t* __restrict__ lora_act) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i >= M * 32) return;
+  const int m = i >> 5, col = i & 31;
+  const float uf = __fmul_rn(u_work[i], c);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(uf);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(uf, __bfloat162float(hi)));
+  lora_act[(size_t)m * 64 + col] = __bfloat16_as_ushort(hi);
+  lora_act[(size_t)m * 64 + 32 + col] = __bfloat16_as_ushort(lo);
+}
+}  // namespace
+
+cudaError_t launch_lowrank_finalize(const float* u_work, int M, float lora_scale, uint16_t* lora_act,
+                                    cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((M * 32 + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, lowrank_finalize_kernel, u_work, M, lora_scale, lora_act);
 }
 
 }  // namespace svdq

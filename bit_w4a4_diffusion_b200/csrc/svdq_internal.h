@@ -35,18 +35,16 @@ cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm
 
 // The GELU-MLP epilogue: the up layer's output never leaves the chip; the
 // epilogue applies GELU and the down layer's smoothing, quantizer and
-// low-rank down-projection (partial sums over N tiles reduced in u_work).
+// low-rank down-projection (partial sums over N tiles added into u_work,
+// converted to lora_act by launch_lowrank_finalize afterwards).
 struct GeluQuantParams {
   const float* inv_smooth;    // down layer 1/lambda, fp32 [N]
   const uint16_t* l1t;        // down layer lora_down, fp16 [32, N]
   float s_d;                  // down layer activation tensor scale
   float lr_in_scale;          // 2^-e applied before the fp16 conversion
-  float lora_scale;           // 2^e / (s_d s_w_down)
   uint8_t* codes;             // [M, N/2]
   uint8_t* scales;            // tiled e4m3 with K = N, rows padded to 256
-  uint16_t* lora_act;         // bf16 [M, 64] (hi | lo)
   float* u_work;              // fp32 [M, 32], zero at launch
-  unsigned int* counters;     // one per 32 rows, zero at launch
 };
 
 struct GemmNvfp4Params {
@@ -69,6 +67,9 @@ cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int 
 // Same mainloop, GELU-MLP epilogue (t.y unused).
 cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                                    bool pdl);
+// lora_act bf16 [M, 64] = [hi | lo] of u_work [M, 32] * lora_scale.
+cudaError_t launch_lowrank_finalize(const float* u_work, int M, float lora_scale, uint16_t* lora_act,
+                                    cudaStream_t stream, bool pdl);
 
 // The CTA-pair kernel: B and [L2^T|L2^T] boxes are 128 rows (half a tile),
 // block scales are read through 2D maps of 256-byte rows (box 256 x 8).

@@ -211,8 +211,10 @@ int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const
  * next_lora_down [r, N] as packed) with fp32 accumulation.  The sum over N of
  * the low-rank partials uses fp32 atomic adds, so next_lora_act can differ
  * between runs in its last bits; codes and scales are deterministic.
- * `work` is device scratch of svdq_gelu_quant_work_bytes(M) bytes that the
- * call zeroes on `stream` before use; calls sharing it must not overlap.
+ * `work` is device scratch of svdq_gelu_quant_work_bytes(M) bytes (the fp32
+ * low-rank sums) that the call zeroes on `stream` before use; calls sharing
+ * it must not overlap.  The call launches a memset, the GEMM and a small
+ * kernel that converts the sums to next_lora_act.
  * The outputs feed svdq_w4a4_gemm of the next layer directly.
  * Shapes: M >= 1, N % 256 == 0 (N is the next layer's K), K % 256 == 0,
  * rank == SVDQ_RANK.  NVFP4 only; scales in [2^-100, 2^100). */
