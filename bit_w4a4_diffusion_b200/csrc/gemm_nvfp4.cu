@@ -217,6 +217,17 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
   const int num_tiles = tiles_m * tiles_n;
   const int k_tiles = p.K / 256;
   const int slices = k_tiles + 1;  // + the low-rank slice
+  // Tile schedule.  Plain epilogue: round robin over tiles numbered M-block
+  // fastest.  GELU-MLP epilogue: CTA i takes the contiguous run
+  // [i T / G, (i + 1) T / G) of tiles numbered N-block fastest, so that its
+  // consecutive tiles share an M-block and the epilogue can carry the
+  // low-rank partial of those rows from tile to tile.  (All operands of one
+  // layer fit in L2, so the order does not change DRAM traffic.)
+  const int t_begin = kGelu ? (int)((long long)blockIdx.x * num_tiles / gridDim.x) : (int)blockIdx.x;
+  const int t_end = kGelu ? (int)((long long)(blockIdx.x + 1) * num_tiles / gridDim.x) : num_tiles;
+  const int t_step = kGelu ? 1 : (int)gridDim.x;
+  auto tile_m0 = [&](int tile) { return (kGelu ? tile / tiles_n : tile % tiles_m) * BM; };
+  auto tile_n0 = [&](int tile) { return (kGelu ? tile % tiles_n : tile / tiles_m) * BN; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -264,9 +275,9 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage: load outstanding, its parity
       bool ok = true;
       const uint64_t pol_w = policy_evict_last();
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % tiles_m) * BM;
-        const int n0 = (tile / tiles_m) * BN;
+      for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
+        const int m0 = tile_m0(tile);
+        const int n0 = tile_n0(tile);
         for (int kt = 0; kt < slices; ++kt) {
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
             ok = false;
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
       bool ok = true;
       int it = 0;
       uint32_t ks = 0;  // K slices computed so far (selects the scale buffer)
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = t_begin; tile < t_end && ok; tile += t_step, ++it) {
         const uint32_t d_tmem = tmem + (uint32_t)((it & 1) * ACC_STRIDE);
         if (!mbar_wait(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
           ok = false;
@@ -376,7 +387,7 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, ks = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
         for (int kt = 0; kt < slices; ++kt) {
           if (kt > 0) {
             const uint32_t buf = ks & 1;
@@ -429,9 +440,10 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     // columns 4c..4c+3 of the 16 as its k values (a permutation of k shared by
     // both operands), so its A and B fragments are 8-byte loads.  The tile's
     // 1/lambda and bias columns are staged once per tile in shared memory.
-    // After the tile the partial sums go to u_work with vector reductions
-    // (fire and forget: the conversion to lora_act is a separate kernel that
-    // runs after this grid).  The eight warps share named barriers 2 and 3,
+    // The partial sums of consecutive tiles of one M-block stay in registers
+    // and go to u_work with vector reductions when the M-block changes (fire
+    // and forget: the conversion to lora_act is a separate kernel that runs
+    // after this grid).  The eight warps share named barriers 2 and 3,
     // so every stop decision is taken by all of them.
     constexpr int NT = R::EPI_WARPS * 32;
     const int q = warp & 3, hf = warp >> 2;
@@ -452,9 +464,34 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     constexpr int CPW = NCH / 2;  // chunks per warp
     constexpr int NBUF = 3;
     static_assert(NSH <= NBUF && NBUF <= CPW, "the shared chunks fit the first ring fill of half 0");
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int m0 = (tile % tiles_m) * BM;
-      const int n0 = (tile / tiles_m) * BN;
+    // The warp's low-rank partial of its 32 rows: rows 16t + g (+8), ranks
+    // 8j + 2c (+1); added into u_work when the M-block changes and at the end.
+    float lacc[2][4][4];
+    auto zero_lacc = [&]() {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lacc[t][j][e] = 0.f;
+    };
+    auto flush_lacc = [&](int mb) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r0 = mb + 32 * q + 16 * t + g;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = 8 * j + 2 * c;
+          if (r0 < p.M) red_add_f32x2(gq.u_work + (size_t)r0 * 32 + col, lacc[t][j][0], lacc[t][j][1]);
+          if (r0 + 8 < p.M) red_add_f32x2(gq.u_work + (size_t)(r0 + 8) * 32 + col, lacc[t][j][2], lacc[t][j][3]);
+        }
+      }
+    };
+    zero_lacc();
+    int cur_m0 = -1;
+    for (int tile = t_begin; tile < t_end; tile += t_step, ++it) {
+      const int m0 = tile_m0(tile);
+      const int n0 = tile_n0(tile);
       const int b = it & 1;
       const int row = m0 + 32 * q + lane;
       const bool row_ok = row < p.M;
@@ -469,13 +506,11 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
       tab_bias[et] = my_bias;
       asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory");
       tc_fence_after();
-      float lacc[2][4][4];
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) lacc[t][j][e] = 0.f;
+      if (m0 != cur_m0) {
+        if (cur_m0 >= 0) flush_lacc(cur_m0);
+        zero_lacc();
+        cur_m0 = m0;
+      }
       const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
       // Ring order: the shared columns first (the last ACC_OVERLAP of
       // accumulator 0, the first ACC_OVERLAP of accumulator 1).
@@ -591,19 +626,9 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
         // Refill the block just converted with the chunk three ahead.
         if (ii + NBUF < CPW) tmem_ld_32x32b_x32(acc_base + chunk_col(i0 + ii + NBUF) * LDC, r);
       }
-      // The warp's low-rank partial: rows 16t + g (+8), ranks 8j + 2c (+1).
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int r0 = m0 + 32 * q + 16 * t + g;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int col = 8 * j + 2 * c;
-          if (r0 < p.M) red_add_f32x2(gq.u_work + (size_t)r0 * 32 + col, lacc[t][j][0], lacc[t][j][1]);
-          if (r0 + 8 < p.M) red_add_f32x2(gq.u_work + (size_t)(r0 + 8) * 32 + col, lacc[t][j][2], lacc[t][j][3]);
-        }
-      }
       acc_phase ^= 1;
     }
+    if (cur_m0 >= 0) flush_lacc(cur_m0);
     } else {
     // -------------------------------------------------------------- epilogue
     // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile,
@@ -622,9 +647,9 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     constexpr int NSH = (ACC_OVERLAP + LDC - 1) / LDC;  // chunks holding shared columns
     constexpr int NBUF = 3;
     static_assert(NSH <= NBUF, "the shared chunks fit the first ring fill");
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int m0 = (tile % tiles_m) * BM;
-      const int n0 = (tile / tiles_m) * BN;
+    for (int tile = t_begin; tile < t_end; tile += t_step, ++it) {
+      const int m0 = tile_m0(tile);
+      const int n0 = tile_n0(tile);
       const int b = it & 1;
       uint4 bias8 = make_uint4(0, 0, 0, 0);
       if (p.bias != nullptr && n0 + 8 * lane < p.N) bias8 = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
