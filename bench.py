@@ -41,12 +41,12 @@ L2_BYTES = 126 * 2 ** 20
 # it was taken from: once a source changes the figure no longer applies and
 # the bench reports null.
 GEMM_TRAFFIC = {
-    "bytes": 30494976 + 53262848,
+    "bytes": 30496768 + 52880384,
     "sources": {
         "bit_w4a4_diffusion_b200/csrc/gemm_nvfp4.cu":
-            "0e287ef39c67008611952698abdd2bd3d107f7addebb3afdeb4f0de9137df015",
+            "fa8b08a092104da3a5da49a717ad6e601b015c1ae21161ac0cc705dc69f93f47",
         "bit_w4a4_diffusion_b200/csrc/ptx.cuh":
-            "606656540d9b84a2048833a8cc34bab5e89372da375464192b196a3f4bcd39c1",
+            "9f85b0a5d89f666dbb1ded5928e19d0fede8af584361f283b893195e630aaa34",
     },
 }
 
@@ -419,21 +419,50 @@ def measure_rows(B, wl, dev, peaks):
     return rows
 
 
-def measure_mlp(B, wl, dev):
-    """The DiT MLP block x [4096, 3072] -> 12288 -> 3072, fused (the GELU
-    and the down layer's activation quantizer in the up GEMM's epilogue) and
-    unfused (up layer -> bf16 y -> GELU -> down layer; the GELU there is
-    torch's, for comparison only).  Two rotating weight sets."""
+def mlp_inputs(B, wl, dev, nset):
+    """The DiT MLP block x [4096, 3072] -> 12288 -> 3072 (up: the mlp_up
+    workload with a bias; down: the mlp_down workload's weights and
+    calibration), `nset` device copies of both layers' packed weights."""
     import dataclasses
-    import torch
     iu = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_up"], bias_std=0.1))
     idn = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_down"], bias_std=0.05))
-    M, K, N = iu.case.M, iu.case.K, iu.case.N
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
-    nset = 2
     wus = [B.to_device(pk_u, dev) for _ in range(nset)]
     wds = [B.to_device(pk_d, dev) for _ in range(nset)]
+    return iu, idn, pk_u, wus, wds
+
+
+def run_mlp_calls(calls):
+    """`calls` back-to-back fused MLP calls on the DiT MLP workload, no
+    timing (the command that the MLP profiles are taken with)."""
+    import torch
+    import bit_w4a4_diffusion_b200 as B
+    import workloads as wl
+    dev = torch.device("cuda:0")
+    iu, idn, pk_u, wus, wds = mlp_inputs(B, wl, dev, 1)
+    M, K, N = iu.case.M, iu.case.K, iu.case.N
+    x = B.bits_to_bf16(iu.x_bits, dev)
+    b_u = B.bits_to_bf16(iu.bias_bits, dev)
+    b_d = B.bits_to_bf16(idn.bias_bits, dev)
+    y = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(B.mlp_workspace_bytes(M, K, N), dtype=torch.uint8, device=dev)
+    for _ in range(calls):
+        B.svdq_w4a4_mlp_gelu(x, wus[0], float(iu.act_scale), wds[0], float(idn.act_scale), up_bias=b_u,
+                             down_bias=b_d, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"mlp_calls": calls, "workload": f"x [{M},{K}] -> {N} -> {K}"}), flush=True)
+
+
+def measure_mlp(B, wl, dev):
+    """The DiT MLP block, fused (the GELU and the down layer's activation
+    quantizer in the up GEMM's epilogue) and unfused (up layer -> bf16 y ->
+    GELU -> down layer; the GELU there is torch's, for comparison only).  Two
+    rotating weight sets."""
+    import torch
+    nset = 2
+    iu, idn, pk_u, wus, wds = mlp_inputs(B, wl, dev, nset)
+    M, K, N = iu.case.M, iu.case.K, iu.case.N
     x = B.bits_to_bf16(iu.x_bits, dev)
     b_u = B.bits_to_bf16(iu.bias_bits, dev)
     b_d = B.bits_to_bf16(idn.bias_bits, dev)
@@ -483,10 +512,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ row measurements")
+    ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ / MLP row measurements")
+    ap.add_argument("--mlp-calls", type=int, default=0,
+                    help="only run this many fused DiT MLP calls (untimed; for profiling) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.mlp_calls > 0:
+        run_mlp_calls(args.mlp_calls)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

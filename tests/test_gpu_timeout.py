@@ -1,9 +1,9 @@
-"""Failure detection without a GPU fault: every mbarrier wait in the NVFP4
-and INT4 GEMM kernels is bounded by the library's wait limit.  With the limit
-set to 1 ns the first wait that is not already satisfied gives up; the kernel
-must report a timeout code through dev_status, drain its own copies and MMAs,
-free its tensor memory and return, leaving the context usable: the next call
-with the normal limit gives the correct result."""
+"""Failure detection without a GPU fault: every mbarrier wait in the NVFP4,
+INT4 and GELU-MLP GEMM kernels is bounded by the library's wait limit.  With
+the limit set to 1 ns the first wait that is not already satisfied gives up;
+the kernel must report a timeout code through dev_status, drain its own
+copies and MMAs, free its tensor memory and return, leaving the context
+usable: the next call with the normal limit gives the correct result."""
 import numpy as np
 import pytest
 import torch
@@ -80,3 +80,40 @@ def test_int4_gemm_wait_timeout_reports_and_recovers():
     act = O.quantize_activations("int4", inp.x, ref_pw["inv_lam"], np.float32(1.0))
     y64 = O.linear_f64("int4", act, ref_pw, inp.L1, inp.L2, inp.bias)
     assert_output_close(y.float().cpu().numpy(), y64, "INT4 GEMM after a timed-out call")
+
+
+def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
+    """The GELU-MLP kernel (eight epilogue warps that stop together)."""
+    import dataclasses
+    import bit_w4a4_diffusion_b200 as B
+    up = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=640, K=768, N=1024), bias_std=0.1)
+    dn = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=640, K=1024, N=768), bias_std=0.05)
+    iu, idn = wl.make_svdq_inputs(up), wl.make_svdq_inputs(dn)
+    pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
+    pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
+    wu, wd = B.to_device(pk_u), B.to_device(pk_d)
+    x = B.bits_to_bf16(iu.x_bits, "cuda")
+    b_u = B.bits_to_bf16(iu.bias_bits, "cuda")
+    s_a = float(iu.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, wu["inv_smooth"], wu["lora_down"], s_a, wu["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk_u["weight_scale"][0])))
+    torch.cuda.synchronize()
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, alpha, wd, float(idn.act_scale), bias=b_u,
+                                    dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+
+    status.zero_()
+    hc, hs, hl = B.svdq_w4a4_gemm_gelu_quant(codes, scales, lora, wu, alpha, wd, float(idn.act_scale), bias=b_u,
+                                             dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    from tests.test_gpu_mlp import _check_hidden
+    _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl)
