@@ -416,7 +416,101 @@ def measure_rows(B, wl, dev, peaks):
         del ws, ys
     rows["svdq_w4a4 int4 K=N=3072 (quantize + i8 GEMM)"] = int4
     rows["mlp_gelu"] = measure_mlp(B, wl, dev)
+    rows["dit_block"] = {f"M={M}": measure_block(B, wl, dev, M) for M in (4096, 1024)}
     return rows
+
+
+def block_layers(B, wl, dev, M):
+    """The linear layers of one DiT block at M tokens, hidden 3072: the
+    adaptive-norm modulation (awq_w4a16, 1 row -> 6 x 3072), the fused QKV
+    projection (3072 -> 9216), the attention output projection
+    (3072 -> 3072) and the GELU MLP (3072 -> 12288 -> 3072).  Attention,
+    norms and residual adds are not part of this library; each layer reads
+    its own synthetic input.  Returns a function that enqueues the block
+    (out: dict of output tensors)."""
+    import dataclasses
+    import torch
+    q = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M))
+    o = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, N=3072, name="attn_out"))
+    iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1))
+    idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05))
+    a = wl.make_awq_inputs(1)
+    wq, wo, wu, wd = (B.to_device(B.svdq_pack_weights("nvfp4", i.W_bits, i.lam, i.L1_bits, i.L2_bits), dev)
+                      for i in (q, o, iu, idn))
+    wa = B.to_device(B.awq_pack_weights(a.W_bits), dev)
+    xs = {k: B.bits_to_bf16(v, dev) for k, v in (("q", q.x_bits), ("o", o.x_bits), ("u", iu.x_bits),
+                                                    ("a", a.x_bits))}
+    bq = B.bits_to_bf16(q.bias_bits, dev) if q.bias_bits is not None else None
+    bo = B.bits_to_bf16(o.bias_bits, dev) if o.bias_bits is not None else None
+    bu, bd = B.bits_to_bf16(iu.bias_bits, dev), B.bits_to_bf16(idn.bias_bits, dev)
+    out = {"mod": torch.empty((1, a.N), dtype=torch.bfloat16, device=dev),
+           "qkv": torch.empty((M, 9216), dtype=torch.bfloat16, device=dev),
+           "attn_out": torch.empty((M, 3072), dtype=torch.bfloat16, device=dev),
+           "mlp": torch.empty((M, 3072), dtype=torch.bfloat16, device=dev)}
+    ws = torch.empty(max(B.workspace_bytes("nvfp4", M, 3072), B.mlp_workspace_bytes(M, 3072, 12288)),
+                     dtype=torch.uint8, device=dev)
+
+    def run():
+        B.awq_w4a16_linear(xs["a"], wa, y=out["mod"])
+        B.svdq_w4a4_linear("nvfp4", xs["q"], wq, float(q.act_scale), bias=bq, y=out["qkv"], workspace=ws)
+        B.svdq_w4a4_linear("nvfp4", xs["o"], wo, float(o.act_scale), bias=bo, y=out["attn_out"], workspace=ws)
+        B.svdq_w4a4_mlp_gelu(xs["u"], wu, float(iu.act_scale), wd, float(idn.act_scale), up_bias=bu,
+                             down_bias=bd, y=out["mlp"], workspace=ws)
+    flop = 2.0 * M * 3072 * (9216 + 3072 + 2 * 12288) + 2.0 * 18432 * 3072
+    return run, out, flop
+
+
+def measure_block(B, wl, dev, M, blocks=20):
+    """One DiT block's linear layers, `blocks` blocks back to back: eager
+    (each layer call launches its kernels) against one CUDA graph per block,
+    each with and without programmatic dependent launch (SVDQ_PDL=0)."""
+    import torch
+    run, out, flop = block_layers(B, wl, dev, M)
+    res = {}
+    for pdl in (True, False):
+        if pdl:
+            os.environ.pop("SVDQ_PDL", None)
+        else:
+            os.environ["SVDQ_PDL"] = "0"
+        try:
+            for _ in range(3):
+                run()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(50_000_000)  # let the host queue the eager launches ahead
+            e0.record()
+            for _ in range(blocks):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+            eager = e0.elapsed_time(e1) * 1e3 / blocks
+            g = torch.cuda.CUDAGraph()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                run()
+                torch.cuda.synchronize()
+                with torch.cuda.graph(g, stream=s):
+                    run()
+            torch.cuda.current_stream().wait_stream(s)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(blocks):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            graph = e0.elapsed_time(e1) * 1e3 / blocks
+            del g
+        finally:
+            os.environ.pop("SVDQ_PDL", None)
+        tag = "pdl" if pdl else "no_pdl"
+        res[f"eager_{tag}_us"] = round(eager, 2)
+        res[f"graph_{tag}_us"] = round(graph, 2)
+    res["graph_pdl_TFLOPS"] = round(flop / res["graph_pdl_us"] / 1e6, 1)
+    res["layers"] = "awq_w4a16 1x3072->18432, qkv 3072->9216, attn_out 3072->3072, GELU MLP 3072->12288->3072"
+    return res
 
 
 def mlp_inputs(B, wl, dev, nset):

@@ -86,6 +86,13 @@ int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
 unsigned long long svdq_timeout_ns() { return g_timeout_ns.load(std::memory_order_relaxed); }
 
+// Programmatic dependent launch for every kernel unless SVDQ_PDL=0 (read at
+// every call, so a process can compare the two).
+bool pdl_on() {
+  const char* v = getenv("SVDQ_PDL");
+  return !(v && strcmp(v, "0") == 0);
+}
+
 int check_cuda(cudaError_t e, const char* what) {
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return SVDQ_OK;
@@ -218,10 +225,10 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
     ok &= encode_tmap_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, lora_down, K, SVDQ_RANK, (uint64_t)K * 2, 64, 32,
                          CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the quantize kernel");
-    return check_cuda(launch_quantize_nvfp4(p, tx, tl, nullptr, svdq_timeout_ns(), static_cast<cudaStream_t>(stream)),
+    return check_cuda(launch_quantize_nvfp4(p, tx, tl, nullptr, svdq_timeout_ns(), static_cast<cudaStream_t>(stream), pdl_on()),
                       "quantize_nvfp4 launch");
   }
-  return check_cuda(launch_quantize_act(p, precision == SVDQ_NVFP4, static_cast<cudaStream_t>(stream)),
+  return check_cuda(launch_quantize_act(p, precision == SVDQ_NVFP4, static_cast<cudaStream_t>(stream), pdl_on()),
                     "quantize_act launch");
 }
 
@@ -348,9 +355,9 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
   if (int s = check_device(&sms)) return s;
   if (precision == SVDQ_INT4)
     return gemm_int4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, y, dev_status,
-                          static_cast<cudaStream_t>(stream), false, sms);
+                          static_cast<cudaStream_t>(stream), pdl_on(), sms);
   return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, y,
-                         dev_status, static_cast<cudaStream_t>(stream), false, sms);
+                         dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);
 }
 
 int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
@@ -378,9 +385,9 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   if (int s = check_device(&sms)) return s;
   if (precision == SVDQ_INT4)
     return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
-                          static_cast<cudaStream_t>(stream), true, sms);
+                          static_cast<cudaStream_t>(stream), pdl_on(), sms);
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
-                         y, dev_status, static_cast<cudaStream_t>(stream), true, sms);
+                         y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);
 }
 
 // ------------------------------------------------------------------ GELU-MLP fusion
@@ -435,7 +442,7 @@ static int launch_gelu_quant(int M, int N, int K, const void* act_codes, const v
     return s;
   const float lora_scale = ldexpf(1.0f, e) / (next_act_scale * next_weight_scale);
   return check_cuda(launch_lowrank_finalize(g.u_work, M, lora_scale, static_cast<uint16_t*>(next_lora_act), stream,
-                                            true),
+                                            pdl_on()),
                     "low-rank finalize launch");
 }
 
@@ -482,7 +489,7 @@ int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_cod
   if (int s = gelu_quant_prepare(M, N, next_act_scales, work, st)) return s;
   return launch_gelu_quant(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha,
                            next_inv_smooth, next_lora_down, next_act_scale, next_weight_scale, next_act_codes,
-                           next_act_scales, next_lora_act, work, dev_status, st, false, sms);
+                           next_act_scales, next_lora_act, work, dev_status, st, pdl_on(), sms);
 }
 
 long long svdq_mlp_workspace_bytes(int M, int K, int N_hidden, int rank) {
@@ -538,10 +545,10 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
     return s;
   if (int s = launch_gelu_quant(M, N, K, a_codes, a_scales, a_lora, up_w_codes, up_w_scales, up_lora_up, up_bias,
                                 up_alpha, down_inv_smooth, down_lora_down, down_act_scale, down_weight_scale, h_codes,
-                                h_scales, h_lora, work, dev_status, st, true, sms))
+                                h_scales, h_lora, work, dev_status, st, pdl_on(), sms))
     return s;
   return gemm_nvfp4_impl(M, K, N, h_codes, h_scales, h_lora, down_w_codes, down_w_scales, down_lora_up, down_bias,
-                         down_act_scale * down_weight_scale, y, dev_status, st, true, sms);
+                         down_act_scale * down_weight_scale, y, dev_status, st, pdl_on(), sms);
 }
 
 int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, const void* scales, const void* zeros,
@@ -566,7 +573,7 @@ int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, co
     p.zeros = static_cast<const uint8_t*>(zeros);
     p.bias = static_cast<const uint16_t*>(bias);
     p.y = static_cast<uint16_t*>(y) + (size_t)m0 * N;
-    if (int s = check_cuda(launch_awq(p, sms, static_cast<cudaStream_t>(stream)), "awq launch")) return s;
+    if (int s = check_cuda(launch_awq(p, sms, static_cast<cudaStream_t>(stream), pdl_on()), "awq launch")) return s;
   }
   return SVDQ_OK;
 }

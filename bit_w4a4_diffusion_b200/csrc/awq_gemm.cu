@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(AWQ_WARPS * 32) awq_kernel(AwqParams p) {
   const int n0 = blockIdx.x * AWQ_ROWS;
   const int rA = n0 + g, rB = n0 + g + 8;
   const int K = p.K;
+  pdl_wait();  // x of the previous kernel's making
   const int ngroups = K / 64;
   const int gpw = (ngroups + AWQ_WARPS - 1) / AWQ_WARPS;  // groups per warp
   const int G_begin = warp * gpw;
@@ -170,14 +171,16 @@ __global__ void __launch_bounds__(AWQ_WARPS * 32) awq_kernel(AwqParams p) {
 
 }  // namespace
 
-cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream, bool pdl) {
   (void)num_sms;
-  dim3 grid(p.N / AWQ_ROWS);
-  if (p.M <= 8)
-    awq_kernel<1><<<grid, AWQ_WARPS * 32, 0, stream>>>(p);
-  else
-    awq_kernel<2><<<grid, AWQ_WARPS * 32, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.N / AWQ_ROWS);
+  cfg.blockDim = dim3(AWQ_WARPS * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_pdl(cfg, attr, pdl);
+  if (p.M <= 8) return cudaLaunchKernelEx(&cfg, awq_kernel<1>, p);
+  return cudaLaunchKernelEx(&cfg, awq_kernel<2>, p);
 }
 
 }  // namespace svdq

@@ -139,6 +139,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   pdl_wait();
+  // The next kernel on the stream may be scheduled from now on; it waits for
+  // this grid's completion before it reads anything.
+  pdl_launch_dependents();
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
   const size_t mpad = (size_t)p.M_pad, npad = (size_t)p.N_pad;
 

@@ -157,6 +157,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // Inputs produced by the preceding quantize kernel become visible here.
   pdl_wait();
+  // The next kernel on the stream may be scheduled from now on; it waits for
+  // this grid's completion before it reads anything.
+  pdl_launch_dependents();
 
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
 

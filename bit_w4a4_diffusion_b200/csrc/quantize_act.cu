@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
   const int row1 = row0 + 8;
   const bool ok0 = row0 < p.M, ok1 = row1 < p.M;
   const int K = p.K;
+  pdl_wait();  // x and the weights of the previous kernel's making
   const int nunits = K / (32 * STEP);
 
   const uint16_t* __restrict__ x = p.x;
@@ -357,21 +358,26 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
 
 }  // namespace
 
-cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream) {
+cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl) {
   const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
   dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS);
   const size_t ring_bytes = (size_t)S1_PREFETCH * (nvfp4 ? 1 : 2) * S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(S1_THREADS);
+  cfg.dynamicSmemBytes = ring_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_pdl(cfg, attr, pdl);
   cudaError_t e;
   if (nvfp4) {
     e = cudaFuncSetAttribute(quantize_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ring_bytes);
     if (e != cudaSuccess) return e;
-    quantize_act_kernel<true><<<grid, S1_THREADS, ring_bytes, stream>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(quantize_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ring_bytes);
-    if (e != cudaSuccess) return e;
-    quantize_act_kernel<false><<<grid, S1_THREADS, ring_bytes, stream>>>(p);
+    return cudaLaunchKernelEx(&cfg, quantize_act_kernel<true>, p);
   }
-  return cudaGetLastError();
+  e = cudaFuncSetAttribute(quantize_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ring_bytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, quantize_act_kernel<false>, p);
 }
 
 }  // namespace svdq

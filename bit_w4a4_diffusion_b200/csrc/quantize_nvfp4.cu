@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
   const int K = p.K;
   const int nslices = K / QN_SLICE;
   const int row_base = blockIdx.x * QN_ROWS;
+  pdl_wait();  // x of the previous kernel's making
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QN_STAGES; ++s) {
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
 }  // namespace
 
 cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_l1t,
-                                  int* dev_status, unsigned long long timeout_ns, cudaStream_t stream) {
+                                  int* dev_status, unsigned long long timeout_ns, cudaStream_t stream, bool pdl) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -317,9 +318,14 @@ cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid(p.M_pad / QN_ROWS);  // covers the scale padding rows (zero scales)
-  quantize_nvfp4_kernel<<<grid, QN_THREADS, QN_SMEM_BYTES, stream>>>(tm_x, tm_l1t, p, dev_status, timeout_ns);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.M_pad / QN_ROWS);  // covers the scale padding rows (zero scales)
+  cfg.blockDim = dim3(QN_THREADS);
+  cfg.dynamicSmemBytes = QN_SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_pdl(cfg, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, quantize_nvfp4_kernel, tm_x, tm_l1t, p, dev_status, timeout_ns);
 }
 
 }  // namespace svdq

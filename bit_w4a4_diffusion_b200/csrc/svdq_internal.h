@@ -6,6 +6,17 @@
 
 namespace svdq {
 
+// Every kernel of the library waits for its stream predecessor with
+// griddepcontrol.wait before it touches global memory, so any launch may
+// carry the programmatic-dependent-launch attribute: the kernel's prologue
+// then overlaps the predecessor's tail.
+inline void set_pdl(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[1], bool pdl) {
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+}
+
 // Device-status codes written by bounded waits (0 = fine).
 enum DeviceStatus : int {
   kDevOk = 0,
@@ -28,10 +39,10 @@ struct QuantActParams {
   uint16_t* lora_act;         // bf16 [M, 2r]  (hi | lo)
 };
 
-cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream);
+cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl);
 // NVFP4, TMA-fed: x [M, K] bf16 and L1^T [32, K] fp16 as 64 x 32 SWIZZLE_128B boxes.
 cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_l1t,
-                                  int* dev_status, unsigned long long timeout_ns, cudaStream_t stream);
+                                  int* dev_status, unsigned long long timeout_ns, cudaStream_t stream, bool pdl);
 
 // The GELU-MLP epilogue: the up layer's output never leaves the chip; the
 // epilogue applies GELU and the down layer's smoothing, quantizer and
@@ -106,7 +117,7 @@ struct AwqParams {
   uint16_t* y;             // bf16 [M, N]
 };
 
-cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream, bool pdl);
 
 // Records a message for svdq_last_error() and returns `status`.
 int record_error(int status, const char* fmt, ...);

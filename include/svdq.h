@@ -31,6 +31,10 @@
  *    caller reads it after synchronizing and should clear it beforehand.
  *  - Device calls require a compute-capability 10.0 GPU (B200) as the
  *    current device, else SVDQ_ERR_UNSUPPORTED_DEVICE.  There is no fallback.
+ *  - Every kernel is launched with programmatic dependent launch: it may be
+ *    scheduled while the previous work on the stream finishes, and waits for
+ *    that work's completion before it touches global memory.  Setting the
+ *    environment variable SVDQ_PDL=0 launches plainly (read at every call).
  */
 #ifndef SVDQ_H
 #define SVDQ_H
