@@ -55,6 +55,9 @@ def _load():
         "svdq_mlp_workspace_bytes": (LL, [I, I, I, I]),
         "svdq_w4a4_mlp_gelu": (I, [I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, F, P, P, F, P, P, P, P, LL, P,
                                    P]),
+        "svdq_w4a4_gemm_qkv_norm_rope": (I, [I, I, I, I, P, P, P, P, P, P, P, F, I, I, P, P, P, P, P, P, P]),
+        "svdq_w4a4_qkv_norm_rope_linear": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, P, P, P, P, LL, P,
+                                               P]),
         "svdq_noalloc_scratch_bytes": (LL, []),
         "svdq_w4a4_linear_noalloc": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, P]),
         "awq_pack_weights": (I, [I, I, P, P, P, P]),
@@ -321,6 +324,41 @@ def svdq_w4a4_mlp_gelu(x, w_up, up_act_scale, w_down, down_act_scale, up_bias=No
                                   _ptr(w_down["codes"]), _ptr(w_down["scales"]), w_down["weight_scale_f"],
                                   _ptr(w_down["lora_up"]), _ptr(down_bias), _ptr(y), _ptr(workspace),
                                   workspace.numel(), _ptr(dev_status), _stream(stream)))
+    return y
+
+
+def svdq_w4a4_gemm_qkv_norm_rope(act_codes, act_scales, lora_act, w, alpha, heads, gamma_q, gamma_k, rope_cos,
+                                 rope_sin, bias=None, y=None, dev_status=None, stream=None, head_dim=128):
+    """The fused QKV projection's GEMM with RMSNorm (Q, K heads) and RoPE in
+    its epilogue; w: device dict of the [3 * heads * head_dim, K] layer."""
+    M = act_codes.shape[0]
+    N, K, rank = w["N"], w["K"], w["rank"]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=act_codes.device)
+    _check(lib.svdq_w4a4_gemm_qkv_norm_rope(M, N, K, rank, _ptr(act_codes), _ptr(act_scales), _ptr(lora_act),
+                                            _ptr(w["codes"]), _ptr(w["scales"]), _ptr(w["lora_up"]), _ptr(bias),
+                                            float(alpha), int(heads), int(head_dim), _ptr(gamma_q), _ptr(gamma_k),
+                                            _ptr(rope_cos), _ptr(rope_sin), _ptr(y), _ptr(dev_status),
+                                            _stream(stream)))
+    return y
+
+
+def svdq_w4a4_qkv_norm_rope_linear(x, w, act_scale, heads, gamma_q, gamma_k, rope_cos, rope_sin, bias=None, y=None,
+                                   workspace=None, dev_status=None, stream=None, head_dim=128):
+    _dev_bf16(x, "x")
+    M, K = x.shape
+    N, rank = w["N"], w["rank"]
+    if K != w["K"] or N != 3 * int(heads) * int(head_dim):
+        raise SvdqError(2, f"weights [{N}, {w['K']}] do not match x [{M}, {K}] with {heads} heads of {head_dim}")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(SVDQ_NVFP4, M, K, rank), dtype=torch.uint8, device=x.device)
+    _check(lib.svdq_w4a4_qkv_norm_rope_linear(M, K, int(heads), int(head_dim), rank, _ptr(x), _ptr(w["inv_smooth"]),
+                                              _ptr(w["lora_down"]), float(act_scale), _ptr(w["codes"]),
+                                              _ptr(w["scales"]), w["weight_scale_f"], _ptr(w["lora_up"]), _ptr(bias),
+                                              _ptr(gamma_q), _ptr(gamma_k), _ptr(rope_cos), _ptr(rope_sin), _ptr(y),
+                                              _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream)))
     return y
 
 

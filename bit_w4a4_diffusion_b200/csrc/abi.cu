@@ -244,11 +244,12 @@ static bool use_pair_gemm() {
   return v && strcmp(v, "pair") == 0;
 }
 
-// gq != nullptr selects the GELU-MLP epilogue (single-CTA kernel; y unused).
+// gq != nullptr selects the GELU-MLP epilogue, qk != nullptr the QKV +
+// RMSNorm + RoPE epilogue (single-CTA kernel; y's tensor map unused).
 static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const void* act_scales, const void* lora_act,
                            const void* w_codes, const void* w_scales, const void* lora_up, const void* bias,
                            float alpha, void* y, int* dev_status, cudaStream_t stream, bool pdl, int sms,
-                           const GeluQuantParams* gq = nullptr) {
+                           const GeluQuantParams* gq = nullptr, const QkvParams* qk = nullptr) {
   GemmTmaps t;
   bool ok = true;
   ok &= encode_tmap_2d(&t.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_codes, K / 2, M, K / 2, 128, 128,
@@ -259,7 +260,7 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
                        128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64,
                        256, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (gq == nullptr)
+  if (gq == nullptr && qk == nullptr)
     ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
                          CU_TENSOR_MAP_SWIZZLE_32B);
   else
@@ -278,6 +279,10 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
   if (gq != nullptr) {
     p.gq = *gq;
     return check_cuda(launch_gemm_nvfp4_gelu(p, t, sms, stream, pdl), "gemm_nvfp4 (GELU-MLP epilogue) launch");
+  }
+  if (qk != nullptr) {
+    p.qk = *qk;
+    return check_cuda(launch_gemm_nvfp4_qkv(p, t, sms, stream, pdl), "gemm_nvfp4 (QKV epilogue) launch");
   }
   if (use_pair_gemm()) {
     // CTA-pair kernel: half-tile boxes for B and [L2^T|L2^T], and the block
@@ -549,6 +554,82 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
     return s;
   return gemm_nvfp4_impl(M, K, N, h_codes, h_scales, h_lora, down_w_codes, down_w_scales, down_lora_up, down_bias,
                          down_act_scale * down_weight_scale, y, dev_status, st, pdl_on(), sms);
+}
+
+// ------------------------------------------------------------------ QKV + RMSNorm + RoPE
+
+static int check_qkv_args(int M, int N, int K, int rank, int heads, int head_dim, const float* gamma_q,
+                          const float* gamma_k, const float* rope_cos, const float* rope_sin, void* y) {
+  if (head_dim != 128) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "head_dim=%d; this build supports 128", head_dim);
+  if (heads <= 0 || (long long)N != 3ll * heads * head_dim)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d must be 3 * heads * head_dim (heads=%d)", N, heads);
+  if (int s = check_gemm_args(SVDQ_NVFP4, M, N, K, rank)) return s;
+  if (!gamma_q || !gamma_k || !rope_cos || !rope_sin || !y) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(gamma_q) || !aligned16(gamma_k) || !aligned16(rope_cos) || !aligned16(rope_sin) || !aligned16(y))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return SVDQ_OK;
+}
+
+static QkvParams qkv_params(int heads, const float* gamma_q, const float* gamma_k, const float* rope_cos,
+                            const float* rope_sin, void* y) {
+  QkvParams q{};
+  q.gamma_q = gamma_q;
+  q.gamma_k = gamma_k;
+  q.rope_cos = rope_cos;
+  q.rope_sin = rope_sin;
+  q.eps = 1e-6f;
+  q.hd = heads * 128;
+  q.y = static_cast<uint16_t*>(y);
+  return q;
+}
+
+int svdq_w4a4_gemm_qkv_norm_rope(int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                                 const void* lora_act, const void* w_codes, const void* w_scales,
+                                 const void* lora_up, const void* bias, float alpha, int heads, int head_dim,
+                                 const float* gamma_q, const float* gamma_k, const float* rope_cos,
+                                 const float* rope_sin, void* y, int* dev_status, void* stream) {
+  if (int s = check_qkv_args(M, N, K, rank, heads, head_dim, gamma_q, gamma_k, rope_cos, rope_sin, y)) return s;
+  if (!act_codes || !act_scales || !lora_act || !w_codes || !w_scales || !lora_up)
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(act_codes) || !aligned16(act_scales) || !aligned16(lora_act) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(lora_up) || (bias && !aligned16(bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (!(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  const QkvParams q = qkv_params(heads, gamma_q, gamma_k, rope_cos, rope_sin, y);
+  return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, y,
+                         dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms, nullptr, &q);
+}
+
+int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int rank, const void* x,
+                                   const float* inv_smooth, const void* lora_down, float act_scale,
+                                   const void* w_codes, const void* w_scales, float weight_scale,
+                                   const void* lora_up, const void* bias, const float* gamma_q, const float* gamma_k,
+                                   const float* rope_cos, const float* rope_sin, void* y, void* workspace,
+                                   long long workspace_bytes, int* dev_status, void* stream) {
+  const int N = 3 * heads * head_dim;
+  if (int s = check_qkv_args(M, N, K, rank, heads, head_dim, gamma_q, gamma_k, rope_cos, rope_sin, y)) return s;
+  if (!workspace) return fail(SVDQ_ERR_INVALID_ARG, "null workspace");
+  const long long need = svdq_workspace_bytes(SVDQ_NVFP4, M, K, rank);
+  if (workspace_bytes < need)
+    return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (!w_codes || !w_scales || !lora_up) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || (bias && !aligned16(bias)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* codes = ws;
+  uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
+  uint8_t* lora = scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, K), 256);
+  if (int s = svdq_quantize_act(SVDQ_NVFP4, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
+                                scales, lora, stream))
+    return s;
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  const QkvParams q = qkv_params(heads, gamma_q, gamma_k, rope_cos, rope_sin, y);
+  return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
+                         y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms, nullptr, &q);
 }
 
 int awq_w4a16_linear(int M, int N, int K, const void* x, const void* qweight, const void* scales, const void* zeros,

@@ -58,16 +58,19 @@ constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;       // epilogue staging, 8 KB
 // block-scale copies 6-8.  GELU-MLP epilogue (12 warps, three warpgroups):
 // epilogue 0-7, producer 8, MMA 9, block-scale copies 10-11; the last
 // warpgroup hands registers to the two epilogue warpgroups (setmaxnreg).
-template <bool kGelu>
+// Epilogue kinds: y = bf16(alpha D + b); the GELU-MLP epilogue; the QKV
+// epilogue with RMSNorm and RoPE.  The last two use the wide layout.
+constexpr int EPI_PLAIN = 0, EPI_GELU = 1, EPI_QKV = 2;
+template <bool kWide>
 struct Roles {
-  static constexpr int EPI_WARPS = kGelu ? 8 : 4;
-  static constexpr int PRODUCER = kGelu ? 8 : 0;
-  static constexpr int MMA = kGelu ? 9 : 1;
-  static constexpr int SF_W0 = kGelu ? 10 : 6;
-  static constexpr int SF_WARPS = kGelu ? 2 : 3;
-  static constexpr int NUM_THREADS = (kGelu ? 12 : 9) * 32;
+  static constexpr int EPI_WARPS = kWide ? 8 : 4;
+  static constexpr int PRODUCER = kWide ? 8 : 0;
+  static constexpr int MMA = kWide ? 9 : 1;
+  static constexpr int SF_W0 = kWide ? 10 : 6;
+  static constexpr int SF_WARPS = kWide ? 2 : 3;
+  static constexpr int NUM_THREADS = (kWide ? 12 : 9) * 32;
 };
-// Register split of the GELU-MLP kernel: launched at 168 per thread
+// Register split of the wide layout: launched at 168 per thread
 // (12 warps x 32 x 168 = 64512), then 216 for each epilogue thread and 72 for
 // the rest: 256 x 216 + 128 x 72 = 64512.
 constexpr int GQ_LAUNCH_REGS = 168, GQ_EPI_REGS = 216, GQ_CTL_REGS = 72;
@@ -99,11 +102,12 @@ struct SmemCtl {
 // The GELU-MLP epilogue keeps the tile's 1/lambda (fp32) and bias (bf16)
 // columns in shared memory after the staging buffers.
 constexpr int GQ_TABLE_BYTES = BN * 4 + BN * 2;
-template <bool kGelu>
+template <int kEpi>
 constexpr size_t smem_bytes() {
-  return 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + (kGelu ? GQ_TABLE_BYTES : 0) + sizeof(SmemCtl);
+  return 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + (kEpi == EPI_GELU ? GQ_TABLE_BYTES : 0) +
+         sizeof(SmemCtl);
 }
-static_assert(smem_bytes<true>() <= 232448, "shared memory per block");
+static_assert(smem_bytes<EPI_GELU>() <= 232448, "shared memory per block");
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   block-scaled: a/b format E2M1 (=1) at bits 7/10, N>>3 at 17, UE4M3 scales
@@ -177,6 +181,14 @@ SVDQ_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// A read-only global load kept in program order with the other volatile
+// asm (so that the compiler does not hoist a whole head's worth of them).
+SVDQ_DEV float4 ldg_f4_ordered(const float* addr) {
+  float4 v;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(addr));
+  return v;
+}
+
 SVDQ_DEV void red_add_f32x2(float* addr, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
 }
@@ -199,8 +211,8 @@ SVDQ_DEV uint2 ld_shared_v2(uint32_t addr) {
   return v;
 }
 
-template <bool kGelu>
-__global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
+template <int kEpi>
+__global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                       const __grid_constant__ CUtensorMap tm_y, const GemmNvfp4Params p) {
@@ -208,9 +220,10 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
+  constexpr bool kGelu = kEpi == EPI_GELU, kQkv = kEpi == EPI_QKV, kWide = kEpi != EPI_PLAIN;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kGelu ? GQ_TABLE_BYTES : 0));
 
-  using R = Roles<kGelu>;
+  using R = Roles<kWide>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (p.M + BM - 1) / BM;
   const int tiles_n = (p.N + BN - 1) / BN;
@@ -250,7 +263,7 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_la);
     prefetch_tmap(&tm_lb);
-    if (!kGelu) prefetch_tmap(&tm_y);
+    if (kEpi == EPI_PLAIN) prefetch_tmap(&tm_y);
   }
   if (warp == R::MMA) {
     tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -632,6 +645,123 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
       acc_phase ^= 1;
     }
     if (cur_m0 >= 0) flush_lacc(cur_m0);
+    } else if constexpr (kQkv) {
+      // ------------------------------------------ QKV + RMSNorm + RoPE epilogue
+      // Eight warps: warp w reads TMEM lane quarter w mod 4 (32 rows) and head
+      // w / 4 of the tile (a 256-column tile holds two 128-feature heads).  A
+      // lane loads its row's whole head (128 registers) before the warp
+      // releases the accumulator, so the head holding the columns shared with
+      // the other accumulator is read in full first.  Per lane: v = alpha D + b
+      // on packed fp32x2; for Q and K heads the mean of v^2 over the head,
+      // v * rsqrt(mean + eps) * gamma, and the rotation of each pair (2i, 2i+1)
+      // by the row's cos / sin; bf16 stores straight to y.
+      const int q = warp & 3, hf = warp >> 2;
+      const QkvParams& qp = p.qk;
+      const float2 alpha2 = make_float2(p.alpha, p.alpha);
+      uint32_t acc_phase = 0;
+      int it = 0;
+      for (int tile = t_begin; tile < t_end; tile += t_step, ++it) {
+        const int m0 = tile_m0(tile);
+        const int n0 = tile_n0(tile);
+        const int b = it & 1;
+        const int row = m0 + 32 * q + lane;
+        const bool row_ok = row < p.M;
+        const int n = n0 + 128 * hf;  // first column of this warp's head
+        const bool head_ok = n < p.N;
+        const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
+        if (named_bar_any(2, R::EPI_WARPS * 32, !got)) break;
+        tc_fence_after();
+        const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE + 128 * hf);
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld_32x32b_x32(acc_base + 32 * c4, r[c4]);
+        tmem_ld_wait(r[0]);
+        reg_fence(r[1]);
+        reg_fence(r[2]);
+        reg_fence(r[3]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty));
+        acc_phase ^= 1;
+        if (!head_ok) continue;
+        const int part = n / qp.hd;  // 0: Q, 1: K, 2: V
+        // v = alpha D + b, in place
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8) {
+            const uint4 bw = p.bias != nullptr
+                                 ? __ldg(reinterpret_cast<const uint4*>(p.bias + n + 32 * c4 + 8 * k8))
+                                 : make_uint4(0, 0, 0, 0);
+            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = 8 * k8 + 2 * j;
+              const float2 v = __ffma2_rn(alpha2, make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])),
+                                          make_float2(__uint_as_float(bb[j] << 16), __uint_as_float(bb[j] & 0xFFFF0000u)));
+              r[c4][e] = __float_as_uint(v.x);
+              r[c4][e + 1] = __float_as_uint(v.y);
+            }
+          }
+        }
+        if (part < 2) {
+          float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v = make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1]));
+              ss = __ffma2_rn(v, v, ss);
+            }
+          const float ms = __fmul_rn(__fadd_rn(ss.x, ss.y), 1.0f / 128.0f);
+          const float rn = __frsqrt_rn(__fadd_rn(ms, qp.eps));
+          const float2 rn2 = make_float2(rn, rn);
+          const float* gamma = part == 0 ? qp.gamma_q : qp.gamma_k;
+          const float* cs = qp.rope_cos + (size_t)(row_ok ? row : 0) * 64;
+          const float* sn = qp.rope_sin + (size_t)(row_ok ? row : 0) * 64;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              // features 32 c4 + 8 k4 .. +7: pairs 16 c4 + 4 k4 .. +3
+              const float4 g0 = ldg_f4_ordered(gamma + 32 * c4 + 8 * k4);
+              const float4 g1 = ldg_f4_ordered(gamma + 32 * c4 + 8 * k4 + 4);
+              const float4 co = ldg_f4_ordered(cs + 16 * c4 + 4 * k4);
+              const float4 si = ldg_f4_ordered(sn + 16 * c4 + 4 * k4);
+              const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+              const float cc[4] = {co.x, co.y, co.z, co.w}, ssn[4] = {si.x, si.y, si.z, si.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int e = 8 * k4 + 2 * j;
+                const float2 u = __fmul2_rn(
+                    __fmul2_rn(make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])), rn2),
+                    make_float2(gg[2 * j], gg[2 * j + 1]));
+                // (a, b) -> (a cos - b sin, a sin + b cos)
+                const float x0 = __fmaf_rn(u.x, cc[j], -__fmul_rn(u.y, ssn[j]));
+                const float x1 = __fmaf_rn(u.x, ssn[j], __fmul_rn(u.y, cc[j]));
+                r[c4][e] = __float_as_uint(x0);
+                r[c4][e + 1] = __float_as_uint(x1);
+              }
+            }
+          }
+        }
+        if (row_ok) {
+          uint16_t* yrow = qp.y + (size_t)row * p.N + n;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+              uint32_t w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[c4][8 * k8 + 2 * j]),
+                                                          __uint_as_float(r[c4][8 * k8 + 2 * j + 1]));
+                w[j] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(yrow + 32 * c4 + 8 * k8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+      }
     } else {
     // -------------------------------------------------------------- epilogue
     // Each warp owns 32 rows (its TMEM lane quarter) x 256 columns of a tile,
@@ -732,7 +862,7 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
     }
   };
 
-  if constexpr (kGelu) {
+  if constexpr (kWide) {
     // setmaxnreg is warpgroup-wide: the last warpgroup (producer, MMA, scale
     // copies) gives registers to the two epilogue warpgroups.
     if (warp >= R::EPI_WARPS) {
@@ -770,19 +900,19 @@ __global__ void __launch_bounds__(Roles<kGelu>::NUM_THREADS, 1)
 }  // namespace
 
 namespace {
-template <bool kGelu>
+template <int kEpi>
 cudaError_t launch_impl(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream, bool pdl) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<kGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<kGelu>());
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_bytes<kEpi>());
     if (e != cudaSuccess) return e;
-    if (kGelu) {
+    if (kEpi != EPI_PLAIN) {
       // The epilogue warpgroups' setmaxnreg.inc waits until the others have
       // released enough registers: only launch if the compiled register
       // count makes the split add up.
       cudaFuncAttributes fa;
-      e = cudaFuncGetAttributes(&fa, gemm_nvfp4_kernel<kGelu>);
+      e = cudaFuncGetAttributes(&fa, gemm_nvfp4_kernel<kEpi>);
       if (e != cudaSuccess) return e;
       if (fa.numRegs * Roles<true>::NUM_THREADS < 256 * GQ_EPI_REGS + 128 * GQ_CTL_REGS)
         return cudaErrorInvalidConfiguration;
@@ -792,26 +922,31 @@ cudaError_t launch_impl(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sm
   const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles < num_sms ? tiles : num_sms);
-  cfg.blockDim = dim3(Roles<kGelu>::NUM_THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<kGelu>();
+  cfg.blockDim = dim3(Roles<kEpi != EPI_PLAIN>::NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<kEpi>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel<kGelu>, t.a, t.b, t.la, t.lb, t.y, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel<kEpi>, t.a, t.b, t.la, t.lb, t.y, p);
 }
 }  // namespace
 
 cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                               bool pdl) {
-  return launch_impl<false>(p, t, num_sms, stream, pdl);
+  return launch_impl<EPI_PLAIN>(p, t, num_sms, stream, pdl);
 }
 
 cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                                    bool pdl) {
-  return launch_impl<true>(p, t, num_sms, stream, pdl);
+  return launch_impl<EPI_GELU>(p, t, num_sms, stream, pdl);
+}
+
+cudaError_t launch_gemm_nvfp4_qkv(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                                  bool pdl) {
+  return launch_impl<EPI_QKV>(p, t, num_sms, stream, pdl);
 }
 
 namespace {

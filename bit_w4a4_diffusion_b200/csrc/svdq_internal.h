@@ -58,6 +58,19 @@ struct GeluQuantParams {
   float* u_work;              // fp32 [M, 32], zero at launch
 };
 
+// The QKV epilogue: columns [Q | K | V] of 128-feature heads; RMSNorm with
+// per-feature weights over each Q and K head, then rotation of the feature
+// pairs (2i, 2i + 1) by the token's angle; V gets only the bias.
+struct QkvParams {
+  const float* gamma_q;   // fp32 [128]
+  const float* gamma_k;   // fp32 [128]
+  const float* rope_cos;  // fp32 [M, 64]
+  const float* rope_sin;  // fp32 [M, 64]
+  float eps;
+  int hd;                 // columns per part: heads * 128
+  uint16_t* y;            // bf16 [M, N]
+};
+
 struct GemmNvfp4Params {
   int M, N, K;
   const uint8_t* act_scales;  // tiled e4m3, rows padded to 256
@@ -67,6 +80,7 @@ struct GemmNvfp4Params {
   int* dev_status;            // may be null
   unsigned long long timeout_ns;
   GeluQuantParams gq;         // used by the GELU-MLP epilogue only
+  QkvParams qk;               // used by the QKV epilogue only
 };
 
 struct GemmTmaps {
@@ -78,6 +92,9 @@ cudaError_t launch_gemm_nvfp4(const GemmNvfp4Params& p, const GemmTmaps& t, int 
 // Same mainloop, GELU-MLP epilogue (t.y unused).
 cudaError_t launch_gemm_nvfp4_gelu(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
                                    bool pdl);
+// Same mainloop, QKV + RMSNorm + RoPE epilogue (t.y unused).
+cudaError_t launch_gemm_nvfp4_qkv(const GemmNvfp4Params& p, const GemmTmaps& t, int num_sms, cudaStream_t stream,
+                                  bool pdl);
 // lora_act bf16 [M, 64] = [hi | lo] of u_work [M, 32] * lora_scale.
 cudaError_t launch_lowrank_finalize(const float* u_work, int M, float lora_scale, uint16_t* lora_act,
                                     cudaStream_t stream, bool pdl);

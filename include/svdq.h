@@ -250,6 +250,40 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
                        const void* down_lora_up, const void* down_bias, void* y, void* workspace,
                        long long workspace_bytes, int* dev_status, void* stream);
 
+/* ------------------------------------------------------------------ QKV + RMSNorm + RoPE
+ * "Nunchaku Lite" docs, section "Fused kernels": the original engine combines
+ * the Q, K and V projections with RMSNorm and RoPE.
+ *
+ * svdq_w4a4_gemm_qkv_norm_rope: the fused QKV projection's NVFP4 GEMM
+ * (svdq_w4a4_gemm's arguments up to alpha) whose output
+ *   v = alpha * ( sum_k deq(a) deq(w) + lora_act . lora_up^T ) + bias   (fp32)
+ * is, per row and before rounding, treated as [Q | K | V] with `heads` heads
+ * of head_dim = 128 features each (head h of a part in its columns
+ * [128 h, 128 h + 128)):
+ *   Q and K heads: u = v / sqrt(mean(v^2) + 1e-6) * gamma (gamma_q for Q,
+ *                  gamma_k for K, fp32 [128]), then each feature pair
+ *                  (u[2i], u[2i+1]) is rotated by the row's angle i:
+ *                  (a, b) -> (a cos - b sin, a sin + b cos) with
+ *                  cos = rope_cos[m][i], sin = rope_sin[m][i] (fp32 [M, 64]);
+ *   V heads:       unchanged;
+ * then rounded to bf16 into y [M, N].  N = 3 * heads * 128, K % 256 == 0.
+ *
+ * svdq_w4a4_qkv_norm_rope_linear: svdq_quantize_act of x then the call above,
+ * with svdq_w4a4_linear's arguments and workspace; the weights must be those
+ * of a [3 * heads * head_dim, K] layer (N is derived from heads, so the
+ * library cannot check it against the buffers). */
+int svdq_w4a4_gemm_qkv_norm_rope(int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
+                                 const void* lora_act, const void* w_codes, const void* w_scales,
+                                 const void* lora_up, const void* bias, float alpha, int heads, int head_dim,
+                                 const float* gamma_q, const float* gamma_k, const float* rope_cos,
+                                 const float* rope_sin, void* y, int* dev_status, void* stream);
+int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int rank, const void* x,
+                                   const float* inv_smooth, const void* lora_down, float act_scale,
+                                   const void* w_codes, const void* w_scales, float weight_scale,
+                                   const void* lora_up, const void* bias, const float* gamma_q, const float* gamma_k,
+                                   const float* rope_cos, const float* rope_sin, void* y, void* workspace,
+                                   long long workspace_bytes, int* dev_status, void* stream);
+
 /* ------------------------------------------------------------------ AWQ W4A16
  * "Nunchaku Lite" docs, "Supported quantization types" table: awq_w4a16,
  * int4, group size 64 -- an INT4 weight-only AWQ-style kernel for the

@@ -233,3 +233,16 @@ def make_awq_inputs(M, N=18432, K=3072, seed=4, with_bias=False):
 
 
 AWQ_MS = (1, 2, 8, 16)
+
+
+def make_rope_norm_inputs(M, heads, seed=5, head_dim=128, base=10000.0):
+    """Per-feature RMSNorm weights for Q and K heads (uniform in [0.5, 1.5])
+    and rotary tables of tokens 0..M-1: angle(m, i) = m * base^(-2i/head_dim),
+    as fp32 cos / sin [M, head_dim/2]."""
+    g = _rng(seed)
+    gamma_q = g.uniform(0.5, 1.5, head_dim).astype(np.float32)
+    gamma_k = g.uniform(0.5, 1.5, head_dim).astype(np.float32)
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    ang = np.arange(M, dtype=np.float64)[:, None] * base ** (-2.0 * i[None, :] / head_dim)
+    return gamma_q, gamma_k, np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
