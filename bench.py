@@ -416,14 +416,66 @@ def measure_rows(B, wl, dev, peaks):
         del ws, ys
     rows["svdq_w4a4 int4 K=N=3072 (quantize + i8 GEMM)"] = int4
     rows["mlp_gelu"] = measure_mlp(B, wl, dev)
+    rows["qkv_norm_rope"] = measure_qkv(B, wl, dev)
     rows["dit_block"] = {f"M={M}": measure_block(B, wl, dev, M) for M in (4096, 1024)}
     return rows
+
+
+def measure_qkv(B, wl, dev, heads=24):
+    """The DiT QKV projection (4096 tokens, 3072 -> 9216) with RMSNorm and
+    RoPE on its Q and K heads: fused in the GEMM's epilogue, against the
+    layer followed by the same normalization and rotation as separate torch
+    operations (for comparison only).  Two rotating weight sets."""
+    import torch
+    c = wl.SVDQ_CASES["qkv"]
+    M, K, N = c.M, c.K, c.N
+    inp = wl.make_svdq_inputs(c)
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    nset = 2
+    ws_ = [B.to_device(pk, dev) for _ in range(nset)]
+    gq, gk, cos_m, sin_m = wl.make_rope_norm_inputs(M, heads)
+    gq, gk = torch.from_numpy(gq).to(dev), torch.from_numpy(gk).to(dev)
+    cos = torch.from_numpy(np.ascontiguousarray(cos_m.T)).to(dev)      # pair-major [64, M]
+    sin = torch.from_numpy(np.ascontiguousarray(sin_m.T)).to(dev)
+    x = B.bits_to_bf16(inp.x_bits, dev)
+    bias = B.bits_to_bf16(inp.bias_bits, dev)
+    s_a = float(inp.act_scale)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wsp = torch.empty(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
+    hd = heads * 128
+
+    def torch_norm_rope(t, g):
+        t32 = t.float().view(M, heads, 128)
+        t32 = t32 * torch.rsqrt(t32.pow(2).mean(-1, keepdim=True) + 1e-6) * g
+        a, b = t32[..., 0::2], t32[..., 1::2]
+        c_, s_ = cos.t().reshape(M, 1, 64), sin.t().reshape(M, 1, 64)
+        return torch.stack((a * c_ - b * s_, a * s_ + b * c_), dim=-1).view(M, hd).to(torch.bfloat16)
+
+    def unfused(i):
+        B.svdq_w4a4_linear("nvfp4", x, ws_[i], s_a, bias=bias, y=y, workspace=wsp)
+        y[:, :hd] = torch_norm_rope(y[:, :hd], gq)
+        y[:, hd:2 * hd] = torch_norm_rope(y[:, hd:2 * hd], gk)
+
+    fused = [lambda i=i: B.svdq_w4a4_qkv_norm_rope_linear(x, ws_[i], s_a, heads, gq, gk, cos, sin, bias=bias, y=y,
+                                                          workspace=wsp) for i in range(nset)]
+    plain = [lambda i=i: B.svdq_w4a4_linear("nvfp4", x, ws_[i], s_a, bias=bias, y=y, workspace=wsp)
+             for i in range(nset)]
+    t_f = _event_time_us(torch, fused, 40)
+    t_p = _event_time_us(torch, plain, 40)
+    t_u = _event_time_us(torch, [lambda i=i: unfused(i) for i in range(nset)], 40)
+    flop = 2.0 * M * N * K
+    del ws_
+    return {"workload": f"x [{M},{K}] -> [{M},{N}], {heads} heads of 128, NVFP4 r32, bias",
+            "fused_us": round(t_f, 2), "fused_TFLOPS": round(flop / t_f / 1e6, 1),
+            "unfused_us": round(t_u, 2), "speedup": round(t_u / t_f, 3),
+            "layer_without_norm_rope_us": round(t_p, 2)}
 
 
 def block_layers(B, wl, dev, M):
     """The linear layers of one DiT block at M tokens, hidden 3072: the
     adaptive-norm modulation (awq_w4a16, 1 row -> 6 x 3072), the fused QKV
-    projection (3072 -> 9216), the attention output projection
+    projection with RMSNorm and RoPE on Q and K (3072 -> 9216, 24 heads),
+    the attention output projection
     (3072 -> 3072) and the GELU MLP (3072 -> 12288 -> 3072).  Attention,
     norms and residual adds are not part of this library; each layer reads
     its own synthetic input.  Returns a function that enqueues the block
@@ -435,6 +487,8 @@ def block_layers(B, wl, dev, M):
     iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1))
     idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05))
     a = wl.make_awq_inputs(1)
+    rq = [torch.from_numpy(np.ascontiguousarray(t.T if t.ndim == 2 else t)).to(dev)
+          for t in wl.make_rope_norm_inputs(M, 24)]
     wq, wo, wu, wd = (B.to_device(B.svdq_pack_weights("nvfp4", i.W_bits, i.lam, i.L1_bits, i.L2_bits), dev)
                       for i in (q, o, iu, idn))
     wa = B.to_device(B.awq_pack_weights(a.W_bits), dev)
@@ -452,7 +506,8 @@ def block_layers(B, wl, dev, M):
 
     def run():
         B.awq_w4a16_linear(xs["a"], wa, y=out["mod"])
-        B.svdq_w4a4_linear("nvfp4", xs["q"], wq, float(q.act_scale), bias=bq, y=out["qkv"], workspace=ws)
+        B.svdq_w4a4_qkv_norm_rope_linear(xs["q"], wq, float(q.act_scale), 24, *rq, bias=bq, y=out["qkv"],
+                                         workspace=ws)
         B.svdq_w4a4_linear("nvfp4", xs["o"], wo, float(o.act_scale), bias=bo, y=out["attn_out"], workspace=ws)
         B.svdq_w4a4_mlp_gelu(xs["u"], wu, float(iu.act_scale), wd, float(idn.act_scale), up_bias=bu,
                              down_bias=bd, y=out["mlp"], workspace=ws)
@@ -509,7 +564,8 @@ def measure_block(B, wl, dev, M, blocks=20):
         res[f"eager_{tag}_us"] = round(eager, 2)
         res[f"graph_{tag}_us"] = round(graph, 2)
     res["graph_pdl_TFLOPS"] = round(flop / res["graph_pdl_us"] / 1e6, 1)
-    res["layers"] = "awq_w4a16 1x3072->18432, qkv 3072->9216, attn_out 3072->3072, GELU MLP 3072->12288->3072"
+    res["layers"] = ("awq_w4a16 1x3072->18432, qkv+RMSNorm+RoPE 3072->9216, attn_out 3072->3072, "
+                     "GELU MLP 3072->12288->3072")
     return res
 
 

@@ -330,7 +330,8 @@ def svdq_w4a4_mlp_gelu(x, w_up, up_act_scale, w_down, down_act_scale, up_bias=No
 def svdq_w4a4_gemm_qkv_norm_rope(act_codes, act_scales, lora_act, w, alpha, heads, gamma_q, gamma_k, rope_cos,
                                  rope_sin, bias=None, y=None, dev_status=None, stream=None, head_dim=128):
     """The fused QKV projection's GEMM with RMSNorm (Q, K heads) and RoPE in
-    its epilogue; w: device dict of the [3 * heads * head_dim, K] layer."""
+    its epilogue; w: device dict of the [3 * heads * head_dim, K] layer;
+    rope_cos / rope_sin: fp32 [head_dim / 2, M] (pair-major)."""
     M = act_codes.shape[0]
     N, K, rank = w["N"], w["K"], w["rank"]
     if y is None:

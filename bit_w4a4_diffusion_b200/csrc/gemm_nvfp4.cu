@@ -104,7 +104,7 @@ struct SmemCtl {
 constexpr int GQ_TABLE_BYTES = BN * 4 + BN * 2;
 template <int kEpi>
 constexpr size_t smem_bytes() {
-  return 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + (kEpi == EPI_GELU ? GQ_TABLE_BYTES : 0) +
+  return 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + (kEpi != EPI_PLAIN ? GQ_TABLE_BYTES : 0) +
          sizeof(SmemCtl);
 }
 static_assert(smem_bytes<EPI_GELU>() <= 232448, "shared memory per block");
@@ -181,14 +181,6 @@ SVDQ_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// A read-only global load kept in program order with the other volatile
-// asm (so that the compiler does not hoist a whole head's worth of them).
-SVDQ_DEV float4 ldg_f4_ordered(const float* addr) {
-  float4 v;
-  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(addr));
-  return v;
-}
-
 SVDQ_DEV void red_add_f32x2(float* addr, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
 }
@@ -203,6 +195,13 @@ SVDQ_DEV size_t tiled_scale_offset(int row, int group, int K) {
 // both the row-per-lane stores and the fragment loads are conflict-free).
 SVDQ_DEV uint32_t hseg16(uint32_t base, int r, int s) {
   return base + (uint32_t)r * 32u + (uint32_t)((s ^ ((r >> 2) & 1)) << 4);
+}
+
+SVDQ_DEV uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
 }
 
 SVDQ_DEV uint2 ld_shared_v2(uint32_t addr) {
@@ -221,7 +220,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
   constexpr bool kGelu = kEpi == EPI_GELU, kQkv = kEpi == EPI_QKV, kWide = kEpi != EPI_PLAIN;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kGelu ? GQ_TABLE_BYTES : 0));
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kWide ? GQ_TABLE_BYTES : 0));
 
   using R = Roles<kWide>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -654,10 +653,20 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
       // the other accumulator is read in full first.  Per lane: v = alpha D + b
       // on packed fp32x2; for Q and K heads the mean of v^2 over the head,
       // v * rsqrt(mean + eps) * gamma, and the rotation of each pair (2i, 2i+1)
-      // by the row's cos / sin; bf16 stores straight to y.
+      // by the row's angle; bf16 out through a 1 KB shared slab per warp (32
+      // rows x 16 columns), written back as whole 32-byte row segments.  The
+      // gamma vectors (for the whole kernel) and the tile's bias columns sit in
+      // shared memory; the rotary tables are pair-major ([64][M]), so that the
+      // 32 rows of a warp read one line per pair.
+      constexpr int NT = R::EPI_WARPS * 32;
       const int q = warp & 3, hf = warp >> 2;
+      const int et = threadIdx.x;  // 0..255 over the epilogue warps
       const QkvParams& qp = p.qk;
       const float2 alpha2 = make_float2(p.alpha, p.alpha);
+      float* tab_g = reinterpret_cast<float*>(epi_base + EPI_BYTES);                  // gamma_q | gamma_k
+      uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + 1024);  // 256 bf16
+      const uint32_t slab = smem_u32(epi_base + warp * 1024);
+      tab_g[et] = et < 128 ? __ldg(qp.gamma_q + et) : __ldg(qp.gamma_k + et - 128);
       uint32_t acc_phase = 0;
       int it = 0;
       for (int tile = t_begin; tile < t_end; tile += t_step, ++it) {
@@ -668,8 +677,13 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
         const bool row_ok = row < p.M;
         const int n = n0 + 128 * hf;  // first column of this warp's head
         const bool head_ok = n < p.N;
+        const uint16_t my_bias = (p.bias != nullptr && n0 + et < p.N) ? __ldg(p.bias + n0 + et) : (uint16_t)0;
         const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
-        if (named_bar_any(2, R::EPI_WARPS * 32, !got)) break;
+        // All epilogue threads decide together; this barrier also ends every
+        // read of the previous tile's bias columns.
+        if (named_bar_any(2, NT, !got)) break;
+        tab_bias[et] = my_bias;
+        asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory");
         tc_fence_after();
         const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE + 128 * hf);
         uint32_t r[4][32];
@@ -690,9 +704,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
         for (int c4 = 0; c4 < 4; ++c4) {
 #pragma unroll
           for (int k8 = 0; k8 < 4; ++k8) {
-            const uint4 bw = p.bias != nullptr
-                                 ? __ldg(reinterpret_cast<const uint4*>(p.bias + n + 32 * c4 + 8 * k8))
-                                 : make_uint4(0, 0, 0, 0);
+            const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + 128 * hf + 32 * c4 + 8 * k8);
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -716,50 +728,58 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           const float ms = __fmul_rn(__fadd_rn(ss.x, ss.y), 1.0f / 128.0f);
           const float rn = __frsqrt_rn(__fadd_rn(ms, qp.eps));
           const float2 rn2 = make_float2(rn, rn);
-          const float* gamma = part == 0 ? qp.gamma_q : qp.gamma_k;
-          const float* cs = qp.rope_cos + (size_t)(row_ok ? row : 0) * 64;
-          const float* sn = qp.rope_sin + (size_t)(row_ok ? row : 0) * 64;
+          const float* gamma = tab_g + 128 * part;
+          const float* cs = qp.rope_cos + (row_ok ? row : 0);
+          const float* sn = qp.rope_sin + (row_ok ? row : 0);
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-              // features 32 c4 + 8 k4 .. +7: pairs 16 c4 + 4 k4 .. +3
-              const float4 g0 = ldg_f4_ordered(gamma + 32 * c4 + 8 * k4);
-              const float4 g1 = ldg_f4_ordered(gamma + 32 * c4 + 8 * k4 + 4);
-              const float4 co = ldg_f4_ordered(cs + 16 * c4 + 4 * k4);
-              const float4 si = ldg_f4_ordered(sn + 16 * c4 + 4 * k4);
+              // features 32 c4 + 8 k4 .. +7: pairs i = 16 c4 + 4 k4 .. +3
+              const float4 g0 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4);
+              const float4 g1 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4 + 4);
               const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-              const float cc[4] = {co.x, co.y, co.z, co.w}, ssn[4] = {si.x, si.y, si.z, si.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
+                const size_t i = (size_t)(16 * c4 + 4 * k4 + j);
+                const float cc = __ldg(cs + i * p.M), sv = __ldg(sn + i * p.M);
                 const int e = 8 * k4 + 2 * j;
                 const float2 u = __fmul2_rn(
                     __fmul2_rn(make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])), rn2),
                     make_float2(gg[2 * j], gg[2 * j + 1]));
                 // (a, b) -> (a cos - b sin, a sin + b cos)
-                const float x0 = __fmaf_rn(u.x, cc[j], -__fmul_rn(u.y, ssn[j]));
-                const float x1 = __fmaf_rn(u.x, ssn[j], __fmul_rn(u.y, cc[j]));
-                r[c4][e] = __float_as_uint(x0);
-                r[c4][e + 1] = __float_as_uint(x1);
+                r[c4][e] = __float_as_uint(__fmaf_rn(u.x, cc, -__fmul_rn(u.y, sv)));
+                r[c4][e + 1] = __float_as_uint(__fmaf_rn(u.x, sv, __fmul_rn(u.y, cc)));
               }
             }
           }
         }
-        if (row_ok) {
-          uint16_t* yrow = qp.y + (size_t)row * p.N + n;
+        // 16 columns at a time: each lane writes its row's 32 bytes into the
+        // slab (16-byte halves XOR-ed with (row / 4) mod 2: conflict-free), then
+        // lane l stores halves l and l + 32, i.e. rows l / 2 and 16 + l / 2.
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t w[8];
 #pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) {
-              uint32_t w[4];
+          for (int j = 0; j < 8; ++j) {
+            const int e = 16 * (c16 & 1) + 2 * j;
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[c16 >> 1][e]), __uint_as_float(r[c16 >> 1][e + 1]));
+            w[j] = *reinterpret_cast<uint32_t*>(&h2);
+          }
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[c4][8 * k8 + 2 * j]),
-                                                          __uint_as_float(r[c4][8 * k8 + 2 * j + 1]));
-                w[j] = *reinterpret_cast<uint32_t*>(&h2);
-              }
-              *reinterpret_cast<uint4*>(yrow + 32 * c4 + 8 * k8) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+          for (int h = 0; h < 2; ++h)
+            st_shared_v4(slab + lane * 32 + ((h ^ ((lane >> 2) & 1)) << 4),
+                         make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int pc = lane + 32 * k, rr = pc >> 1, h = pc & 1;
+            const uint4 v = ld_shared_v4(slab + rr * 32 + ((h ^ ((rr >> 2) & 1)) << 4));
+            const int grow = m0 + 32 * q + rr;
+            if (grow < p.M)
+              *reinterpret_cast<uint4*>(qp.y + (size_t)grow * p.N + n + 16 * c16 + 8 * h) = v;
+          }
+          __syncwarp();  // the slab's reads precede the next writes
         }
       }
     } else {

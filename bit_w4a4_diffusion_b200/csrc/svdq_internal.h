@@ -64,8 +64,8 @@ struct GeluQuantParams {
 struct QkvParams {
   const float* gamma_q;   // fp32 [128]
   const float* gamma_k;   // fp32 [128]
-  const float* rope_cos;  // fp32 [M, 64]
-  const float* rope_sin;  // fp32 [M, 64]
+  const float* rope_cos;  // fp32 [64, M] (pair-major)
+  const float* rope_sin;  // fp32 [64, M]
   float eps;
   int hd;                 // columns per part: heads * 128
   uint16_t* y;            // bf16 [M, N]

@@ -264,7 +264,9 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
  *                  gamma_k for K, fp32 [128]), then each feature pair
  *                  (u[2i], u[2i+1]) is rotated by the row's angle i:
  *                  (a, b) -> (a cos - b sin, a sin + b cos) with
- *                  cos = rope_cos[m][i], sin = rope_sin[m][i] (fp32 [M, 64]);
+ *                  cos = rope_cos[i * M + m], sin = rope_sin[i * M + m]
+ *                  (fp32 [64, M], pair-major: the tables of all tokens for
+ *                  pair 0, then pair 1, ...);
  *   V heads:       unchanged;
  * then rounded to bf16 into y [M, N].  N = 3 * heads * 128, K % 256 == 0.
  *

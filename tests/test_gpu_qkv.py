@@ -25,7 +25,9 @@ def _setup(M, K, heads):
     inp = wl.make_svdq_inputs(c)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     gq, gk, cos, sin = wl.make_rope_norm_inputs(M, heads)
-    dev = {k: torch.from_numpy(v).cuda() for k, v in (("gq", gq), ("gk", gk), ("cos", cos), ("sin", sin))}
+    # the library takes the rotary tables pair-major: [64, M]
+    dev = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda()
+           for k, v in (("gq", gq), ("gk", gk), ("cos", cos.T), ("sin", sin.T))}
     return inp, pk, B.to_device(pk), (gq, gk, cos, sin), dev
 
 
