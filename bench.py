@@ -424,8 +424,8 @@ def measure_rows(B, wl, dev, peaks):
 def measure_qkv(B, wl, dev, heads=24):
     """The DiT QKV projection (4096 tokens, 3072 -> 9216) with RMSNorm and
     RoPE on its Q and K heads: fused in the GEMM's epilogue, against the
-    layer followed by the same normalization and rotation as separate torch
-    operations (for comparison only).  Two rotating weight sets."""
+    layer followed by the same normalization and rotation as separate bf16
+    torch operations (for comparison only).  Two rotating weight sets."""
     import torch
     c = wl.SVDQ_CASES["qkv"]
     M, K, N = c.M, c.K, c.N
@@ -444,17 +444,19 @@ def measure_qkv(B, wl, dev, heads=24):
     wsp = torch.empty(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
     hd = heads * 128
 
+    gq16, gk16 = gq.to(torch.bfloat16), gk.to(torch.bfloat16)
+    c16 = cos.t().reshape(M, 1, 64).to(torch.bfloat16)
+    s16 = sin.t().reshape(M, 1, 64).to(torch.bfloat16)
+
     def torch_norm_rope(t, g):
-        t32 = t.float().view(M, heads, 128)
-        t32 = t32 * torch.rsqrt(t32.pow(2).mean(-1, keepdim=True) + 1e-6) * g
-        a, b = t32[..., 0::2], t32[..., 1::2]
-        c_, s_ = cos.t().reshape(M, 1, 64), sin.t().reshape(M, 1, 64)
-        return torch.stack((a * c_ - b * s_, a * s_ + b * c_), dim=-1).view(M, hd).to(torch.bfloat16)
+        n = torch.nn.functional.rms_norm(t.view(M, heads, 128), (128,), g, eps=1e-6)
+        a, b = n[..., 0::2], n[..., 1::2]
+        return torch.stack((a * c16 - b * s16, a * s16 + b * c16), dim=-1).view(M, hd)
 
     def unfused(i):
         B.svdq_w4a4_linear("nvfp4", x, ws_[i], s_a, bias=bias, y=y, workspace=wsp)
-        y[:, :hd] = torch_norm_rope(y[:, :hd], gq)
-        y[:, hd:2 * hd] = torch_norm_rope(y[:, hd:2 * hd], gk)
+        y[:, :hd] = torch_norm_rope(y[:, :hd], gq16)
+        y[:, hd:2 * hd] = torch_norm_rope(y[:, hd:2 * hd], gk16)
 
     fused = [lambda i=i: B.svdq_w4a4_qkv_norm_rope_linear(x, ws_[i], s_a, heads, gq, gk, cos, sin, bias=bias, y=y,
                                                           workspace=wsp) for i in range(nset)]

@@ -1,5 +1,5 @@
 """Failure detection without a GPU fault: every mbarrier wait in the NVFP4,
-INT4 and GELU-MLP GEMM kernels is bounded by the library's wait limit.  With
+INT4, GELU-MLP and QKV GEMM kernels is bounded by the library's wait limit.  With
 the limit set to 1 ns the first wait that is not already satisfied gives up;
 the kernel must report a timeout code through dev_status, drain its own
 copies and MMAs, free its tensor memory and return, leaving the context
@@ -117,3 +117,38 @@ def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
     assert int(status.item()) == 0
     from tests.test_gpu_mlp import _check_hidden
     _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl)
+
+
+def test_qkv_gemm_wait_timeout_reports_and_recovers():
+    """The QKV + RMSNorm + RoPE kernel (eight epilogue warps that stop together)."""
+    import bit_w4a4_diffusion_b200 as B
+    from oracle import qkv as OQ
+    M, K, heads = 384, 512, 2
+    inp = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, K=K, N=3 * heads * 128))
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    gq, gk, cos, sin = wl.make_rope_norm_inputs(M, heads)
+    d = [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in (gq, gk, cos.T, sin.T)]
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    bias = B.bits_to_bf16(inp.bias_bits, "cuda")
+    s_a = float(inp.act_scale)
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", x, w["inv_smooth"], w["lora_down"], s_a, w["weight_scale_f"])
+    alpha = float(np.float32(np.float32(s_a) * np.float32(pk["weight_scale"][0])))
+    torch.cuda.synchronize()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_gemm_qkv_norm_rope(codes, scales, lora, w, alpha, heads, *d, bias=bias, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+    status.zero_()
+    y = B.svdq_w4a4_gemm_qkv_norm_rope(codes, scales, lora, w, alpha, heads, *d, bias=bias, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
+    ref = OQ.qkv_layer_f64(act, ref_pw, inp.L1, inp.L2, inp.bias, gq, gk, cos, sin, heads)
+    assert_output_close(y.float().cpu().numpy(), ref, "QKV GEMM after a timed-out call")
