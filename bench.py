@@ -211,7 +211,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     case = wl.SVDQ_CASES[WORKLOAD]
-    inp = wl.make_svdq_inputs(case)
+    inp = wl.make_svdq_inputs(case, B.svdq_calibrate)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     s_a = float(inp.act_scale)
     M, N, K = case.M, case.N, case.K
@@ -403,7 +403,7 @@ def measure_rows(B, wl, dev, peaks):
     int4 = {}
     for M in (1024, 2048, 4096, 8192):
         c = wl.SVDQ_CASES[f"int4_m{M}"]
-        inp = wl.make_svdq_inputs(c)
+        inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
         pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
         nset = 4
         ws = [B.to_device(pk, dev) for _ in range(nset)]
@@ -429,7 +429,7 @@ def measure_qkv(B, wl, dev, heads=24):
     import torch
     c = wl.SVDQ_CASES["qkv"]
     M, K, N = c.M, c.K, c.N
-    inp = wl.make_svdq_inputs(c)
+    inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     nset = 2
     ws_ = [B.to_device(pk, dev) for _ in range(nset)]
@@ -484,10 +484,10 @@ def block_layers(B, wl, dev, M):
     (out: dict of output tensors)."""
     import dataclasses
     import torch
-    q = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M))
-    o = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, N=3072, name="attn_out"))
-    iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1))
-    idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05))
+    q = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M), B.svdq_calibrate)
+    o = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, N=3072, name="attn_out"), B.svdq_calibrate)
+    iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1), B.svdq_calibrate)
+    idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05), B.svdq_calibrate)
     a = wl.make_awq_inputs(1)
     rq = [torch.from_numpy(np.ascontiguousarray(t.T if t.ndim == 2 else t)).to(dev)
           for t in wl.make_rope_norm_inputs(M, 24)]
@@ -576,8 +576,8 @@ def mlp_inputs(B, wl, dev, nset):
     workload with a bias; down: the mlp_down workload's weights and
     calibration), `nset` device copies of both layers' packed weights."""
     import dataclasses
-    iu = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_up"], bias_std=0.1))
-    idn = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_down"], bias_std=0.05))
+    iu = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_up"], bias_std=0.1), B.svdq_calibrate)
+    idn = wl.make_svdq_inputs(dataclasses.replace(wl.SVDQ_CASES["mlp_down"], bias_std=0.05), B.svdq_calibrate)
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
     wus = [B.to_device(pk_u, dev) for _ in range(nset)]
@@ -682,8 +682,9 @@ def main():
         if rank != 0:
             return
         import workloads as wl
+        from oracle import calibrate as OC
         case = wl.SVDQ_CASES[WORKLOAD]
-        inp = wl.make_svdq_inputs(case)
+        inp = wl.make_svdq_inputs(case, OC.calibrate)
         budget = max(30.0, min(150.0, 1.0 * (args.steps + args.warmup)))
         tf, dt, rows = time_oracle(case, inp, args.steps, args.warmup, budget)
         cores = _cpu_threads()

@@ -47,6 +47,7 @@ def _load():
         "svdq_scales_to_rowmajor": (I, [I, I, P, P]),
         "svdq_scales_from_rowmajor": (I, [I, I, P, P]),
         "svdq_pack_weights": (I, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
+        "svdq_calibrate": (I, [I, I, I, I, I, I, P, P, P, P, P, P, P]),
         "svdq_quantize_act": (I, [I, I, I, I, P, P, P, F, F, P, P, P, P]),
         "svdq_w4a4_gemm": (I, [I, I, I, I, I, P, P, P, P, P, P, P, F, P, P, P]),
         "svdq_w4a4_linear": (I, [I, I, I, I, I, P, P, P, F, P, P, F, P, P, P, P, LL, P, P]),
@@ -169,6 +170,24 @@ def svdq_pack_weights(precision, W_bits, smooth, L1_bits, L2_bits, rank=SVDQ_RAN
         out["lora_down"] = out["lora_down"].view(np.float16)   # fp16 operand for NVFP4
     out["N"], out["K"], out["rank"], out["precision"] = N, K, rank, p
     return out
+
+
+def svdq_calibrate(x_bits, W_bits, omega, rank=SVDQ_RANK, power_iters=4):
+    """Host calibration: x_bits [M, K], W_bits [N, K] (uint16 bf16 patterns),
+    omega [N, rank + p] fp64.  Returns (smooth fp32 [K], L1 bits [K, rank],
+    L2 bits [rank, N], act_scale fp32)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    omega = np.ascontiguousarray(omega, dtype=np.float64)
+    M, K = x_bits.shape
+    N = W_bits.shape[0]
+    smooth = np.empty(K, np.float32)
+    L1 = np.empty((K, rank), np.uint16)
+    L2 = np.empty((rank, N), np.uint16)
+    s_a = np.zeros(1, np.float32)
+    _check(lib.svdq_calibrate(N, K, M, rank, omega.shape[1] - rank, power_iters, _ptr(W_bits), _ptr(x_bits),
+                              _ptr(omega), _ptr(smooth), _ptr(L1), _ptr(L2), _ptr(s_a)))
+    return smooth, L1, L2, np.float32(s_a[0])
 
 
 def awq_pack_weights(W_bits):

@@ -20,11 +20,11 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-fmad=false",
                      "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
-CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-ffp-contract=off", "-pthread", "-I", INCLUDE,
+CXX_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-ffp-contract=off", "-pthread", "-I", INCLUDE,
              "-I", "/usr/local/cuda/include"]
 
 CU_SOURCES = ["abi.cu", "quantize_act.cu", "quantize_nvfp4.cu", "gemm_nvfp4.cu", "gemm_nvfp4_pair.cu", "gemm_int4.cu", "awq_gemm.cu", "noalloc.cu"]
-CXX_SOURCES = ["pack.cpp"]
+CXX_SOURCES = ["pack.cpp", "calib.cpp"]
 
 
 def _headers():

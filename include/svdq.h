@@ -118,6 +118,30 @@ int svdq_pack_weights(int precision, int N, int K, int rank, const uint16_t* W, 
                       const uint16_t* L1, const uint16_t* L2, uint8_t* codes, uint8_t* scales, float* weight_scale,
                       float* inv_smooth, uint16_t* lora_down, uint16_t* lora_up);
 
+/* ------------------------------------------------------------------ host calibration
+ * svdq_calibrate: the offline step that produces a layer's smoothing
+ * factors, low-rank factors and static activation scale from its weights
+ * and a calibration batch ("SVDQuant and the Nunchaku engine": outliers
+ * migrate into the weights; a 16-bit low-rank branch from a decomposition
+ * of the weights absorbs their hardest part).  Host only, untimed:
+ *   smooth[k] = sqrt(max_i |x[i,k]| / max_n |W[n,k]|) in fp32, 1 where a max is 0;
+ *   A = (W diag(smooth))^T [K, N] in fp64;
+ *   randomized subspace iteration (Halko, Martinsson & Tropp 2011, Alg. 4.4)
+ *   with the caller's Gaussian test matrix omega [N, rank + oversample]
+ *   (fp64, row-major) and power_iters iterations: Q = qr(A omega); repeat:
+ *   Z = qr(A^T Q), Q = qr(A Z); B = Q^T A = Ub S Vt; U = Q Ub; each column of
+ *   U negated if its largest-magnitude entry (the first on a tie) is
+ *   negative, with the matching row of Vt;
+ *   L1 = bf16(U[:, :rank] S[:rank]) [K, rank], L2 = bf16(Vt[:rank]) [rank, N];
+ *   act_scale = max |x[i,k] * fp32(1/smooth[k])| / 2688 (fp32; 1 if 0).
+ * Inputs (host): W bf16 [N, K], x bf16 [M, K] (the calibration batch),
+ * omega.  Outputs (host, caller-allocated): smooth fp32 [K], L1 and L2 bf16,
+ * act_scale (1 float).  The result does not depend on the number of host
+ * threads used.  rank + oversample <= min(K, N). */
+int svdq_calibrate(int N, int K, int M, int rank, int oversample, int power_iters, const uint16_t* W,
+                   const uint16_t* x, const double* omega, float* smooth, uint16_t* L1, uint16_t* L2,
+                   float* act_scale);
+
 /* ------------------------------------------------------------------ device
  * svdq_quantize_act: smoothing + activation quantization + low-rank
  * down-projection in one pass over x (the Nunchaku engine's fused

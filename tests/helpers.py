@@ -77,3 +77,11 @@ def check_nvfp4_near_boundary(v_ref, s, codes, scales, delta):
     assert np.all(ok), f"{np.sum(~ok)} codes are off by more than the value error"
     ref_codes, _ = O.nvfp4_quantize(v_ref.astype(np.float32), s32)
     return float(np.mean(ref_codes != np.asarray(codes)))
+
+
+def svdq_inputs(case):
+    """The seeded inputs of `case`, calibrated by the oracle (smoothing,
+    rank-r factors, activation scale)."""
+    import workloads as wl
+    from oracle import calibrate as OC
+    return wl.make_svdq_inputs(case, OC.calibrate)

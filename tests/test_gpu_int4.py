@@ -7,7 +7,7 @@ import torch
 
 import workloads as wl
 from oracle import svdq as O
-from tests.helpers import assert_output_close, nibbles
+from tests.helpers import assert_output_close, nibbles, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ def test_int4_linear_matches_oracle(name, kw):
     c = wl.SVDQ_CASES[name]
     if kw:
         c = wl.scaled_case(c, **kw)
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     x = B.bits_to_bf16(inp.x_bits, "cuda")

@@ -17,7 +17,7 @@ import torch
 import workloads as wl
 from oracle import mlp as OM
 from oracle import svdq as O
-from tests.helpers import check_nvfp4_near_boundary, nibbles, output_errors
+from tests.helpers import check_nvfp4_near_boundary, nibbles, output_errors, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -66,8 +66,8 @@ def _mlp_case(M, K, N, seed_shift=0):
 
 def _setup(up_case, down_case):
     B = _lib()
-    iu = wl.make_svdq_inputs(up_case)
-    idn = wl.make_svdq_inputs(down_case)
+    iu = svdq_inputs(up_case)
+    idn = svdq_inputs(down_case)
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
     return iu, idn, pk_u, pk_d, B.to_device(pk_u), B.to_device(pk_d)
@@ -176,7 +176,7 @@ def test_fused_codes_are_deterministic():
 def test_fused_rejects_bad_shapes_before_launch():
     B = _lib()
     up_case, down_case = _mlp_case(64, 256, 384)        # N = 384 is not a multiple of 256
-    iu = wl.make_svdq_inputs(up_case)
+    iu = svdq_inputs(up_case)
     pk = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     wu = B.to_device(pk)
     fake_next = dict(wu, K=384)

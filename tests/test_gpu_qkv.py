@@ -9,7 +9,7 @@ import torch
 import workloads as wl
 from oracle import qkv as OQ
 from oracle import svdq as O
-from tests.helpers import assert_output_close
+from tests.helpers import assert_output_close, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -22,7 +22,7 @@ def _lib():
 def _setup(M, K, heads):
     B = _lib()
     c = wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, K=K, N=3 * heads * 128)
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     gq, gk, cos, sin = wl.make_rope_norm_inputs(M, heads)
     # the library takes the rotary tables pair-major: [64, M]

@@ -12,7 +12,7 @@ import torch
 
 import workloads as wl
 from oracle import svdq as O
-from tests.helpers import assert_output_close, nibbles
+from tests.helpers import assert_output_close, nibbles, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -65,7 +65,7 @@ def _check_s1(inp, codes, scales, lora, pk, rows=None):
 
 def _layer(c):
     B = _lib()
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     bias = B.bits_to_bf16(inp.bias_bits, "cuda") if inp.bias_bits is not None else None

@@ -10,7 +10,7 @@ import torch
 
 import workloads as wl
 from oracle import svdq as O
-from tests.helpers import assert_output_close
+from tests.helpers import assert_output_close, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -22,7 +22,7 @@ def test_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     import bit_w4a4_diffusion_b200 as B
     monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     c = wl.scaled_case(wl.SVDQ_CASES["qkv"], M=640, N=2048)   # several tiles per CTA
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     bias = B.bits_to_bf16(inp.bias_bits, "cuda") if inp.bias_bits is not None else None
@@ -55,7 +55,7 @@ def test_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
 def test_int4_gemm_wait_timeout_reports_and_recovers():
     import bit_w4a4_diffusion_b200 as B
     c = wl.scaled_case(wl.SVDQ_CASES["int4_m1024"], M=1024)
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     x = B.bits_to_bf16(inp.x_bits, "cuda")
@@ -88,7 +88,7 @@ def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
     import bit_w4a4_diffusion_b200 as B
     up = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=640, K=768, N=1024), bias_std=0.1)
     dn = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=640, K=1024, N=768), bias_std=0.05)
-    iu, idn = wl.make_svdq_inputs(up), wl.make_svdq_inputs(dn)
+    iu, idn = svdq_inputs(up), svdq_inputs(dn)
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
     wu, wd = B.to_device(pk_u), B.to_device(pk_d)
@@ -124,7 +124,7 @@ def test_qkv_gemm_wait_timeout_reports_and_recovers():
     import bit_w4a4_diffusion_b200 as B
     from oracle import qkv as OQ
     M, K, heads = 384, 512, 2
-    inp = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, K=K, N=3 * heads * 128))
+    inp = svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, K=K, N=3 * heads * 128))
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     gq, gk, cos, sin = wl.make_rope_norm_inputs(M, heads)

@@ -10,6 +10,7 @@ import pytest
 
 import bit_w4a4_diffusion_b200 as B
 import workloads as wl
+from tests.helpers import svdq_inputs
 from oracle import awq as OA
 from oracle import svdq as O
 
@@ -33,7 +34,7 @@ def test_pack_weights_matches_oracle(name, kw):
     c = wl.SVDQ_CASES[name]
     if kw:
         c = wl.scaled_case(c, **kw)
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights(c.precision, inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     ref = O.pack_weights(c.precision, inp.W, inp.lam, inp.L1, inp.L2)
     assert np.array_equal(pk["inv_smooth"], ref["inv_lam"])

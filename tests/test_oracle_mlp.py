@@ -14,6 +14,7 @@ from scipy.optimize import brentq
 from scipy.stats import norm
 
 import workloads as wl
+from oracle.calibrate import smoothing_factors
 from oracle import formats as F
 from oracle import mlp as OM
 from oracle import svdq as O
@@ -109,7 +110,7 @@ def test_mlp_matches_brute_force_loops():
     _, L1u = wl.to_bf16(rng.standard_normal((K, r)).astype(np.float32) * 0.1)
     _, L2u = wl.to_bf16(rng.standard_normal((r, N)).astype(np.float32) * 0.1)
     bu = wl.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.3)[1]
-    lam_u = wl.smoothing_factors(x, Wu)
+    lam_u = smoothing_factors(x, Wu)
     _, Wd = wl.to_bf16(rng.standard_normal((Nd, N)).astype(np.float32) * 0.1)
     _, L1d = wl.to_bf16(rng.standard_normal((N, r)).astype(np.float32) * 0.1)
     _, L2d = wl.to_bf16(rng.standard_normal((r, Nd)).astype(np.float32) * 0.1)

@@ -12,6 +12,7 @@ import math
 import numpy as np
 
 import workloads as wl
+from oracle.calibrate import smoothing_factors
 from oracle import qkv as OQ
 from oracle import svdq as O
 
@@ -72,7 +73,7 @@ def test_qkv_layer_matches_brute_force_loops():
     _, L1 = wl.to_bf16(rng.standard_normal((K, r)).astype(np.float32) * 0.1)
     _, L2 = wl.to_bf16(rng.standard_normal((r, N)).astype(np.float32) * 0.1)
     b = wl.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.1)[1]
-    lam = wl.smoothing_factors(x, W)
+    lam = smoothing_factors(x, W)
     gq, gk = rng.uniform(0.5, 1.5, d), rng.uniform(0.5, 1.5, d)
     phi = rng.uniform(-3, 3, (M, d // 2))
     pw = O.pack_weights("nvfp4", W, lam, L1, L2)

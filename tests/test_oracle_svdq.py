@@ -10,6 +10,8 @@ import numpy as np
 import pytest
 
 import workloads as wl
+from oracle.calibrate import smoothing_factors
+from tests.helpers import svdq_inputs
 from oracle import formats as F
 from oracle import svdq as O
 
@@ -183,7 +185,7 @@ def test_int4_error_bound_and_no_minus_eight():
 def _tiny_case(rng, M, K, N, r, bias=True):
     _, x = wl.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
     _, W = wl.to_bf16(rng.standard_normal((N, K)).astype(np.float32) * 0.05)
-    lam = wl.smoothing_factors(x, W)
+    lam = smoothing_factors(x, W)
     _, L1 = wl.to_bf16(rng.standard_normal((K, r)).astype(np.float32) * 0.1)
     _, L2 = wl.to_bf16(rng.standard_normal((r, N)).astype(np.float32) * 0.1)
     b = wl.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.1)[1] if bias else None
@@ -278,7 +280,7 @@ def test_quantized_layer_approximates_full_precision():
     """End-to-end sanity on the tiny workload: the W4A4 + low-rank output is a
     few percent from the unquantized x W^T (the method's purpose), and the
     low-rank branch carries most of the output."""
-    inp = wl.make_svdq_inputs(wl.SVDQ_CASES["tiny"])
+    inp = svdq_inputs(wl.SVDQ_CASES["tiny"])
     y, y64, act, pw = O.svdq_linear("nvfp4", inp.x, inp.W, inp.lam, inp.L1, inp.L2, inp.bias)
     ref = inp.x.astype(np.float64) @ inp.W.astype(np.float64).T
     rel = np.linalg.norm(y64 - ref) / np.linalg.norm(ref)

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import workloads as wl
-from tests.helpers import assert_output_close
+from tests.helpers import assert_output_close, svdq_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 def _layer(name, **kw):
     import bit_w4a4_diffusion_b200 as B
     c = wl.scaled_case(wl.SVDQ_CASES[name], **kw)
-    inp = wl.make_svdq_inputs(c)
+    inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
     x = B.bits_to_bf16(inp.x_bits, "cuda")

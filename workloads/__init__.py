@@ -1,18 +1,14 @@
 """Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
 
-This module holds no step of the layer itself (no smoothing application, no
-residual, no quantization, no GEMM): it draws random tensors and runs the
-offline calibration recipe that produces the layer's *inputs*:
-
-* lambda_j = sqrt(max_i |x_ij| / max_n |W_nj|) (1 where either max is 0), the
-  SmoothQuant-style migration strength 0.5;
-* a rank-r factorisation L1 [K, r], L2 [r, N] of (W diag(lambda))^T, taken
-  from a seeded randomized subspace iteration in fp64 (Halko, Martinsson &
-  Tropp 2011, Alg. 4.4) with all of Sigma put on L1, both rounded to bf16;
-* the static NVFP4 activation tensor scale s_a = amax|x_ij / lambda_j| / 2688
-  over the calibration batch (the batch itself), in fp32;
-* for the AWQ layer, the per-input-channel scale s_j = mean_i(|x_ij|)^0.5
-  folded as W diag(s) and x / s, both rounded to bf16.
+This module holds no step of the method: it draws random tensors (x, W,
+bias, the Gaussian test matrix of the low-rank calibration, rotary tables)
+and hands x and W to a caller-supplied calibration function that returns the
+layer's remaining inputs (smoothing factors, the rank-r factors and the
+static activation scale): the tests pass the oracle's, the benchmark the
+library's own ``svdq_calibrate``.  For the AWQ layer it folds the
+per-input-channel scale s_j = mean_i(|x_ij|)^0.5 into W diag(s) and x / s
+(both rounded to bf16), which shapes the inputs without entering the
+layer's arithmetic.
 
 The pages' own workloads (ERNIE-Image-Turbo and Flux Schnell weights and
 prompts) are not available; these shapes and distributions stand in for
@@ -62,40 +58,13 @@ def gaussian_weight(rng, N, K, std, n_outlier_entries=0, factor=1.0):
     return W
 
 
-def smoothing_factors(x, W):
-    """lambda_j = sqrt(max_i|x_ij| / max_n|W_nj|) in fp32; 1 where a max is 0."""
-    ax = np.max(np.abs(x), axis=0).astype(np.float32)
-    aw = np.max(np.abs(W), axis=0).astype(np.float32)
-    ok = (ax > 0) & (aw > 0)
-    lam = np.ones_like(ax)
-    lam[ok] = np.sqrt(ax[ok] / aw[ok]).astype(np.float32)
-    return lam.astype(np.float32)
+OVERSAMPLE = 8       # columns of the calibration test matrix beyond the rank
 
 
-def lowrank_factors(A, r, seed, oversample=8, power_iters=4):
-    """Rank-r factors of A [K, N] (fp64) by seeded randomized subspace iteration.
-
-    Returns L1 = U_r Sigma_r [K, r] and L2 = V_r^T [r, N] in fp64.  Column
-    signs are fixed so that the largest-magnitude entry of each column of U is
-    positive.
-    """
-    K, N = A.shape
-    g = _rng(seed)
-    Om = g.standard_normal((N, r + oversample))
-    Q, _ = np.linalg.qr(A @ Om)
-    for _ in range(power_iters):
-        Z, _ = np.linalg.qr(A.T @ Q)
-        Q, _ = np.linalg.qr(A @ Z)
-    B = Q.T @ A                                        # [(r+p), N]
-    Ub, S, Vt = np.linalg.svd(B, full_matrices=False)
-    U = Q @ Ub[:, :r]
-    S = S[:r]
-    Vt = Vt[:r]
-    sign = np.sign(U[np.argmax(np.abs(U), axis=0), np.arange(r)])
-    sign[sign == 0] = 1.0
-    U *= sign[None, :]
-    Vt *= sign[:, None]
-    return U * S[None, :], Vt
+def calibration_test_matrix(case):
+    """The Gaussian test matrix [N, rank + OVERSAMPLE] (fp64) of the case's
+    low-rank calibration, from its own seeded stream."""
+    return _rng([*np.atleast_1d(_seed(case.seed)), 7]).standard_normal((case.N, case.rank + OVERSAMPLE))
 
 
 # --------------------------------------------------------------- cases ------
@@ -144,8 +113,9 @@ def _seed(seed):
     return list(seed) if isinstance(seed, (tuple, list)) else seed
 
 
-def make_svdq_inputs(case: SvdqCase) -> SvdqInputs:
-    """Draw x, W, bias for ``case`` and run the calibration recipe."""
+def make_svdq_inputs(case: SvdqCase, calibrate) -> SvdqInputs:
+    """Draw x, W, bias for ``case``; ``calibrate(x_bits, W_bits, omega, rank)``
+    returns (lambda fp32 [K], L1 bf16 bits [K, r], L2 bf16 bits [r, N], s_a)."""
     rng = _rng(_seed(case.seed))
     x = outlier_activations(rng, case.M, case.K, case.n_outlier_ch, case.outlier_factor, case.gelu)
     W = gaussian_weight(rng, case.N, case.K, case.w_std, case.w_outlier_entries, case.w_outlier_factor)
@@ -154,24 +124,17 @@ def make_svdq_inputs(case: SvdqCase) -> SvdqInputs:
         bias = rng.standard_normal(case.N, dtype=np.float32) * np.float32(case.bias_std)
     x_bits, x_v = to_bf16(x)
     W_bits, W_v = to_bf16(W)
-    lam = smoothing_factors(x_v, W_v)
-    W_hat_T = (W_v.astype(np.float64) * lam.astype(np.float64)[None, :]).T     # [K, N]
-    L1, L2 = lowrank_factors(W_hat_T, case.rank, seed=[*np.atleast_1d(_seed(case.seed)), 7])
-    L1_bits, L1_v = to_bf16(L1.astype(np.float32))
-    L2_bits, L2_v = to_bf16(L2.astype(np.float32))
+    lam, L1_bits, L2_bits, s_a = calibrate(x_bits, W_bits, calibration_test_matrix(case), case.rank)
+    lam = np.asarray(lam, dtype=np.float32)
+    L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    L1_v = (L1_bits.astype(np.uint32) << 16).view(np.float32)
+    L2_v = (L2_bits.astype(np.uint32) << 16).view(np.float32)
     b_bits = b_v = None
     if bias is not None:
         b_bits, b_v = to_bf16(bias)
     return SvdqInputs(case, x_bits, x_v, W_bits, W_v, lam, L1_bits, L1_v, L2_bits, L2_v, b_bits, b_v,
-                      calibrated_act_scale(x_v, lam))
-
-
-def calibrated_act_scale(x, lam):
-    """Static activation tensor scale from a calibration batch: amax over
-    x_ij * (1/lambda_j) (fp32 reciprocal, fp32 product), divided by 6 * 448."""
-    inv = (np.float32(1.0) / lam.astype(np.float32)).astype(np.float32)
-    amax = np.float32(np.max(np.abs((x.astype(np.float32) * inv[None, :]).astype(np.float32))))
-    return np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
+                      np.float32(s_a))
 
 
 # The five workloads (diffusion-transformer shapes).  "1% of channels" is
