@@ -606,6 +606,55 @@ def run_mlp_calls(calls):
     print(json.dumps({"mlp_calls": calls, "workload": f"x [{M},{K}] -> {N} -> {K}"}), flush=True)
 
 
+def run_profile_calls(row, calls):
+    """`calls` back-to-back calls of one row's entry point at its workload
+    size, untimed (the commands the per-row profiles are taken with):
+    awq (M = 1, N = 18432, K = 3072, six rotating weight sets), int4 (the
+    INT4 layer at M = 4096, K = N = 3072, four sets), qkv (the fused QKV
+    projection with RMSNorm and RoPE, two sets), mlp (the fused DiT MLP)."""
+    import torch
+    import bit_w4a4_diffusion_b200 as B
+    import workloads as wl
+    if row == "mlp":
+        return run_mlp_calls(calls)
+    dev = torch.device("cuda:0")
+    if row == "awq":
+        a = wl.make_awq_inputs(1)
+        pk = B.awq_pack_weights(a.W_bits)
+        ws = [B.to_device(pk, dev) for _ in range(6)]
+        x = B.bits_to_bf16(a.x_bits, dev)
+        y = torch.empty((1, a.N), dtype=torch.bfloat16, device=dev)
+        fns = [lambda i=i: B.awq_w4a16_linear(x, ws[i], y=y) for i in range(6)]
+    elif row == "int4":
+        c = wl.SVDQ_CASES["int4_m4096"]
+        inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
+        pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+        ws = [B.to_device(pk, dev) for _ in range(4)]
+        x = B.bits_to_bf16(inp.x_bits, dev)
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(B.workspace_bytes("int4", c.M, c.K), dtype=torch.uint8, device=dev)
+        fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=y, workspace=wsp) for i in range(4)]
+    elif row == "qkv":
+        c = wl.SVDQ_CASES["qkv"]
+        inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
+        pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+        ws = [B.to_device(pk, dev) for _ in range(2)]
+        gq, gk, cm, sm = wl.make_rope_norm_inputs(c.M, 24)
+        t = [torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (gq, gk, cm.T, sm.T)]
+        x = B.bits_to_bf16(inp.x_bits, dev)
+        bias = B.bits_to_bf16(inp.bias_bits, dev)
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device=dev)
+        fns = [lambda i=i: B.svdq_w4a4_qkv_norm_rope_linear(x, ws[i], float(inp.act_scale), 24, *t, bias=bias, y=y,
+                                                            workspace=wsp) for i in range(2)]
+    else:
+        raise SystemExit(f"unknown row {row!r}")
+    for i in range(calls):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_row": row, "calls": calls}), flush=True)
+
+
 def measure_mlp(B, wl, dev):
     """The DiT MLP block, fused (the GELU and the down layer's activation
     quantizer in the up GEMM's epilogue) and unfused (up layer -> bf16 y ->
@@ -667,11 +716,17 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ / MLP row measurements")
     ap.add_argument("--mlp-calls", type=int, default=0,
                     help="only run this many fused DiT MLP calls (untimed; for profiling) and exit")
+    ap.add_argument("--profile", choices=["awq", "int4", "qkv", "mlp"], default=None,
+                    help="only run --calls calls of one row's entry point (untimed; for profiling) and exit")
+    ap.add_argument("--calls", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.mlp_calls > 0:
         run_mlp_calls(args.mlp_calls)
+        return
+    if args.profile is not None:
+        run_profile_calls(args.profile, args.calls)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
