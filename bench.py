@@ -71,6 +71,34 @@ def _gemm_traffic():
     return GEMM_TRAFFIC["bytes"]
 
 
+# ------------------------------------------------------------------ ranks
+# One process per GPU, each a replica on its own batch (tokens are
+# independent rows; no data-path collective).  The only cross-rank steps are
+# the barriers around the timed region and the max over ranks of its
+# duration; `value` counts the tokens of all ranks.
+
+def rank_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_max(v, world, device=None):
+    """max over ranks of a per-rank duration (every rank gets it)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step, steps, world, max_ms):
+    """TFLOP/s of the whole job: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def _cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -240,15 +268,10 @@ def run_gpu(args, rank, world, local_rank):
                            stream=st if st is not None else torch.cuda.current_stream(dev))
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(v, world, dev)
 
     # ---- timed region: K steps of the whole layer, replayed from a CUDA graph
     # of G consecutive steps (rotating the sets) so host launch cost is off the
@@ -281,7 +304,7 @@ def run_gpu(args, rank, world, local_rank):
     barrier()
     t_ms = max_over_ranks(e0.elapsed_time(e1))
     ms_per_step = t_ms / args.steps
-    value = world * flops * args.steps / (t_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, t_ms)
 
     # ---- per-kernel durations (events around each kernel, same rotation)
     nk = max(20, min(args.steps, 400))
@@ -351,7 +374,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     te_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e_value = world * flops * ke / (te_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(flops, ke, world, te_ms)
 
     peaks, peak_src = _measured_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
