@@ -11,30 +11,42 @@
 //      + [hi(u/alpha) | lo(u/alpha)] . [L2^T|L2^T]        (kind::f16, same D)
 //   y  = bf16(alpha * D + bias),   alpha = s_a * s_w
 //
-// Why pairs: the single-CTA kernel streams 54 KB of operands per K slice into
-// every SM and is bound by that load ring, not by the tensor cores.  Here a
-// cluster of two CTAs computes a 256 x 256 output tile: CTA r holds rows
+// A cluster of two CTAs computes a 256 x 256 output tile: CTA r holds rows
 // [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128) of the B
 // tile (half of N), the tensor cores of the two SMs exchange the B halves,
 // and each CTA accumulates its 128 rows x all 256 columns in its own tensor
-// memory.  Per SM and K slice that is A 16 KB + B 16 KB + scales 6 KB = 38 KB,
-// so five stages fit where four did.  Each CTA needs the scales of its own A
-// rows and of all 256 B rows (the block-scale layout of the M = 128 half).
+// memory.  Per SM and K slice that is A 16 KB + B 16 KB + scales 6 KB = 38 KB
+// of operands, against 54 KB for a 128 x 256 tile on one SM.
 //
-// Roles (9 warps per CTA; the MMA and scale-copy warps are idle in CTA 1):
-//   warp 0      TMA producer, both CTAs: loads into its own shared memory,
+// Tensor memory (512 columns per CTA) holds ONE accumulator (columns 0-255)
+// and one 48-column block-scale buffer per shared-memory stage (columns 256 +
+// 48 s).  The MMA warp copies a stage's scales into its buffer itself, right
+// before the MMAs that read them (tcgen05.cp then tcgen05.mma from the same
+// thread are executed in order; no barrier between them).  Tying the buffer
+// to the stage makes the copy safe without any wait either: a stage is
+// refilled only after the MMAs that read it, and its scale buffer, have
+// completed.  The price is the single accumulator: the MMAs of the next tile
+// start once the eight epilogue warps have pulled all 256 columns into
+// registers, which they do with four loads each, one wait, and an immediate
+// release.
+//
+// Every role loop runs on a whole warp and issues from one elected lane: the
+// tcgen05 and TMA instructions take uniform-register operands, and a loop
+// run by lane 0 alone keeps its addresses in per-thread registers, which
+// made each issue several times slower and the MMA warp, not the tensor
+// pipe, the bottleneck.
+//
+// Roles (10 warps per CTA; the MMA warp is idle in CTA 1):
+//   warps 0..7  epilogue, both CTAs: warp w reads TMEM lane quarter w % 4,
+//               columns [128 (w / 4), + 128) -> bf16 -> TMA store
+//   warp 8      TMA producer, both CTAs: loads into its own shared memory,
 //               completion bytes counted on CTA 0's full barrier
-//   warp 1      CTA 0: MMA issuer for the pair
-//   warps 2..5  epilogue, both CTAs: own accumulator rows -> bf16 -> TMA store
-//   warps 6..8  CTA 0: block-scale copies smem -> TMEM for both CTAs
-//               (tcgen05.cp .cta_group::2), one K slice ahead of the MMAs
+//   warp 9      CTA 0: block-scale copies and MMAs for the pair
 // Synchronisation across the pair:
 //   full[s]     CTA 0 only; CTA 0's producer arms it with both CTAs' bytes
 //   empty[s]    both CTAs; the MMA warp's commit multicasts to both
 //   acc_full    both CTAs; multicast commit after a tile's last MMA
-//   acc_empty   CTA 0 only; the epilogue warps of both CTAs arrive on it
-// Tensor memory per CTA as in the single-CTA kernel: accumulators at columns
-// 0 and 160 (96 shared), two 48-column scale buffers at 416 and 464.
+//   acc_empty   CTA 0 only; the 16 epilogue warps of both CTAs arrive on it
 // Every mbarrier wait is bounded; on timeout the kernel records a status code,
 // drains what it can observe, and both CTAs meet at the final cluster barrier.
 #include <cuda_bf16.h>
@@ -57,20 +69,19 @@ constexpr int SFA_BYTES = 4 * 512;                // 4 K64 chunks x 128 rows
 constexpr int SFB_BYTES = 2 * SFA_BYTES;          // both 128-row blocks of the tile's 256 B rows
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 38 KB
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of SWIZZLE_128B");
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int NUM_THREADS = (MMA_WARP + 1) * 32;
+constexpr int EPI_COLS = BN / 2;                  // columns per epilogue warp
 constexpr int EPI_CHUNK = 16;                     // columns per TMA store
 constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
-constexpr int SF_WARPS = 3;
-constexpr int SF_WARP0 = 2 + EPI_WARPS;
-constexpr int NUM_THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_STRIDE = 160;
-constexpr int ACC_OVERLAP = 2 * 256 - (ACC_STRIDE + 256);
-constexpr int SF_COLS = 48;
-constexpr int TMEM_SF0 = ACC_STRIDE + 256;
+constexpr int SF_COLS = 48;                       // SFA 16 + SFB 32 columns per K slice
+constexpr int TMEM_SF0 = BN;                      // scale buffer s at TMEM_SF0 + s * SF_COLS
 constexpr int TMEM_SFA_OFF = 0, TMEM_SFB_OFF = 16;
-static_assert(TMEM_SF0 + 2 * SF_COLS <= TMEM_COLS, "two scale buffers above the accumulators");
+static_assert(TMEM_SF0 + STAGES * SF_COLS <= TMEM_COLS, "one scale buffer per stage above the accumulator");
 constexpr uint16_t PAIR_MASK = 0x3;
 constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 
@@ -79,15 +90,13 @@ struct SmemCtl {
   uint64_t empty[STAGES];
   uint64_t acc_full;
   uint64_t acc_empty;
-  uint64_t sf_full[2];
-  uint64_t sf_empty[2];
   uint64_t drain;
-  uint64_t sf_drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + sizeof(SmemCtl);
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 // Instruction descriptors for M = 256 (the pair), N = 256.
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
@@ -96,6 +105,10 @@ constexpr uint32_t IDESC_BF16 =
 
 SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
+
+// bf16 pair (low half = the even column) -> two floats.
+SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+SVDQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -115,10 +128,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int tiles_n = (p.N + BN - 1) / BN;
   const int num_tiles = tiles_m * tiles_n;
   const int k_tiles = p.K / 256;
-  const int slices = k_tiles + 1;  // + the low-rank slice
+  const int slices = k_tiles + 1;  // + the low-rank slice (slice 0, no block scales)
 
   // Every CTA initialises the same barrier set; only CTA 0's full[],
-  // acc_empty and scale barriers are used.
+  // acc_empty and drain barriers are used.
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
@@ -126,16 +139,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(smem_u32(&ctl->acc_full), 1);
     mbar_init(smem_u32(&ctl->acc_empty), 2 * EPI_WARPS);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&ctl->sf_full[b]), SF_WARPS);
-      mbar_init(smem_u32(&ctl->sf_empty[b]), 1);
-    }
     mbar_init(smem_u32(&ctl->drain), 1);
-    mbar_init(smem_u32(&ctl->sf_drain), SF_WARPS);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_la);
@@ -144,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tmap(&tm_sfa);
     prefetch_tmap(&tm_sfb);
   }
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
     tmem_relinquish_pair();
   }
@@ -163,9 +171,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp == PRODUCER_WARP) {
+    {
       // ------------------------------------------------------------ producer
+      // The whole warp runs the loop; one elected lane issues the copies.
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;  // CTA 0: per stage, load outstanding and its parity
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int n0 = (tile / tiles_m) * BN;                          // the tile's B rows
         const int nb = n0 + (int)rank * BN_HALF;                       // this CTA's half of them
         for (int kt = 0; kt < slices; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
             ok = false;
             break;
           }
@@ -187,7 +196,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* ssfb = ssfa + SFA_BYTES;
           const uint32_t full_local = smem_u32(&ctl->full[stage]);
           const uint32_t full = rank == 0 ? full_local : mapa_shared(full_local, 0);
-          if (kt == 0) {
+          if (!elect_one()) {
+          } else if (kt == 0) {
             if (rank == 0) mbar_arrive_expect_tx(full_local, 2 * (A_BYTES + B_BYTES));
             tma_load_2d_pair(smem_u32(sa), &tm_la, 0, m0, full, pol);
             tma_load_2d_pair(smem_u32(sb), &tm_lb, 0, nb, full, pol);
@@ -203,6 +213,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d_pair(smem_u32(ssfb + SFA_BYTES), &tm_sfb, 0, ((n0 / 128 + 1) * kch + kb * 4) * 2, full,
                              pol);
           }
+          __syncwarp();
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -221,145 +232,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_wait(smem_u32(&ctl->full[s]), (issued_phase >> s) & 1, drain_ctx, kDevTimeoutDrain);
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+  } else if (warp == MMA_WARP) {
+    if (rank == 0) {
       // ------------------------------------------------------------ MMA issuer (CTA 0)
+      // The whole warp runs the loop; the same elected lane (the lowest)
+      // issues every MMA and commit, since a commit tracks the MMAs of the
+      // thread that issues it.
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      int it = 0;
-      uint32_t ks = 0;  // K slices computed so far (selects the scale buffer)
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
-        const uint32_t d_tmem = tmem + (uint32_t)((it & 1) * ACC_STRIDE);
-        // Both CTAs' epilogues have taken the shared columns of this accumulator.
-        if (!mbar_wait(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        // Both CTAs' epilogues have taken the previous tile's accumulator.
+        if (!mbar_wait_warp(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int kt = 0; kt < slices; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          if (kt == 0) {
+          const bool leader = elect_one();
+          if (!leader) {
+          } else if (kt == 0) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_bf16_pair(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
+              mma_bf16_pair(tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
           } else {
-            const uint32_t buf = ks & 1;
-            if (!mbar_wait(smem_u32(&ctl->sf_full[buf]), (ks >> 1) & 1, wctx, kDevTimeoutMma)) {
-              ok = false;
-              break;
+            // Scales smem -> this stage's TMEM buffer in both CTAs: per K64
+            // chunk j, SFA (4 columns) and the SFB of the tile's two 128-row
+            // blocks (4 columns each).
+            const uint32_t sf = tmem + TMEM_SF0 + stage * SF_COLS;
+            const uint32_t ssf = sa + A_BYTES + B_BYTES;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_pair_32x128_warpx4(sf + TMEM_SFA_OFF + 4 * j, sf_desc(ssf + 512 * j));
+              tmem_cp_pair_32x128_warpx4(sf + TMEM_SFB_OFF + 8 * j, sf_desc(ssf + SFA_BYTES + 512 * j));
+              tmem_cp_pair_32x128_warpx4(sf + TMEM_SFB_OFF + 4 + 8 * j, sf_desc(ssf + 2 * SFA_BYTES + 512 * j));
             }
-            tc_fence_after();
-            const uint32_t sf = tmem + TMEM_SF0 + buf * SF_COLS;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_nvfp4_pair(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_NVFP4,
+              mma_nvfp4_pair(tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_NVFP4,
                              sf + TMEM_SFA_OFF + 4 * j, sf + TMEM_SFB_OFF + 8 * j, 1u);
-            tc_commit_pair(smem_u32(&ctl->sf_empty[buf]));
-            ++ks;
           }
-          // Both CTAs may refill this stage once the MMAs reading it are done.
-          tc_commit_pair_mc(smem_u32(&ctl->empty[stage]), PAIR_MASK);
+          // Both CTAs may refill this stage (and its scale buffer) once the
+          // copies and MMAs reading it are done.
+          if (leader) tc_commit_pair_mc(smem_u32(&ctl->empty[stage]), PAIR_MASK);
+          __syncwarp();
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit_pair_mc(smem_u32(&ctl->acc_full), PAIR_MASK);
+        if (elect_one()) tc_commit_pair_mc(smem_u32(&ctl->acc_full), PAIR_MASK);
+        __syncwarp();
         acc_phase ^= 1;
       }
-      // Wait for every MMA this thread issued before tensor memory is freed.
-      tc_commit_pair(smem_u32(&ctl->drain));
+      // Wait for every MMA the elected lane issued before tensor memory is freed.
+      if (elect_one()) tc_commit_pair(smem_u32(&ctl->drain));
+      __syncwarp();
       volatile int never = 0;
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
     }
-  } else if (warp >= SF_WARP0) {
-    if (lane == 0 && rank == 0) {
-      // ------------------------------------------------------------ scale copies (CTA 0, for both)
-      // Warp SF_WARP0 + w copies part w of every K slice's block scales in
-      // both CTAs: w = 0: SFA, w = 1 / 2: SFB rows 0-127 / 128-255 of the tile.
-      const int w = warp - SF_WARP0;
-      int stage = 0;
-      uint32_t phase = 0, ks = 0;
-      bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        for (int kt = 0; kt < slices; ++kt) {
-          if (kt > 0) {
-            const uint32_t buf = ks & 1;
-            // The MMAs of the K slice two back read this buffer; wait for them.
-            if (ks >= 2 && !mbar_wait(smem_u32(&ctl->sf_empty[buf]), ((ks - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
-              ok = false;
-              break;
-            }
-            // full[] completes only when both CTAs' scales have landed.
-            if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t ssfa = smem_u32(stage_base + stage * STAGE_BYTES) + A_BYTES + B_BYTES;
-            const uint32_t src = ssfa + SFA_BYTES * w;
-            const uint32_t dst = tmem + TMEM_SF0 + buf * SF_COLS + (w == 0 ? TMEM_SFA_OFF : TMEM_SFB_OFF + 4 * (w - 1));
-            const uint32_t col_step = w == 0 ? 4 : 8;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_cp_pair_32x128_warpx4(dst + col_step * j, sf_desc(src + 512 * j));
-            tc_commit_pair(smem_u32(&ctl->sf_full[buf]));
-            ++ks;
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      tc_commit_pair(smem_u32(&ctl->sf_drain));
-      volatile int never = 0;
-      WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
-      mbar_wait(smem_u32(&ctl->sf_drain), 0, drain_ctx, kDevTimeoutDrain);
-    }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
-    // Each warp owns 32 rows (its TMEM lane quarter) of this CTA's 128 rows x
-    // 256 columns, read from TMEM 32 columns at a time into a ring of three
-    // register blocks: the chunks holding the columns shared with the other
-    // accumulator first, one wait, then the release on CTA 0's acc_empty
-    // (remote for CTA 1) before anything is converted.
-    const int q = warp & 3;
-    uint8_t* buf0 = epi_base + (warp - 2) * 2 * EPI_BUF_BYTES;
+    // Warp w owns 32 rows (TMEM lane quarter w % 4) x 128 columns (half
+    // w / 4) of this CTA's 128 x 256 accumulator.  It loads all of them with
+    // four TMEM loads and one wait, releases the accumulator on CTA 0's
+    // acc_empty (remote for CTA 1), and only then converts and stores.
+    const int q = warp & 3, h = warp >> 2;
+    uint8_t* buf0 = epi_base + warp * 2 * EPI_BUF_BYTES;
     const uint32_t acc_empty_local = smem_u32(&ctl->acc_empty);
     const uint32_t acc_empty_leader = rank == 0 ? acc_empty_local : mapa_shared(acc_empty_local, 0);
+    const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * EPI_COLS);
     uint32_t acc_phase = 0;
-    int chunk_seq = 0, it = 0;
-    constexpr int LDC = 32;
-    constexpr int NCH = BN / LDC;
-    constexpr int NSH = (ACC_OVERLAP + LDC - 1) / LDC;
-    constexpr int NBUF = 3;
-    static_assert(NSH <= NBUF, "the shared chunks fit the first ring fill");
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+    int chunk_seq = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
       const int m0 = (tile % tiles_m) * 2 * BM + (int)rank * BM;
-      const int n0 = (tile / tiles_m) * BN;
-      const int b = it & 1;
-      uint4 bias8 = make_uint4(0, 0, 0, 0);
-      if (p.bias != nullptr && n0 + 8 * lane < p.N) bias8 = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + lane);
+      const int nw = (tile / tiles_m) * BN + h * EPI_COLS;   // this warp's first column
+      // Lane l holds the bias of columns nw + 4 l .. nw + 4 l + 3.
+      uint2 bias4 = make_uint2(0, 0);
+      if (p.bias != nullptr && nw + 4 * lane < p.N) bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + nw) + lane);
       const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
       tc_fence_after();
-      const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
-      auto chunk_col = [&](int i) { return b == 0 ? (i + NCH - NSH) % NCH : i; };
-      uint32_t rb[NBUF][32];
+      uint32_t r[4][32];
 #pragma unroll
-      for (int i = 0; i < NBUF; ++i) tmem_ld_32x32b_x32(acc_base + chunk_col(i) * LDC, rb[i]);
-      tmem_ld_wait(rb[0]);
-      reg_fence(rb[1]);
-      reg_fence(rb[2]);
+      for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(acc_base + 32 * i, r[i]);
+      tmem_ld_wait(r[0]);
+      reg_fence(r[1]);
+      reg_fence(r[2]);
+      reg_fence(r[3]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -369,33 +338,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive_cluster(acc_empty_leader);
       }
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        uint32_t(&r)[32] = rb[i % NBUF];
-        if (i >= NBUF && i % NBUF == 0) {
-          tmem_ld_wait(rb[0]);
-          reg_fence(rb[1]);
-          reg_fence(rb[2]);
-        }
-        const int cc = chunk_col(i);
+      for (int i = 0; i < 4; ++i) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {      // two 16-column halves per TMEM load
-          const int ncol = n0 + cc * LDC + hh * EPI_CHUNK;
-          const int src_lane = (cc * LDC + hh * EPI_CHUNK) / 8;  // lanes src_lane, src_lane + 1
+          const int c0 = 32 * i + EPI_CHUNK * hh;
+          const int ncol = nw + c0;
           uint32_t bw[8];
-          bw[0] = __shfl_sync(0xffffffffu, bias8.x, src_lane);
-          bw[1] = __shfl_sync(0xffffffffu, bias8.y, src_lane);
-          bw[2] = __shfl_sync(0xffffffffu, bias8.z, src_lane);
-          bw[3] = __shfl_sync(0xffffffffu, bias8.w, src_lane);
-          bw[4] = __shfl_sync(0xffffffffu, bias8.x, src_lane + 1);
-          bw[5] = __shfl_sync(0xffffffffu, bias8.y, src_lane + 1);
-          bw[6] = __shfl_sync(0xffffffffu, bias8.z, src_lane + 1);
-          bw[7] = __shfl_sync(0xffffffffu, bias8.w, src_lane + 1);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            bw[2 * j] = __shfl_sync(0xffffffffu, bias4.x, c0 / 4 + j);
+            bw[2 * j + 1] = __shfl_sync(0xffffffffu, bias4.y, c0 / 4 + j);
+          }
           uint32_t packed[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float b0 = __uint_as_float(bw[k] << 16), b1 = __uint_as_float(bw[k] & 0xFFFF0000u);
-            const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[hh * 16 + 2 * k]), b0);
-            const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[hh * 16 + 2 * k + 1]), b1);
+            const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[i][hh * 16 + 2 * k]), bf16_lo(bw[k]));
+            const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[i][hh * 16 + 2 * k + 1]), bf16_hi(bw[k]));
             __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
             packed[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
@@ -415,7 +373,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) bulk_commit();
           ++chunk_seq;
         }
-        if (i + NBUF < NCH) tmem_ld_32x32b_x32(acc_base + chunk_col(i + NBUF) * LDC, r);
       }
       acc_phase ^= 1;
     }
@@ -427,7 +384,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncwarp();
   tc_fence_before();
   cluster_sync();
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, TMEM_COLS);
   }

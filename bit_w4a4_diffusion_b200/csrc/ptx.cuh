@@ -74,6 +74,27 @@ SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int c
   }
 }
 
+// The same wait taken by a whole converged warp, with a warp-uniform result
+// (false if any lane gave up).  Role loops run on all 32 lanes and issue
+// their single-thread instructions from one elected lane, so that the
+// compiler keeps the loop's addresses and descriptors in uniform registers,
+// which tcgen05 and TMA instructions take as operands.
+SVDQ_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int code) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctx, code));
+}
+
+// True in exactly one lane of the converged warp (the lowest active lane,
+// so the same lane every time the whole warp calls it).
+SVDQ_DEV bool elect_one() {
+  uint32_t is;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(is));
+  return is != 0;
+}
+
 // Named barrier `id` over `nthreads` threads that also returns, to every
 // participant, whether any of them passed a true `flag` (bar.red.or): a
 // decision taken this way is the same in every thread.
