@@ -282,8 +282,12 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
 
   // ---------------------------------------------------------------- roles
+  // Role loops run on the whole warp and issue from one elected lane (the
+  // lowest, the same one every time): tcgen05 and TMA instructions take
+  // uniform-register operands, which a loop run by lane 0 alone does not
+  // keep, and each issue then costs several times more.
   auto role_producer = [&]() {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ producer
       int stage = 0;
       uint32_t phase = 0;
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
         const int m0 = tile_m0(tile);
         const int n0 = tile_n0(tile);
         for (int kt = 0; kt < slices; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
             ok = false;
             break;
           }
@@ -303,7 +307,8 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           uint8_t* ssfa = sb + B_BYTES;
           uint8_t* ssfb = ssfa + SFA_BYTES;
           const uint32_t full = smem_u32(&ctl->full[stage]);
-          if (kt == 0) {
+          if (!elect_one()) {
+          } else if (kt == 0) {
             mbar_arrive_expect_tx(full, A_BYTES + B_BYTES);
             tma_load_2d(smem_u32(sa), &tm_la, 0, m0, full);
             tma_load_2d_hint(smem_u32(sb), &tm_lb, 0, n0, full, pol_w);
@@ -318,6 +323,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
             bulk_load(smem_u32(ssfb + SFA_BYTES), p.w_scales + ((size_t)(n0 / 128 + 1) * kch + kb * 4) * 512,
                       SFA_BYTES, full);
           }
+          __syncwarp();
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
     }
   };
   auto role_mma = [&]() {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
@@ -344,13 +350,13 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
       uint32_t ks = 0;  // K slices computed so far (selects the scale buffer)
       for (int tile = t_begin; tile < t_end && ok; tile += t_step, ++it) {
         const uint32_t d_tmem = tmem + (uint32_t)((it & 1) * ACC_STRIDE);
-        if (!mbar_wait(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
+        if (!mbar_wait_warp(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int kt = 0; kt < slices; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
             ok = false;
             break;
           }
@@ -358,43 +364,52 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
           if (kt == 0) {
+            if (elect_one()) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              mma_bf16(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
+              for (int j = 0; j < 4; ++j)
+                mma_bf16(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
+            }
+            __syncwarp();
           } else {
             const uint32_t buf = ks & 1;
-            if (!mbar_wait(smem_u32(&ctl->sf_full[buf]), (ks >> 1) & 1, wctx, kDevTimeoutMma)) {
+            if (!mbar_wait_warp(smem_u32(&ctl->sf_full[buf]), (ks >> 1) & 1, wctx, kDevTimeoutMma)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t sf = tmem + TMEM_SF0 + buf * SF_COLS;
+            if (elect_one()) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              mma_nvfp4(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_NVFP4,
-                        sf + TMEM_SFA_OFF + 4 * j, sf + TMEM_SFB_OFF + 8 * j, 1u);
-            tc_commit(smem_u32(&ctl->sf_empty[buf]));
+              for (int j = 0; j < 4; ++j)
+                mma_nvfp4(d_tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_NVFP4,
+                          sf + TMEM_SFA_OFF + 4 * j, sf + TMEM_SFB_OFF + 8 * j, 1u);
+              tc_commit(smem_u32(&ctl->sf_empty[buf]));
+            }
+            __syncwarp();
             ++ks;
           }
-          tc_commit(smem_u32(&ctl->empty[stage]));
+          if (elect_one()) tc_commit(smem_u32(&ctl->empty[stage]));
+          __syncwarp();
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(&ctl->acc_full));
+        if (elect_one()) tc_commit(smem_u32(&ctl->acc_full));
+        __syncwarp();
         acc_phase ^= 1;
       }
-      // Wait for every MMA / copy this thread issued before TMEM is freed.
-      tc_commit(smem_u32(&ctl->drain));
+      // Wait for every MMA the elected lane issued before TMEM is freed.
+      if (elect_one()) tc_commit(smem_u32(&ctl->drain));
+      __syncwarp();
       volatile int never = 0;
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
     }
   };
   auto role_scale_copies = [&]() {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ scale copies
       // Three jobs per K slice: 0 = SFA (4 copies), 1 / 2 = SFB rows 0-127 /
       // 128-255 (4 each); scale-copy warp w takes jobs w, w + SF_WARPS, ...
@@ -407,17 +422,19 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           if (kt > 0) {
             const uint32_t buf = ks & 1;
             // The MMAs of the K slice two back read this buffer; wait for them.
-            if (ks >= 2 && !mbar_wait(smem_u32(&ctl->sf_empty[buf]), ((ks - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+            if (ks >= 2 &&
+                !mbar_wait_warp(smem_u32(&ctl->sf_empty[buf]), ((ks - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
               ok = false;
               break;
             }
-            if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
+            if (!mbar_wait_warp(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutMma)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t ssfa = smem_u32(stage_base + stage * STAGE_BYTES) + A_BYTES + B_BYTES;
-            for (int job = w; job < 3; job += R::SF_WARPS) {
+            const bool leader = elect_one();
+            for (int job = w; job < 3 && leader; job += R::SF_WARPS) {
               const uint32_t src = job == 0 ? ssfa : ssfa + SFA_BYTES * job;
               const uint32_t dst =
                   tmem + TMEM_SF0 + buf * SF_COLS + (job == 0 ? TMEM_SFA_OFF : TMEM_SFB_OFF + 4 * (job - 1));
@@ -425,7 +442,8 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
 #pragma unroll
               for (int j = 0; j < 4; ++j) tmem_cp_32x128_warpx4(dst + col_step * j, sf_desc(src + 512 * j));
             }
-            tc_commit(smem_u32(&ctl->sf_full[buf]));
+            if (leader) tc_commit(smem_u32(&ctl->sf_full[buf]));
+            __syncwarp();
             ++ks;
           }
           if (++stage == STAGES) {
@@ -434,7 +452,8 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           }
         }
       }
-      tc_commit(smem_u32(&ctl->sf_drain));
+      if (elect_one()) tc_commit(smem_u32(&ctl->sf_drain));
+      __syncwarp();
       volatile int never = 0;
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->sf_drain), 0, drain_ctx, kDevTimeoutDrain);

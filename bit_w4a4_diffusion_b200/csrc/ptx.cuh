@@ -44,6 +44,25 @@ SVDQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread stays suspended at most about `hint_ns` nanoseconds
+// waiting for the phase (the suspend-time hint of mbarrier.try_wait).
+SVDQ_DEV bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits below this (nanoseconds) are also passed to try_wait as its suspend
+// hint, so that a single poll cannot outlast the limit; longer limits keep the
+// hardware's own suspend window.
+constexpr unsigned long long kShortWaitNs = 100000ull;
+
 // Bounded wait on an mbarrier phase.  Gives up (returns false) when the shared
 // abort word is set by another role, or when `limit_ns` of wall time has
 // passed, in which case it records `code` in the caller's device status word
@@ -55,7 +74,10 @@ struct WaitCtx {
 };
 
 SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool short_limit = ctx.limit_ns < kShortWaitNs;
+  const uint32_t hint = (uint32_t)ctx.limit_ns;
+  auto poll = [&]() { return short_limit ? mbar_try_wait_hint(bar, parity, hint) : mbar_try_wait(bar, parity); };
+  if (poll()) return true;
   const uint64_t t0 = globaltimer_ns();
   // The abort word and the clock are read after the first failed poll and
   // then every 64 polls (try_wait itself suspends the thread for a while, so
@@ -70,7 +92,7 @@ SVDQ_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx, int c
         return false;
       }
     }
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll()) return true;
   }
 }
 

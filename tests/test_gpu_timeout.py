@@ -86,7 +86,9 @@ def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
     """The GELU-MLP kernel (eight epilogue warps that stop together)."""
     import dataclasses
     import bit_w4a4_diffusion_b200 as B
-    up = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=640, K=768, N=1024), bias_std=0.1)
+    # K = 3072: thirteen K slices per tile, so that the load ring fills and
+    # the waits last longer than the device clock's resolution.
+    up = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=640, K=3072, N=1024), bias_std=0.1)
     dn = dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=640, K=1024, N=768), bias_std=0.05)
     iu, idn = svdq_inputs(up), svdq_inputs(dn)
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
@@ -123,7 +125,7 @@ def test_qkv_gemm_wait_timeout_reports_and_recovers():
     """The QKV + RMSNorm + RoPE kernel (eight epilogue warps that stop together)."""
     import bit_w4a4_diffusion_b200 as B
     from oracle import qkv as OQ
-    M, K, heads = 384, 512, 2
+    M, K, heads = 640, 3072, 2       # thirteen K slices per tile, as above
     inp = svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, K=K, N=3 * heads * 128))
     pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
