@@ -26,9 +26,9 @@
 // to the stage makes the copy safe without any wait either: a stage is
 // refilled only after the MMAs that read it, and its scale buffer, have
 // completed.  The price is the single accumulator: the MMAs of the next tile
-// start once the eight epilogue warps have pulled all 256 columns into
-// registers, which they do with four loads each, one wait, and an immediate
-// release.
+// start once the eight epilogue warps of both CTAs have pulled all 256
+// columns into registers, which they do with four loads each, one wait, and
+// an immediate release (about 0.3 us after the tile's last MMA completes).
 //
 // Every role loop runs on a whole warp and issues from one elected lane: the
 // tcgen05 and TMA instructions take uniform-register operands, and a loop
@@ -329,13 +329,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       reg_fence(r[1]);
       reg_fence(r[2]);
       reg_fence(r[3]);
+      // The loads are complete (wait::ld) and ordered before the arrive by
+      // the tcgen05 fence, which is all the MMA warp needs before it
+      // overwrites the accumulator: CTA 1's remote arrive is relaxed.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         if (rank == 0)
           mbar_arrive(acc_empty_local);
         else
-          mbar_arrive_cluster(acc_empty_leader);
+          mbar_arrive_cluster_relaxed(acc_empty_leader);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
