@@ -36,17 +36,17 @@ FP4_PER_BF16 = 4.0                  # nominal dense FP4 : BF16 throughput ratio
 L2_BYTES = 126 * 2 ** 20
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# gemm_nvfp4 launch on this workload, from the ncu capture summarised in
-# profiles/gemm_nvfp4_mlp_up.md, keyed by the SHA-256 of the kernel sources
-# it was taken from: once a source changes the figure no longer applies and
-# the bench reports null.
+# gemm_nvfp4_pair launch (the S2 kernel of this workload) from the ncu
+# capture summarised in profiles/gemm_nvfp4_pair_mlp_up.md, keyed by the
+# SHA-256 of the kernel sources it was taken from: once a source changes the
+# figure no longer applies and the bench reports null.
 GEMM_TRAFFIC = {
-    "bytes": 30504448 + 52442112,
+    "bytes": 30466304 + 51708160,
     "sources": {
-        "bit_w4a4_diffusion_b200/csrc/gemm_nvfp4.cu":
-            "9127be58f1dd95c4b0094de9c40f9cf65701338b256744677e628ed834efbe36",
+        "bit_w4a4_diffusion_b200/csrc/gemm_nvfp4_pair.cu":
+            "335cb9e52d85dde5c510513bdeba394f5bc2da09c6ae070b2cac9260be98ae70",
         "bit_w4a4_diffusion_b200/csrc/ptx.cuh":
-            "9f85b0a5d89f666dbb1ded5928e19d0fede8af584361f283b893195e630aaa34",
+            "0fc4f8397b047cb7e671a96e27db4ae851492977f51770aa6068061781bf9cae",
     },
 }
 
@@ -387,7 +387,7 @@ def run_gpu(args, rank, world, local_rank):
         "config": workload_config(M, K, N, world),
         "pct_of_fp4_peak": {"spec_dense_9pf": round(100 * value / world / FP4_SPEC_DENSE_TFLOPS, 2),
                             f"{peak_src}_bf16x4": round(100 * value / world / fp4_peak, 2)},
-        "roofline": {"kernel": "gemm_nvfp4 (S2)", "bound": "tensor", "achieved": round(s2_tflops, 1),
+        "roofline": {"kernel": "gemm_nvfp4_pair (S2)", "bound": "tensor", "achieved": round(s2_tflops, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(s2_tflops / fp4_peak, 4),
                      "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} "
                                     f"(nominal fp4:bf16 dense ratio)",
@@ -661,7 +661,11 @@ def run_profile_calls(row, calls):
     size, untimed (the commands the per-row profiles are taken with):
     awq (M = 1, N = 18432, K = 3072, six rotating weight sets), int4 (the
     INT4 layer at M = 4096, K = N = 3072, four sets), qkv (the fused QKV
-    projection with RMSNorm and RoPE, two sets), mlp (the fused DiT MLP)."""
+    projection with RMSNorm and RoPE, two sets), mlp (the fused DiT MLP),
+    layer (the headline NVFP4 layer, M = 4096, K = 3072, N = 12288, four
+    sets), cublas_fp4 (for comparison only: torch's block-scaled NVFP4 matmul,
+    a cuBLAS kernel, on the same shape with random codes and unit scales,
+    three weight sets; no low-rank branch, no bias)."""
     import torch
     import bit_w4a4_diffusion_b200 as B
     import workloads as wl
@@ -684,6 +688,25 @@ def run_profile_calls(row, calls):
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
         wsp = torch.empty(B.workspace_bytes("int4", c.M, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=y, workspace=wsp) for i in range(4)]
+    elif row == "cublas_fp4":
+        M, K, N = 4096, 3072, 12288
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2)
+        bs = [torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2)
+              for _ in range(3)]
+        sa = torch.ones((M, K // 16), device=dev).to(torch.float8_e4m3fn)
+        sb = torch.ones((N, K // 16), device=dev).to(torch.float8_e4m3fn)
+        fns = [lambda i=i: torch._scaled_mm(a, bs[i].t(), sa, sb, out_dtype=torch.bfloat16) for i in range(3)]
+    elif row == "layer":
+        c = wl.SVDQ_CASES[WORKLOAD]
+        inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
+        pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+        ws = [B.to_device(pk, dev) for _ in range(4)]
+        x = B.bits_to_bf16(inp.x_bits, dev)
+        bias = B.bits_to_bf16(inp.bias_bits, dev) if inp.bias_bits is not None else None
+        y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device=dev)
+        fns = [lambda i=i: B.svdq_w4a4_linear("nvfp4", x, ws[i], float(inp.act_scale), bias=bias, y=y, workspace=wsp)
+               for i in range(4)]
     elif row == "qkv":
         c = wl.SVDQ_CASES["qkv"]
         inp = wl.make_svdq_inputs(c, B.svdq_calibrate)
@@ -766,7 +789,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ / MLP row measurements")
     ap.add_argument("--mlp-calls", type=int, default=0,
                     help="only run this many fused DiT MLP calls (untimed; for profiling) and exit")
-    ap.add_argument("--profile", choices=["awq", "int4", "qkv", "mlp"], default=None,
+    ap.add_argument("--profile", choices=["awq", "int4", "qkv", "mlp", "layer", "cublas_fp4"], default=None,
                     help="only run --calls calls of one row's entry point (untimed; for profiling) and exit")
     ap.add_argument("--calls", type=int, default=5)
     args = ap.parse_args()
