@@ -25,6 +25,14 @@
 // every slice for rows [16 (w / 8), 16 (w / 8) + 16).  Lane (g, c) holds 8
 // consecutive elements of two rows, which are its mma.m16n8k16 A fragments
 // under the k-permutation of the first kernel.
+//
+// Two orderings keep the memory system busy.  CTA b walks the K slices
+// starting at slice b mod (K / 256): in lockstep every CTA would read the
+// same 16 KB of L1^T from the same few L2 slices at once.  And lane (g, c)
+// takes rows (and ranks) perm(g), perm(g) + 8 with perm = 0 4 1 5 2 6 3 7:
+// the 128-byte swizzle places rows r and r + 1 in the same bank groups, so
+// the two rows of one quarter-warp load must differ in bit 2 to avoid a
+// two-way bank conflict.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -56,7 +64,9 @@ struct QnCtl {
   int abort_flag;
 };
 
-constexpr size_t QN_SMEM_BYTES = 1024 + QN_STAGES * QN_STAGE_BYTES + sizeof(QnCtl);
+// 1/d for every E4M3 scale byte (d = E4M3(b) * s_a), 0 where d = 0.
+constexpr int QN_RCP_BYTES = 256 * 4;
+constexpr size_t QN_SMEM_BYTES = 1024 + QN_STAGES * QN_STAGE_BYTES + QN_RCP_BYTES + sizeof(QnCtl);
 constexpr unsigned long long kQnDrainLimitNs = 2000000000ull;
 
 // Address of the 16-byte chunk holding elements [8 j, 8 j + 8) of row r in a
@@ -85,11 +95,18 @@ SVDQ_DEV uint32_t f16x2(float lo, float hi) {
   return out;  // lo in the low half
 }
 
-// Two fp32 -> one byte of two E2M1 codes (lo in bits 0-3), RNE, satfinite.
-SVDQ_DEV uint32_t e2m1x2(float lo, float hi) {
+// Eight fp32 (pairs lo, hi) -> four bytes of E2M1 codes, element 2i in bits
+// 8i..8i+3 and element 2i+1 in bits 8i+4..8i+7; RNE, satfinite.
+SVDQ_DEV uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
   uint32_t out;
-  asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
-      : "=r"(out) : "f"(lo), "f"(hi));
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
   return out;
 }
 
@@ -110,13 +127,21 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
                           const QuantActParams p, int* dev_status, unsigned long long timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  QnCtl* ctl = reinterpret_cast<QnCtl*>(smem + QN_STAGES * QN_STAGE_BYTES);
+  float* rcp_tab = reinterpret_cast<float*>(smem + QN_STAGES * QN_STAGE_BYTES);
+  QnCtl* ctl = reinterpret_cast<QnCtl*>(smem + QN_STAGES * QN_STAGE_BYTES + QN_RCP_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = p.K;
   const int nslices = K / QN_SLICE;
   const int row_base = blockIdx.x * QN_ROWS;
+  const int slice0 = (int)(blockIdx.x % (unsigned)nslices);   // this CTA's first K slice
   pdl_wait();  // x of the previous kernel's making
 
+  if (threadIdx.x < 256) {
+    // The reciprocal each group's codes are scaled by, for every scale byte
+    // the quantizer can produce (the formula of the per-group computation).
+    const float d = __fmul_rn(e4m3_to_float(threadIdx.x), p.act_scale);
+    rcp_tab[threadIdx.x] = d != 0.f ? __frcp_rn(d) : 0.f;   // 0 marks an all-zero group
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < QN_STAGES; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
@@ -140,7 +165,8 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
         if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) break;
         const uint32_t base = smem_u32(smem + stage * QN_STAGE_BYTES);
         const uint32_t full = smem_u32(&ctl->full[stage]);
-        const int k0 = sl * QN_SLICE;
+        const int ks = sl + slice0 < nslices ? sl + slice0 : sl + slice0 - nslices;
+        const int k0 = ks * QN_SLICE;
         mbar_arrive_expect_tx(full, QN_STAGE_BYTES);
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
@@ -163,7 +189,8 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
     const int blk = warp & 7;            // 32-wide block within each slice
     const int half = warp >> 3;          // rows [16 half, 16 half + 16)
     const int g = lane >> 2, c = lane & 3;
-    const int r0 = 16 * half + g, r1 = r0 + 8;           // rows within the CTA
+    const int pg = ((g & 1) << 2) | (g >> 1);            // perm(g): see the header
+    const int r0 = 16 * half + pg, r1 = r0 + 8;          // rows within the CTA
     const int row0 = row_base + r0, row1 = row_base + r1;
     const bool ok0 = row0 < p.M, ok1 = row1 < p.M;
     const int box = blk >> 1;                            // 64-wide box holding this block
@@ -177,6 +204,13 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+    // This lane's code word and (even lanes) scale byte of K slice 0; slice
+    // ks adds ks * 128 code bytes and ks * 2048 scale bytes (the tiled scale
+    // layout: group 16 ks + 2 blk + c / 2).
+    uint8_t* const code0 = p.act_codes + (size_t)row0 * (K / 2) + blk * 16 + 4 * c;
+    uint8_t* const code1 = p.act_codes + (size_t)row1 * (K / 2) + blk * 16 + 4 * c;
+    uint8_t* const sc0 = p.act_scales + scale_offset(row0, 2 * blk + (c >> 1), K);
+    uint8_t* const sc1 = p.act_scales + scale_offset(row1, 2 * blk + (c >> 1), K);
 
     for (int sl = 0; sl < nslices; ++sl) {
       const int stage = sl % QN_STAGES;
@@ -192,7 +226,7 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
       const uint4 i0 = lds128(iaddr), i1 = lds128(iaddr + 16);
       uint4 bw[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bw[j] = lds128(sw128_chunk(lbox, 8 * j + g, chunk));
+      for (int j = 0; j < 4; ++j) bw[j] = lds128(sw128_chunk(lbox, 8 * j + pg, chunk));   // rank 8 j + perm(g)
       // Every read of this stage is in registers: release it.
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->empty[stage]));
@@ -221,35 +255,26 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
       a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
       // The even lane derives row g's scale, the odd lane row g+8's; they swap.
       const uint32_t sb_m = cvt_e4m3(__fmul_rn(odd ? a1 : a0, inv_six_s));
-      const float d_m = __fmul_rn(e4m3_to_float(sb_m), s_a);
-      const float r_m = d_m != 0.f ? __frcp_rn(d_m) : 0.f;   // 0 marks an all-zero group
+      const float r_m = rcp_tab[sb_m & 0xFF];                   // 0 marks an all-zero group
       const float r_o = __shfl_xor_sync(0xffffffffu, r_m, 1);
       const uint32_t sb_o = __shfl_xor_sync(0xffffffffu, sb_m, 1);
       const float q0 = odd ? r_o : r_m, q1 = odd ? r_m : r_o;
-      uint32_t w0 = 0, w1 = 0;
-      if (q0 != 0.f) {
-        const float2 qq = make_float2(q0, q0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 t = __fmul2_rn(v0[i], qq);
-          w0 |= e2m1x2(t.x, t.y) << (8 * i);
-        }
-      }
-      if (q1 != 0.f) {
-        const float2 qq = make_float2(q1, q1);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 t = __fmul2_rn(v1[i], qq);
-          w1 |= e2m1x2(t.x, t.y) << (8 * i);
-        }
-      }
-      const int k = sl * QN_SLICE + blk * 32 + 8 * c;
-      if (ok0) __stcs(reinterpret_cast<unsigned int*>(p.act_codes + (size_t)row0 * (K / 2) + k / 2), w0);
-      if (ok1) __stcs(reinterpret_cast<unsigned int*>(p.act_codes + (size_t)row1 * (K / 2) + k / 2), w1);
+      // An all-zero group (scale byte 0) gets all-zero codes, also where a
+      // value is -0 or a tiny negative.
+      const float2 qq0 = make_float2(q0, q0), qq1 = make_float2(q1, q1);
+      const uint32_t w0 = q0 != 0.f ? e2m1x8(__fmul2_rn(v0[0], qq0), __fmul2_rn(v0[1], qq0), __fmul2_rn(v0[2], qq0),
+                                             __fmul2_rn(v0[3], qq0))
+                                    : 0u;
+      const uint32_t w1 = q1 != 0.f ? e2m1x8(__fmul2_rn(v1[0], qq1), __fmul2_rn(v1[1], qq1), __fmul2_rn(v1[2], qq1),
+                                             __fmul2_rn(v1[3], qq1))
+                                    : 0u;
+      const int ks = sl + slice0 < nslices ? sl + slice0 : sl + slice0 - nslices;
+      if (ok0) __stcs(reinterpret_cast<unsigned int*>(code0 + ks * (QN_SLICE / 2)), w0);
+      if (ok1) __stcs(reinterpret_cast<unsigned int*>(code1 + ks * (QN_SLICE / 2)), w1);
       if (!odd) {
-        const int grp = k >> 4;
-        p.act_scales[scale_offset(row0, grp, K)] = (uint8_t)(odd ? sb_o : sb_m);  // rows >= M: zero input, scale 0
-        p.act_scales[scale_offset(row1, grp, K)] = (uint8_t)(odd ? sb_m : sb_o);
+        // 16 groups of 16 per slice = 4 chunks of 512 scale bytes.
+        sc0[(size_t)ks * 2048] = (uint8_t)sb_m;  // rows >= M: zero input, scale 0
+        sc1[(size_t)ks * 2048] = (uint8_t)sb_o;
       }
 
       // ---- low-rank down-projection: A = x_hat * 2^-e in fp16.
@@ -281,12 +306,14 @@ __global__ void __launch_bounds__(QN_THREADS, 1)
     __syncwarp();
     asm volatile("bar.sync 1, %0;" ::"n"(QN_COMPUTE_WARPS * 32));
     float(*red)[QN_ROWS][33] = reinterpret_cast<float(*)[QN_ROWS][33]>(smem);
+    // Accumulator columns 2c, 2c + 1 of n-tile j are ranks 8 j + perm(2c) =
+    // 8 j + c and 8 j + perm(2c + 1) = 8 j + 4 + c.
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      red[blk][r0][8 * j + 2 * c] = acc[j][0];
-      red[blk][r0][8 * j + 2 * c + 1] = acc[j][1];
-      red[blk][r1][8 * j + 2 * c] = acc[j][2];
-      red[blk][r1][8 * j + 2 * c + 1] = acc[j][3];
+      red[blk][r0][8 * j + c] = acc[j][0];
+      red[blk][r0][8 * j + 4 + c] = acc[j][1];
+      red[blk][r1][8 * j + c] = acc[j][2];
+      red[blk][r1][8 * j + 4 + c] = acc[j][3];
     }
     asm volatile("bar.sync 1, %0;" ::"n"(QN_COMPUTE_WARPS * 32));
     for (int idx = threadIdx.x; idx < QN_ROWS * 32; idx += QN_COMPUTE_WARPS * 32) {
