@@ -232,17 +232,22 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
                     "quantize_act launch");
 }
 
-// NVFP4 GEMM kernel: the CTA-pair kernel (256 x 256 tiles on two SMs)
-// unless SVDQ_NVFP4_GEMM_KERNEL=single asks for the one-CTA-per-tile kernel
-// (read at every call, so a process can compare the two).  Both give
-// bit-identical results.  On B200 the pair kernel is 14-26% faster on the DiT
-// layer shapes: it streams 38 KB of operands per SM and K slice instead of 54,
-// and keeps one block-scale buffer per stage so its MMA warp never waits on
-// the scale copies.  The fused GELU-MLP and QKV epilogues use the
-// single-CTA kernel.
-static bool use_pair_gemm() {
+// NVFP4 GEMM kernel per epilogue kind.  SVDQ_NVFP4_GEMM_KERNEL=pair or
+// =single (read at every call, so a process can compare them) forces the
+// CTA-pair kernel (256 x 256 tiles on two SMs) or the one-CTA-per-tile
+// kernel for every kind; both give bit-identical results (up to the order of
+// the GELU-MLP epilogue's atomic low-rank sums).  By default the pair kernel
+// runs the plain and QKV epilogues: it streams 38 KB of operands per SM and K
+// slice instead of 54 and keeps one block-scale buffer per stage, 14-26%
+// faster on the DiT layer shapes and 10% on the fused QKV projection.  The
+// GELU-MLP epilogue stays on the single-CTA kernel: it is bound by its own
+// arithmetic, which the pair's faster main loop does not shorten, and the
+// pair's single accumulator makes it 4% slower there.
+static bool use_pair_gemm(bool gelu) {
   const char* v = getenv("SVDQ_NVFP4_GEMM_KERNEL");
-  return !(v && strcmp(v, "single") == 0);
+  if (v && strcmp(v, "single") == 0) return false;
+  if (v && strcmp(v, "pair") == 0) return true;
+  return !gelu;
 }
 
 // gq != nullptr selects the GELU-MLP epilogue, qk != nullptr the QKV +
@@ -277,15 +282,9 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
   p.alpha = alpha;
   p.dev_status = dev_status;
   p.timeout_ns = svdq_timeout_ns();
-  if (gq != nullptr) {
-    p.gq = *gq;
-    return check_cuda(launch_gemm_nvfp4_gelu(p, t, sms, stream, pdl), "gemm_nvfp4 (GELU-MLP epilogue) launch");
-  }
-  if (qk != nullptr) {
-    p.qk = *qk;
-    return check_cuda(launch_gemm_nvfp4_qkv(p, t, sms, stream, pdl), "gemm_nvfp4 (QKV epilogue) launch");
-  }
-  if (use_pair_gemm()) {
+  if (gq != nullptr) p.gq = *gq;
+  if (qk != nullptr) p.qk = *qk;
+  if (use_pair_gemm(gq != nullptr)) {
     // CTA-pair kernel: half-tile boxes for B and [L2^T|L2^T], and the block
     // scales as 2D maps of 256-byte rows (8 rows = one 2 KB chunk group).
     GemmPairTmaps u;
@@ -303,8 +302,16 @@ static int gemm_nvfp4_impl(int M, int N, int K, const void* act_codes, const voi
     ok &= encode_tmap_2d(&u.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 256, sfb_rows, 256, 256, 8,
                          CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the CTA-pair GEMM");
+    if (gq != nullptr)
+      return check_cuda(launch_gemm_nvfp4_pair_gelu(p, u, stream, pdl), "gemm_nvfp4_pair (GELU-MLP epilogue) launch");
+    if (qk != nullptr)
+      return check_cuda(launch_gemm_nvfp4_pair_qkv(p, u, stream, pdl), "gemm_nvfp4_pair (QKV epilogue) launch");
     return check_cuda(launch_gemm_nvfp4_pair(p, u, stream, pdl), "gemm_nvfp4_pair launch");
   }
+  if (gq != nullptr)
+    return check_cuda(launch_gemm_nvfp4_gelu(p, t, sms, stream, pdl), "gemm_nvfp4 (GELU-MLP epilogue) launch");
+  if (qk != nullptr)
+    return check_cuda(launch_gemm_nvfp4_qkv(p, t, sms, stream, pdl), "gemm_nvfp4 (QKV epilogue) launch");
   return check_cuda(launch_gemm_nvfp4(p, t, sms, stream, pdl), "gemm_nvfp4 launch");
 }
 

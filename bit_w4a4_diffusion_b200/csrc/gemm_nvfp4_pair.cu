@@ -36,12 +36,22 @@
 // made each issue several times slower and the MMA warp, not the tensor
 // pipe, the bottleneck.
 //
-// Roles (10 warps per CTA; the MMA warp is idle in CTA 1):
+// Roles (10 warps per CTA, 12 with a fused epilogue; the MMA warp is idle in
+// CTA 1):
 //   warps 0..7  epilogue, both CTAs: warp w reads TMEM lane quarter w % 4,
-//               columns [128 (w / 4), + 128) -> bf16 -> TMA store
+//               columns [128 (w / 4), + 128) of the tile
 //   warp 8      TMA producer, both CTAs: loads into its own shared memory,
 //               completion bytes counted on CTA 0's full barrier
 //   warp 9      CTA 0: block-scale copies and MMAs for the pair
+//   warps 10,11 fused epilogues only: idle (they complete the third
+//               warpgroup, which hands registers to the epilogue warpgroups
+//               with setmaxnreg)
+// Epilogues: y = bf16(alpha D + b) through TMA stores; the GELU-MLP
+// epilogue (GELU, the down layer's NVFP4 quantizer and its low-rank
+// down-projection partials); the QKV epilogue (RMSNorm of the Q and K heads
+// and RoPE).  The fused ones are those of the single-CTA kernel
+// (gemm_nvfp4.cu), reading the whole 128-column accumulator slice of a warp
+// before releasing it.
 // Synchronisation across the pair:
 //   full[s]     CTA 0 only; CTA 0's producer arms it with both CTAs' bytes
 //   empty[s]    both CTAs; the MMA warp's commit multicasts to both
@@ -52,6 +62,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "epilogue.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -72,7 +83,14 @@ static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of S
 constexpr int EPI_WARPS = 8;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int NUM_THREADS = (MMA_WARP + 1) * 32;
+constexpr int EPI_PLAIN = 0, EPI_GELU = 1, EPI_QKV = 2;
+template <int kEpi>
+constexpr int num_threads() { return kEpi == EPI_PLAIN ? (MMA_WARP + 1) * 32 : 12 * 32; }
+// Fused epilogues: launched at 168 registers per thread; the third warpgroup
+// (producer, MMA, two idle warps) drops to 72 and the two epilogue
+// warpgroups rise to 216.
+constexpr int FUSED_LAUNCH_REGS = 168, FUSED_EPI_REGS = 216, FUSED_CTL_REGS = 72;
+static_assert(256 * FUSED_EPI_REGS + 128 * FUSED_CTL_REGS <= 384 * FUSED_LAUNCH_REGS, "register split");
 constexpr int EPI_COLS = BN / 2;                  // columns per epilogue warp
 constexpr int EPI_CHUNK = 16;                     // columns per TMA store
 constexpr int EPI_BUF_BYTES = 32 * EPI_CHUNK * 2;
@@ -95,8 +113,14 @@ struct SmemCtl {
   int abort_flag;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + sizeof(SmemCtl);
-static_assert(SMEM_BYTES <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
+// The fused epilogues keep per-tile column tables after the staging area:
+// GELU 1/lambda (fp32) + bias (bf16), QKV gamma_q | gamma_k (fp32) + bias.
+constexpr int TABLE_BYTES = BN * 4 + BN * 2;
+template <int kEpi>
+constexpr size_t smem_bytes() {
+  return 1024 + STAGES * STAGE_BYTES + EPI_BYTES + (kEpi != EPI_PLAIN ? TABLE_BYTES : 0) + sizeof(SmemCtl);
+}
+static_assert(smem_bytes<EPI_GELU>() <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 // Instruction descriptors for M = 256 (the pair), N = 256.
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
@@ -110,7 +134,8 @@ SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); 
 SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 SVDQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int kEpi>
+__global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                            const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_sfa,
@@ -119,7 +144,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES);
+  constexpr bool kGelu = kEpi == EPI_GELU, kQkv = kEpi == EPI_QKV, kFused = kEpi != EPI_PLAIN;
+  static_assert(!kFused || kGelu || kQkv, "epilogue kind");
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kFused ? TABLE_BYTES : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();     // 0: leader (issues the MMAs), 1: peer
@@ -129,6 +156,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_tiles = tiles_m * tiles_n;
   const int k_tiles = p.K / 256;
   const int slices = k_tiles + 1;  // + the low-rank slice (slice 0, no block scales)
+  // Tile schedule.  Plain and QKV epilogues: round robin over tiles numbered
+  // M-block fastest.  GELU-MLP epilogue: cluster i takes the contiguous run
+  // [i T / G, (i + 1) T / G) of tiles numbered N-block fastest, so that its
+  // consecutive tiles share an M-block and the epilogue can carry the
+  // low-rank partial of those rows from tile to tile.
+  const int t_begin = kGelu ? (int)((long long)pair * num_tiles / num_pairs) : pair;
+  const int t_end = kGelu ? (int)((long long)(pair + 1) * num_tiles / num_pairs) : num_tiles;
+  const int t_step = kGelu ? 1 : num_pairs;
+  auto tile_m0 = [&](int tile) { return (kGelu ? tile / tiles_n : tile % tiles_m) * 2 * BM + (int)rank * BM; };
+  auto tile_n0 = [&](int tile) { return (kGelu ? tile % tiles_n : tile / tiles_m) * BN; };
 
   // Every CTA initialises the same barrier set; only CTA 0's full[],
   // acc_empty and drain barriers are used.
@@ -171,7 +208,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
 
-  if (warp == PRODUCER_WARP) {
+  // ---------------------------------------------------------------- roles
+  auto role_producer = [&]() {
     {
       // ------------------------------------------------------------ producer
       // The whole warp runs the loop; one elected lane issues the copies.
@@ -181,9 +219,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       const uint64_t pol = policy_evict_last();   // every operand is re-read by other tiles
       const int kch = p.K / 64;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int m0 = (tile % tiles_m) * 2 * BM + (int)rank * BM;     // this CTA's A rows
-        const int n0 = (tile / tiles_m) * BN;                          // the tile's B rows
+      for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
+        const int m0 = tile_m0(tile);                                  // this CTA's A rows
+        const int n0 = tile_n0(tile);                                  // the tile's B rows
         const int nb = n0 + (int)rank * BN_HALF;                       // this CTA's half of them
         for (int kt = 0; kt < slices; ++kt) {
           if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
@@ -232,7 +270,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_wait(smem_u32(&ctl->full[s]), (issued_phase >> s) & 1, drain_ctx, kDevTimeoutDrain);
       }
     }
-  } else if (warp == MMA_WARP) {
+  };
+  auto role_mma = [&]() {
     if (rank == 0) {
       // ------------------------------------------------------------ MMA issuer (CTA 0)
       // The whole warp runs the loop; the same elected lane (the lowest)
@@ -241,7 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
         // Both CTAs' epilogues have taken the previous tile's accumulator.
         if (!mbar_wait_warp(smem_u32(&ctl->acc_empty), acc_phase ^ 1, wctx, kDevTimeoutMma)) {
           ok = false;
@@ -300,7 +339,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
     }
-  } else {
+  };
+  auto role_epilogue_plain = [&]() {
     // -------------------------------------------------------------- epilogue (both CTAs)
     // Warp w owns 32 rows (TMEM lane quarter w % 4) x 128 columns (half
     // w / 4) of this CTA's 128 x 256 accumulator.  It loads all of them with
@@ -313,9 +353,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * EPI_COLS);
     uint32_t acc_phase = 0;
     int chunk_seq = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
-      const int m0 = (tile % tiles_m) * 2 * BM + (int)rank * BM;
-      const int nw = (tile / tiles_m) * BN + h * EPI_COLS;   // this warp's first column
+    for (int tile = t_begin; tile < t_end; tile += t_step) {
+      const int m0 = tile_m0(tile);
+      const int nw = tile_n0(tile) + h * EPI_COLS;   // this warp's first column
       // Lane l holds the bias of columns nw + 4 l .. nw + 4 l + 3.
       uint2 bias4 = make_uint2(0, 0);
       if (p.bias != nullptr && nw + 4 * lane < p.N) bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + nw) + lane);
@@ -380,6 +420,356 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc_phase ^= 1;
     }
     if (lane == 0) bulk_wait<0>();
+  };
+  // Release of the accumulator by one epilogue warp: CTA 0's warps arrive
+  // locally, CTA 1's remotely with relaxed semantics (the TMEM loads are
+  // complete and fenced before it).
+  auto release_acc = [&]() {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t local = smem_u32(&ctl->acc_empty);
+      if (rank == 0)
+        mbar_arrive(local);
+      else
+        mbar_arrive_cluster_relaxed(mapa_shared(local, 0));
+    }
+  };
+  // Loads this warp's 32 rows x 128 columns of the accumulator, one wait.
+  auto load_acc = [&](uint32_t (&r)[4][32], int q, int half) {
+    const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * EPI_COLS);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(acc_base + 32 * i, r[i]);
+    tmem_ld_wait(r[0]);
+    reg_fence(r[1]);
+    reg_fence(r[2]);
+    reg_fence(r[3]);
+  };
+
+  auto role_epilogue_gelu = [&]() {
+    // ------------------------------------------------------ GELU-MLP epilogue
+    // Warp w: rows 32 (w mod 4) of the CTA's 128, tile columns
+    // [128 (w / 4), + 128).  Per 32-column chunk each lane (one row) forms
+    // h_hat = GELU(alpha D + b) * inv_lambda_down in fp32, quantizes its two
+    // 16-groups with the down layer's NVFP4 rule (16 bytes of codes, 2 scale
+    // bytes), and, 16 columns at a time, stages fp16(h_hat 2^-e) in a 32 x 16
+    // shared tile from which the warp accumulates its rows' share of the down
+    // layer's low-rank projection on mma.sync (lane (g, c) takes fp16
+    // columns 4c..4c+3 of the 16 as its k values, a permutation of k shared
+    // by both operands).  The tile's 1/lambda and bias columns are staged once
+    // per tile in shared memory.  Partial sums of consecutive tiles of one
+    // M-block stay in registers and go to u_work with vector reductions when
+    // the M-block changes (a separate kernel converts them to lora_act after
+    // this grid).  The eight warps share named barriers 2 and 3, so every
+    // stop decision is taken by all of them.
+    constexpr int NT = EPI_WARPS * 32;
+    const int q = warp & 3, hf = warp >> 2;
+    const int g = lane >> 2, c = lane & 3;
+    const int et = threadIdx.x;  // 0..255 over the epilogue warps
+    const GeluQuantParams& gq = p.gq;
+    const uint32_t hbase = smem_u32(epi_base + warp * 1024);
+    float* tab_inv = reinterpret_cast<float*>(epi_base + EPI_BYTES);
+    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + BN * 4);
+    const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
+    const float2 alpha2 = make_float2(p.alpha, p.alpha);
+    const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
+    uint32_t acc_phase = 0;
+    // The warp's low-rank partial of its 32 rows: rows 16t + g (+8), ranks
+    // 8j + 2c (+1).
+    float lacc[2][4][4];
+    auto zero_lacc = [&]() {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lacc[t][j][e] = 0.f;
+    };
+    auto flush_lacc = [&](int mb) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r0 = mb + 32 * q + 16 * t + g;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = 8 * j + 2 * c;
+          if (r0 < p.M) red_add_f32x2(gq.u_work + (size_t)r0 * 32 + col, lacc[t][j][0], lacc[t][j][1]);
+          if (r0 + 8 < p.M) red_add_f32x2(gq.u_work + (size_t)(r0 + 8) * 32 + col, lacc[t][j][2], lacc[t][j][3]);
+        }
+      }
+    };
+    zero_lacc();
+    int cur_m0 = -1;
+    for (int tile = t_begin; tile < t_end; tile += t_step) {
+      const int m0 = tile_m0(tile);
+      const int n0 = tile_n0(tile);
+      const int row = m0 + 32 * q + lane;
+      const bool row_ok = row < p.M;
+      // This thread's table column, fetched before the wait.
+      const float my_inv = __ldg(gq.inv_smooth + n0 + et);
+      const uint16_t my_bias = p.bias != nullptr ? __ldg(p.bias + n0 + et) : (uint16_t)0;
+      const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
+      // All epilogue threads decide together; this barrier also ends every
+      // read of the previous tile's table.
+      if (named_bar_any(2, NT, !got)) break;
+      tab_inv[et] = my_inv;
+      tab_bias[et] = my_bias;
+      asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory");
+      tc_fence_after();
+      if (m0 != cur_m0) {
+        if (cur_m0 >= 0) flush_lacc(cur_m0);
+        zero_lacc();
+        cur_m0 = m0;
+      }
+      uint32_t rb[4][32];
+      load_acc(rb, q, hf);
+      release_acc();
+      acc_phase ^= 1;
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        uint32_t(&r)[32] = rb[ii];
+        const int cl = hf * EPI_COLS + 32 * ii;  // column within the tile
+        const int n = n0 + cl;
+        // The chunk's low-rank B fragments (from L1 / L2), needed last.
+        uint2 bq[2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            bq[hh][j] =
+                __ldg(reinterpret_cast<const uint2*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 16 * hh + 4 * c));
+        // h_hat in place of the accumulator values (zero for rows past M, so
+        // their scales come out zero and they add nothing).
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const float4 i0v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8);
+          const float4 i1v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8 + 4);
+          const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + cl + 8 * k8);
+          const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+          const float il[8] = {i0v.x, i0v.y, i0v.z, i0v.w, i1v.x, i1v.y, i1v.z, i1v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 v = __ffma2_rn(alpha2,
+                                        make_float2(__uint_as_float(r[8 * k8 + 2 * j]),
+                                                    __uint_as_float(r[8 * k8 + 2 * j + 1])),
+                                        make_float2(bf16_lo(bb[j]), bf16_hi(bb[j])));
+            const float2 h = __fmul2_rn(gelu2(v), make_float2(il[2 * j], il[2 * j + 1]));
+            r[8 * k8 + 2 * j] = __float_as_uint(row_ok ? h.x : 0.f);
+            r[8 * k8 + 2 * j + 1] = __float_as_uint(row_ok ? h.y : 0.f);
+          }
+        }
+        // NVFP4 quantization of the two 16-groups (the down layer's rule).
+        uint32_t cw[4], sbs = 0;
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          float a = 0.f;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) a = fmaxf(a, fabsf(__uint_as_float(r[16 * grp + k])));
+          const uint32_t sb = cvt_e4m3(__fmul_rn(a, inv_six_s));
+          const float d = __fmul_rn(e4m3_to_f32(sb), gq.s_d);
+          uint32_t w0 = 0, w1 = 0;
+          if (d != 0.f) {
+            const float rr = __frcp_rn(d);
+            const float2 r2 = make_float2(rr, rr);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 t0 = __fmul2_rn(
+                  make_float2(__uint_as_float(r[16 * grp + 2 * k]), __uint_as_float(r[16 * grp + 2 * k + 1])), r2);
+              const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[16 * grp + 8 + 2 * k]),
+                                                       __uint_as_float(r[16 * grp + 9 + 2 * k])),
+                                           r2);
+              w0 |= cvt_e2m1x2(t0.x, t0.y) << (8 * k);
+              w1 |= cvt_e2m1x2(t1.x, t1.y) << (8 * k);
+            }
+          }
+          cw[2 * grp] = w0;
+          cw[2 * grp + 1] = w1;
+          sbs |= sb << (8 * grp);
+        }
+        if (row_ok)
+          *reinterpret_cast<uint4*>(gq.codes + (size_t)row * (p.N / 2) + n / 2) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint16_t*>(gq.scales + tiled_scale_offset(row, n / 16, p.N)) = (uint16_t)sbs;
+        // Low-rank partial, 16 columns at a time.
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+          for (int sg = 0; sg < 2; ++sg) {
+            uint32_t hv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 16 * hh + 8 * sg + 2 * k;
+              const float2 t = __fmul2_rn(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), lr2);
+              hv[k] = half2_bits(t.x, t.y);
+            }
+            st_shared_v4(hseg16(hbase, lane, sg), make_uint4(hv[0], hv[1], hv[2], hv[3]));
+          }
+          __syncwarp();
+          uint2 xa[2], xb[2];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            xa[t] = ld_shared_v2(hseg16(hbase, 16 * t + g, c >> 1) + (c & 1) * 8);
+            xb[t] = ld_shared_v2(hseg16(hbase, 16 * t + 8 + g, c >> 1) + (c & 1) * 8);
+          }
+          __syncwarp();  // every lane's loads precede the next stores
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+              mma_16816(lacc[t][j], xa[t].x, xb[t].x, xa[t].y, xb[t].y, bq[hh][j].x, bq[hh][j].y);
+        }
+      }
+    }
+    if (cur_m0 >= 0) flush_lacc(cur_m0);
+  };
+
+  auto role_epilogue_qkv = [&]() {
+    // ------------------------------------------ QKV + RMSNorm + RoPE epilogue
+    // Warp w: rows 32 (w mod 4) of the CTA's 128, head w / 4 of the tile (a
+    // 256-column tile holds two 128-feature heads).  Per lane: v = alpha D + b
+    // on packed fp32x2; for Q and K heads the mean of v^2 over the head,
+    // v * rsqrt(mean + eps) * gamma, and the rotation of each pair (2i, 2i+1)
+    // by the row's angle; bf16 out through a 1 KB shared slab per warp (32
+    // rows x 16 columns), written back as whole 32-byte row segments.  The
+    // gamma vectors (for the whole kernel) and the tile's bias columns sit in
+    // shared memory; the rotary tables are pair-major ([64][M]), so that the
+    // 32 rows of a warp read one line per pair.
+    constexpr int NT = EPI_WARPS * 32;
+    const int q = warp & 3, hf = warp >> 2;
+    const int et = threadIdx.x;  // 0..255 over the epilogue warps
+    const QkvParams& qp = p.qk;
+    const float2 alpha2 = make_float2(p.alpha, p.alpha);
+    float* tab_g = reinterpret_cast<float*>(epi_base + EPI_BYTES);                  // gamma_q | gamma_k
+    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + 1024);  // 256 bf16
+    const uint32_t slab = smem_u32(epi_base + warp * 1024);
+    tab_g[et] = et < 128 ? __ldg(qp.gamma_q + et) : __ldg(qp.gamma_k + et - 128);
+    uint32_t acc_phase = 0;
+    for (int tile = t_begin; tile < t_end; tile += t_step) {
+      const int m0 = tile_m0(tile);
+      const int n0 = tile_n0(tile);
+      const int row = m0 + 32 * q + lane;
+      const bool row_ok = row < p.M;
+      const int n = n0 + EPI_COLS * hf;  // first column of this warp's head
+      const bool head_ok = n < p.N;
+      const uint16_t my_bias = (p.bias != nullptr && n0 + et < p.N) ? __ldg(p.bias + n0 + et) : (uint16_t)0;
+      const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
+      // All epilogue threads decide together; this barrier also ends every
+      // read of the previous tile's bias columns.
+      if (named_bar_any(2, NT, !got)) break;
+      tab_bias[et] = my_bias;
+      asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory");
+      tc_fence_after();
+      uint32_t r[4][32];
+      load_acc(r, q, hf);
+      release_acc();
+      acc_phase ^= 1;
+      if (!head_ok) continue;
+      const int part = n / qp.hd;  // 0: Q, 1: K, 2: V
+      // v = alpha D + b, in place
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + EPI_COLS * hf + 32 * c4 + 8 * k8);
+          const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = 8 * k8 + 2 * j;
+            const float2 v = __ffma2_rn(alpha2, make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])),
+                                        make_float2(bf16_lo(bb[j]), bf16_hi(bb[j])));
+            r[c4][e] = __float_as_uint(v.x);
+            r[c4][e + 1] = __float_as_uint(v.y);
+          }
+        }
+      }
+      if (part < 2) {
+        float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v = make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1]));
+            ss = __ffma2_rn(v, v, ss);
+          }
+        const float ms = __fmul_rn(__fadd_rn(ss.x, ss.y), 1.0f / 128.0f);
+        const float rn = __frsqrt_rn(__fadd_rn(ms, qp.eps));
+        const float2 rn2 = make_float2(rn, rn);
+        const float* gamma = tab_g + 128 * part;
+        const float* cs = qp.rope_cos + (row_ok ? row : 0);
+        const float* sn = qp.rope_sin + (row_ok ? row : 0);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            // features 32 c4 + 8 k4 .. +7: pairs i = 16 c4 + 4 k4 .. +3
+            const float4 g0 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4);
+            const float4 g1 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4 + 4);
+            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const size_t i = (size_t)(16 * c4 + 4 * k4 + j);
+              const float cc = __ldg(cs + i * p.M), sv = __ldg(sn + i * p.M);
+              const int e = 8 * k4 + 2 * j;
+              const float2 u = __fmul2_rn(
+                  __fmul2_rn(make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])), rn2),
+                  make_float2(gg[2 * j], gg[2 * j + 1]));
+              // (a, b) -> (a cos - b sin, a sin + b cos)
+              r[c4][e] = __float_as_uint(__fmaf_rn(u.x, cc, -__fmul_rn(u.y, sv)));
+              r[c4][e + 1] = __float_as_uint(__fmaf_rn(u.x, sv, __fmul_rn(u.y, cc)));
+            }
+          }
+        }
+      }
+      // 16 columns at a time: each lane writes its row's 32 bytes into the
+      // slab (16-byte halves XOR-ed with (row / 4) mod 2: conflict-free), then
+      // lane l stores halves l and l + 32, i.e. rows l / 2 and 16 + l / 2.
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int e = 16 * (c16 & 1) + 2 * j;
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[c16 >> 1][e]), __uint_as_float(r[c16 >> 1][e + 1]));
+          w[j] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          st_shared_v4(slab + lane * 32 + ((h ^ ((lane >> 2) & 1)) << 4),
+                       make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int pc = lane + 32 * k, rr = pc >> 1, h = pc & 1;
+          const uint4 v = ld_shared_v4(slab + rr * 32 + ((h ^ ((rr >> 2) & 1)) << 4));
+          const int grow = m0 + 32 * q + rr;
+          if (grow < p.M) *reinterpret_cast<uint4*>(qp.y + (size_t)grow * p.N + n + 16 * c16 + 8 * h) = v;
+        }
+        __syncwarp();  // the slab's reads precede the next writes
+      }
+    }
+  };
+
+  if constexpr (kFused) {
+    // setmaxnreg is warpgroup-wide: the third warpgroup (producer, MMA and
+    // two idle warps) gives registers to the two epilogue warpgroups.
+    if (warp >= EPI_WARPS) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(FUSED_CTL_REGS));
+      if (warp == PRODUCER_WARP)
+        role_producer();
+      else if (warp == MMA_WARP)
+        role_mma();
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(FUSED_EPI_REGS));
+      if constexpr (kGelu)
+        role_epilogue_gelu();
+      else
+        role_epilogue_qkv();
+    }
+  } else {
+    if (warp == PRODUCER_WARP)
+      role_producer();
+    else if (warp == MMA_WARP)
+      role_mma();
+    else
+      role_epilogue_plain();
   }
 
   // Both CTAs leave together: CTA 0's MMAs write CTA 1's tensor memory, and
@@ -395,16 +785,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
+namespace {
+template <int kEpi>
+cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
   static int max_pairs = -1;
   if (max_pairs < 0) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_bytes<kEpi>());
     if (e != cudaSuccess) return e;
+    if (kEpi != EPI_PLAIN) {
+      // The epilogue warpgroups' setmaxnreg.inc waits until the third
+      // warpgroup has released enough registers: only launch if the compiled
+      // register count makes the split add up.
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, gemm_nvfp4_pair_kernel<kEpi>);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs * num_threads<kEpi>() < 256 * FUSED_EPI_REGS + 128 * FUSED_CTL_REGS)
+        return cudaErrorInvalidConfiguration;
+    }
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2);
-    q.blockDim = dim3(NUM_THREADS);
-    q.dynamicSmemBytes = SMEM_BYTES;
+    q.blockDim = dim3(num_threads<kEpi>());
+    q.dynamicSmemBytes = smem_bytes<kEpi>();
     cudaLaunchAttribute ca[1];
     ca[0].id = cudaLaunchAttributeClusterDimension;
     ca[0].val.clusterDim.x = 2;
@@ -413,7 +815,7 @@ cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps
     q.attrs = ca;
     q.numAttrs = 1;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &q);
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kEpi>, &q);
     if (e != cudaSuccess) return e;
     if (n < 1) return cudaErrorInvalidConfiguration;
     max_pairs = n;
@@ -422,8 +824,8 @@ cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.blockDim = dim3(num_threads<kEpi>());
+  cfg.dynamicSmemBytes = smem_bytes<kEpi>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -434,7 +836,22 @@ cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel, t.a, t.b, t.la, t.lb, t.y, t.sfa, t.sfb, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel<kEpi>, t.a, t.b, t.la, t.lb, t.y, t.sfa, t.sfb, p);
+}
+}  // namespace
+
+cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
+  return launch_pair_impl<EPI_PLAIN>(p, t, stream, pdl);
+}
+
+cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
+                                        bool pdl) {
+  return launch_pair_impl<EPI_GELU>(p, t, stream, pdl);
+}
+
+cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
+                                       bool pdl) {
+  return launch_pair_impl<EPI_QKV>(p, t, stream, pdl);
 }
 
 }  // namespace svdq

@@ -106,6 +106,10 @@ struct GemmPairTmaps {
 };
 
 cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl);
+cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
+                                        bool pdl);
+cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
+                                       bool pdl);
 
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;

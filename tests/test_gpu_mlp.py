@@ -120,8 +120,12 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("kernel", ["single", "pair"])
 @pytest.mark.parametrize("M,K,N", SMALL)
-def test_fused_gelu_quant_matches_oracle(M, K, N):
+def test_fused_gelu_quant_matches_oracle(M, K, N, kernel, monkeypatch):
+    """Both NVFP4 GEMM kernels carry the epilogue (the single-CTA one by
+    default)."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     B = _lib()
     up_case, down_case = _mlp_case(M, K, N)
     iu, idn, pk_u, pk_d, wu, wd = _setup(up_case, down_case)

@@ -43,7 +43,11 @@ def _ref(inp, rows, gq, gk, cos, sin, heads):
     (1, 512, 3),        # a single token, 4.5 tiles
     (512, 768, 4),
 ])
-def test_qkv_norm_rope_matches_oracle(M, K, heads):
+@pytest.mark.parametrize("kernel", ["pair", "single"])
+def test_qkv_norm_rope_matches_oracle(M, K, heads, kernel, monkeypatch):
+    """Both NVFP4 GEMM kernels carry the epilogue (the CTA-pair one by
+    default)."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     B = _lib()
     inp, pk, w, (gq, gk, cos, sin), d = _setup(M, K, heads)
     x = B.bits_to_bf16(inp.x_bits, "cuda")

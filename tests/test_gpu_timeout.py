@@ -82,8 +82,10 @@ def test_int4_gemm_wait_timeout_reports_and_recovers():
     assert_output_close(y.float().cpu().numpy(), y64, "INT4 GEMM after a timed-out call")
 
 
-def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     """The GELU-MLP kernel (eight epilogue warps that stop together)."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     import dataclasses
     import bit_w4a4_diffusion_b200 as B
     # K = 3072: thirteen K slices per tile, so that the load ring fills and
@@ -121,8 +123,10 @@ def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers():
     _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl)
 
 
-def test_qkv_gemm_wait_timeout_reports_and_recovers():
+@pytest.mark.parametrize("kernel", ["pair", "single"])
+def test_qkv_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     """The QKV + RMSNorm + RoPE kernel (eight epilogue warps that stop together)."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
     import bit_w4a4_diffusion_b200 as B
     from oracle import qkv as OQ
     M, K, heads = 640, 3072, 2       # thirteen K slices per tile, as above
