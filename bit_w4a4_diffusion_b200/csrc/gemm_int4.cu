@@ -145,8 +145,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
   const size_t mpad = (size_t)p.M_pad, npad = (size_t)p.N_pad;
 
+  // The producer and MMA loops run on whole warps and issue from one elected
+  // lane (the lowest, every time): TMA and tcgen05 instructions take
+  // uniform-register operands, which a loop run by lane 0 alone does not
+  // keep, and each issue then costs several times more.
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ producer
       int stage = 0;
       // Per stage, the last use: issued (bit), its ring parity, and whether it
@@ -157,32 +161,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
         for (int kt = 0; kt < slices; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
             ok = false;
             break;
           }
+          const bool leader = elect_one();
           if (kt == 0) {
-            // full[] completes once per use of a stage, whatever the slice
-            // kind, so that every waiter's parity follows the ring phase.
-            mbar_arrive(smem_u32(&ctl->full[stage]));
-            const uint32_t bar = smem_u32(&ctl->opnd[stage]);
-            mbar_arrive_expect_tx(bar, A8_BYTES + B8_BYTES);
-            tma_load_2d(smem_u32(a8(stage)), &tm_la, 0, m0, bar);
-            tma_load_2d(smem_u32(b8(stage)), &tm_lb, 0, n0, bar);
+            if (leader) {
+              // full[] completes once per use of a stage, whatever the slice
+              // kind, so that every waiter's parity follows the ring phase.
+              mbar_arrive(smem_u32(&ctl->full[stage]));
+              const uint32_t bar = smem_u32(&ctl->opnd[stage]);
+              mbar_arrive_expect_tx(bar, A8_BYTES + B8_BYTES);
+              tma_load_2d(smem_u32(a8(stage)), &tm_la, 0, m0, bar);
+              tma_load_2d(smem_u32(b8(stage)), &tm_lb, 0, n0, bar);
+            }
             lr_mask |= 1u << stage;
           } else {
-            const int g0 = (kt - 1) * 2;  // first 64-group of the slice
-            const uint32_t bar = smem_u32(&ctl->full[stage]);
-            mbar_arrive_expect_tx(bar, A4_BYTES + B4_BYTES + SC_BYTES);
-            tma_load_2d(smem_u32(a4(stage)), &tm_a, (kt - 1) * (KS / 2), m0, bar);
-            tma_load_2d(smem_u32(b4(stage)), &tm_b, (kt - 1) * (KS / 2), n0, bar);
-            uint16_t* sc = scl(stage);
-            for (int h = 0; h < 2; ++h) {
-              bulk_load(smem_u32(sc + h * BM), p.act_scales + (size_t)(g0 + h) * mpad + m0, BM * 2, bar);
-              bulk_load(smem_u32(sc + 2 * BM + h * BN), p.w_scales + (size_t)(g0 + h) * npad + n0, BN * 2, bar);
+            if (leader) {
+              const int g0 = (kt - 1) * 2;  // first 64-group of the slice
+              const uint32_t bar = smem_u32(&ctl->full[stage]);
+              mbar_arrive_expect_tx(bar, A4_BYTES + B4_BYTES + SC_BYTES);
+              tma_load_2d(smem_u32(a4(stage)), &tm_a, (kt - 1) * (KS / 2), m0, bar);
+              tma_load_2d(smem_u32(b4(stage)), &tm_b, (kt - 1) * (KS / 2), n0, bar);
+              uint16_t* sc = scl(stage);
+              for (int h = 0; h < 2; ++h) {
+                bulk_load(smem_u32(sc + h * BM), p.act_scales + (size_t)(g0 + h) * mpad + m0, BM * 2, bar);
+                bulk_load(smem_u32(sc + 2 * BM + h * BN), p.w_scales + (size_t)(g0 + h) * npad + n0, BN * 2, bar);
+              }
             }
             lr_mask &= ~(1u << stage);
           }
+          __syncwarp();
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
@@ -212,7 +222,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const int lb = it & 1;
         for (int kt = 0; kt < slices && ok; ++kt) {
-          if (!mbar_wait(smem_u32(&ctl->opnd[stage]), phase, wctx, kDevTimeoutMma)) {
+          if (!mbar_wait_warp(smem_u32(&ctl->opnd[stage]), phase, wctx, kDevTimeoutMma)) {
             ok = false;
             break;
           }
@@ -220,39 +230,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sa = smem_u32(a8(stage)), sb = smem_u32(b8(stage));
           if (kt == 0) {
             // Low-rank accumulator lb was last read by the epilogue two tiles ago.
-            if (it >= 2 && !mbar_wait(smem_u32(&ctl->lr_empty[lb]), ((it - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+            if (it >= 2 &&
+                !mbar_wait_warp(smem_u32(&ctl->lr_empty[lb]), ((it - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
               ok = false;
               break;
             }
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              mma_bf16(tmem + TMEM_LR + lb * BN, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16,
-                       j > 0 ? 1u : 0u);
+              for (int j = 0; j < 4; ++j)
+                mma_bf16(tmem + TMEM_LR + lb * BN, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16,
+                         j > 0 ? 1u : 0u);
+            }
+            __syncwarp();
           } else {
             for (int h = 0; h < 2; ++h, ++pcount) {
               const int pb = pcount & 1;
               if (pcount >= 2 &&
-                  !mbar_wait(smem_u32(&ctl->part_empty[pb]), ((pcount - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+                  !mbar_wait_warp(smem_u32(&ctl->part_empty[pb]), ((pcount - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
               const uint32_t d = tmem + TMEM_PART + pb * BN;
-              mma_i8(d, sw128_desc(sa + 64 * h), sw128_desc(sb + 64 * h), IDESC_I8, 0u);
-              mma_i8(d, sw128_desc(sa + 64 * h + 32), sw128_desc(sb + 64 * h + 32), IDESC_I8, 1u);
-              tc_commit(smem_u32(&ctl->part_full[pb]));
+              if (elect_one()) {
+                mma_i8(d, sw128_desc(sa + 64 * h), sw128_desc(sb + 64 * h), IDESC_I8, 0u);
+                mma_i8(d, sw128_desc(sa + 64 * h + 32), sw128_desc(sb + 64 * h + 32), IDESC_I8, 1u);
+                tc_commit(smem_u32(&ctl->part_full[pb]));
+              }
+              __syncwarp();
             }
             if (!ok) break;
           }
-          tc_commit(smem_u32(&ctl->empty[stage]));
+          if (elect_one()) tc_commit(smem_u32(&ctl->empty[stage]));
+          __syncwarp();
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      tc_commit(smem_u32(&ctl->drain));
+      // Every MMA the elected lane issued completes before TMEM is freed.
+      if (elect_one()) tc_commit(smem_u32(&ctl->drain));
+      __syncwarp();
       volatile int never = 0;
       WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
       mbar_wait(smem_u32(&ctl->drain), 0, drain_ctx, kDevTimeoutDrain);
