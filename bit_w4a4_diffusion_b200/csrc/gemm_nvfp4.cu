@@ -375,14 +375,8 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
     // Eight warps: warp w reads TMEM lane quarter w mod 4 (32 rows) and one
     // half of the tile's eight 32-column chunks (w / 4 = 0: the first four in
     // the ring order below, which include the columns shared with the other
-    // accumulator; 1: the last four).  Per chunk each lane (one row) forms
-    // h_hat = GELU(alpha D + b) * inv_lambda_down in fp32, quantizes its two
-    // 16-groups with the down layer's NVFP4 rule (16 bytes of codes, 2 scale
-    // bytes), and, 16 columns at a time, stages fp16(h_hat 2^-e) in a 32 x 16
-    // shared tile from which the warp accumulates its rows' share of the down
-    // layer's low-rank projection on mma.sync.  Lane (g, c) takes fp16
-    // columns 4c..4c+3 of the 16 as its k values (a permutation of k shared by
-    // both operands), so its A and B fragments are 8-byte loads.  The tile's
+    // accumulator; 1: the last four), each by gelu_quant_chunk (epilogue.cuh:
+    // GELU, the down layer's quantizer, its low-rank partials).  The tile's
     // 1/lambda and bias columns are staged once per tile in shared memory.
     // The partial sums of consecutive tiles of one M-block stay in registers
     // and go to u_work with vector reductions when the M-block changes (fire
@@ -400,6 +394,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
     const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
     const float2 alpha2 = make_float2(p.alpha, p.alpha);
     const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
+    const GeluLane L{tab_inv, tab_bias, alpha2, lr2, inv_six_s, hbase, lane, g, c};
     uint32_t acc_phase = 0;
     int it = 0;
     constexpr int LDC = 32;
@@ -478,95 +473,7 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
           reg_fence(rb[2]);
         }
         const int cl = chunk_col(i0 + ii) * LDC;  // column within the tile
-        const int n = n0 + cl;
-        // The chunk's low-rank B fragments (from L1 / L2), needed last.
-        uint2 bq[2][4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            bq[hh][j] =
-                __ldg(reinterpret_cast<const uint2*>(gq.l1t + (size_t)(8 * j + g) * p.N + n + 16 * hh + 4 * c));
-        // h_hat in place of the accumulator values (zero for rows past M, so
-        // their scales come out zero and they add nothing).
-#pragma unroll
-        for (int k8 = 0; k8 < 4; ++k8) {
-          const float4 i0v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8);
-          const float4 i1v = *reinterpret_cast<const float4*>(tab_inv + cl + 8 * k8 + 4);
-          const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + cl + 8 * k8);
-          const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-          const float il[8] = {i0v.x, i0v.y, i0v.z, i0v.w, i1v.x, i1v.y, i1v.z, i1v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 bias2 = make_float2(__uint_as_float(bb[j] << 16), __uint_as_float(bb[j] & 0xFFFF0000u));
-            const float2 v = __ffma2_rn(alpha2,
-                                        make_float2(__uint_as_float(r[8 * k8 + 2 * j]),
-                                                    __uint_as_float(r[8 * k8 + 2 * j + 1])),
-                                        bias2);
-            const float2 h = __fmul2_rn(gelu2(v), make_float2(il[2 * j], il[2 * j + 1]));
-            r[8 * k8 + 2 * j] = __float_as_uint(row_ok ? h.x : 0.f);
-            r[8 * k8 + 2 * j + 1] = __float_as_uint(row_ok ? h.y : 0.f);
-          }
-        }
-        // NVFP4 quantization of the two 16-groups (the down layer's rule).
-        uint32_t cw[4], sbs = 0;
-#pragma unroll
-        for (int grp = 0; grp < 2; ++grp) {
-          float a = 0.f;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) a = fmaxf(a, fabsf(__uint_as_float(r[16 * grp + k])));
-          const uint32_t sb = cvt_e4m3(__fmul_rn(a, inv_six_s));
-          const float d = __fmul_rn(e4m3_to_f32(sb), gq.s_d);
-          uint32_t w0 = 0, w1 = 0;
-          if (d != 0.f) {
-            const float rr = __frcp_rn(d);
-            const float2 r2 = make_float2(rr, rr);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 t0 = __fmul2_rn(
-                  make_float2(__uint_as_float(r[16 * grp + 2 * k]), __uint_as_float(r[16 * grp + 2 * k + 1])), r2);
-              const float2 t1 = __fmul2_rn(make_float2(__uint_as_float(r[16 * grp + 8 + 2 * k]),
-                                                       __uint_as_float(r[16 * grp + 9 + 2 * k])),
-                                           r2);
-              w0 |= cvt_e2m1x2(t0.x, t0.y) << (8 * k);
-              w1 |= cvt_e2m1x2(t1.x, t1.y) << (8 * k);
-            }
-          }
-          cw[2 * grp] = w0;
-          cw[2 * grp + 1] = w1;
-          sbs |= sb << (8 * grp);
-        }
-        if (row_ok)
-          *reinterpret_cast<uint4*>(gq.codes + (size_t)row * (p.N / 2) + n / 2) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        *reinterpret_cast<uint16_t*>(gq.scales + tiled_scale_offset(row, n / 16, p.N)) = (uint16_t)sbs;
-        // Low-rank partial, 16 columns at a time.
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-          for (int sg = 0; sg < 2; ++sg) {
-            uint32_t hv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 16 * hh + 8 * sg + 2 * k;
-              const float2 t = __fmul2_rn(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), lr2);
-              hv[k] = half2_bits(t.x, t.y);
-            }
-            st_shared_v4(hseg16(hbase, lane, sg), make_uint4(hv[0], hv[1], hv[2], hv[3]));
-          }
-          __syncwarp();
-          uint2 xa[2], xb[2];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            xa[t] = ld_shared_v2(hseg16(hbase, 16 * t + g, c >> 1) + (c & 1) * 8);
-            xb[t] = ld_shared_v2(hseg16(hbase, 16 * t + 8 + g, c >> 1) + (c & 1) * 8);
-          }
-          __syncwarp();  // every lane's loads precede the next stores
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-              mma_16816(lacc[t][j], xa[t].x, xb[t].x, xa[t].y, xb[t].y, bq[hh][j].x, bq[hh][j].y);
-        }
+        gelu_quant_chunk(r, L, gq, p.N, cl, n0 + cl, row, row_ok, lacc);
         // Refill the block just converted with the chunk three ahead.
         if (ii + NBUF < CPW) tmem_ld_32x32b_x32(acc_base + chunk_col(i0 + ii + NBUF) * LDC, r);
       }
@@ -579,14 +486,11 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
       // w / 4 of the tile (a 256-column tile holds two 128-feature heads).  A
       // lane loads its row's whole head (128 registers) before the warp
       // releases the accumulator, so the head holding the columns shared with
-      // the other accumulator is read in full first.  Per lane: v = alpha D + b
-      // on packed fp32x2; for Q and K heads the mean of v^2 over the head,
-      // v * rsqrt(mean + eps) * gamma, and the rotation of each pair (2i, 2i+1)
-      // by the row's angle; bf16 out through a 1 KB shared slab per warp (32
-      // rows x 16 columns), written back as whole 32-byte row segments.  The
-      // gamma vectors (for the whole kernel) and the tile's bias columns sit in
-      // shared memory; the rotary tables are pair-major ([64][M]), so that the
-      // 32 rows of a warp read one line per pair.
+      // the other accumulator is read in full first; qkv_head (epilogue.cuh)
+      // does the rest.  The gamma vectors (for the whole kernel) and the
+      // tile's bias columns sit in shared memory; the rotary tables are
+      // pair-major ([64][M]), so that the 32 rows of a warp read one line per
+      // pair.
       constexpr int NT = R::EPI_WARPS * 32;
       const int q = warp & 3, hf = warp >> 2;
       const int et = threadIdx.x;  // 0..255 over the epilogue warps
@@ -628,88 +532,8 @@ __global__ void __launch_bounds__(Roles<kEpi != EPI_PLAIN>::NUM_THREADS, 1)
         acc_phase ^= 1;
         if (!head_ok) continue;
         const int part = n / qp.hd;  // 0: Q, 1: K, 2: V
-        // v = alpha D + b, in place
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-#pragma unroll
-          for (int k8 = 0; k8 < 4; ++k8) {
-            const uint4 bw = *reinterpret_cast<const uint4*>(tab_bias + 128 * hf + 32 * c4 + 8 * k8);
-            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int e = 8 * k8 + 2 * j;
-              const float2 v = __ffma2_rn(alpha2, make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])),
-                                          make_float2(__uint_as_float(bb[j] << 16), __uint_as_float(bb[j] & 0xFFFF0000u)));
-              r[c4][e] = __float_as_uint(v.x);
-              r[c4][e + 1] = __float_as_uint(v.y);
-            }
-          }
-        }
-        if (part < 2) {
-          float2 ss = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 v = make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1]));
-              ss = __ffma2_rn(v, v, ss);
-            }
-          const float ms = __fmul_rn(__fadd_rn(ss.x, ss.y), 1.0f / 128.0f);
-          const float rn = __frsqrt_rn(__fadd_rn(ms, qp.eps));
-          const float2 rn2 = make_float2(rn, rn);
-          const float* gamma = tab_g + 128 * part;
-          const float* cs = qp.rope_cos + (row_ok ? row : 0);
-          const float* sn = qp.rope_sin + (row_ok ? row : 0);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              // features 32 c4 + 8 k4 .. +7: pairs i = 16 c4 + 4 k4 .. +3
-              const float4 g0 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4);
-              const float4 g1 = *reinterpret_cast<const float4*>(gamma + 32 * c4 + 8 * k4 + 4);
-              const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const size_t i = (size_t)(16 * c4 + 4 * k4 + j);
-                const float cc = __ldg(cs + i * p.M), sv = __ldg(sn + i * p.M);
-                const int e = 8 * k4 + 2 * j;
-                const float2 u = __fmul2_rn(
-                    __fmul2_rn(make_float2(__uint_as_float(r[c4][e]), __uint_as_float(r[c4][e + 1])), rn2),
-                    make_float2(gg[2 * j], gg[2 * j + 1]));
-                // (a, b) -> (a cos - b sin, a sin + b cos)
-                r[c4][e] = __float_as_uint(__fmaf_rn(u.x, cc, -__fmul_rn(u.y, sv)));
-                r[c4][e + 1] = __float_as_uint(__fmaf_rn(u.x, sv, __fmul_rn(u.y, cc)));
-              }
-            }
-          }
-        }
-        // 16 columns at a time: each lane writes its row's 32 bytes into the
-        // slab (16-byte halves XOR-ed with (row / 4) mod 2: conflict-free), then
-        // lane l stores halves l and l + 32, i.e. rows l / 2 and 16 + l / 2.
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint32_t w[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int e = 16 * (c16 & 1) + 2 * j;
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[c16 >> 1][e]), __uint_as_float(r[c16 >> 1][e + 1]));
-            w[j] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            st_shared_v4(slab + lane * 32 + ((h ^ ((lane >> 2) & 1)) << 4),
-                         make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]));
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int pc = lane + 32 * k, rr = pc >> 1, h = pc & 1;
-            const uint4 v = ld_shared_v4(slab + rr * 32 + ((h ^ ((rr >> 2) & 1)) << 4));
-            const int grow = m0 + 32 * q + rr;
-            if (grow < p.M)
-              *reinterpret_cast<uint4*>(qp.y + (size_t)grow * p.N + n + 16 * c16 + 8 * h) = v;
-          }
-          __syncwarp();  // the slab's reads precede the next writes
-        }
+        qkv_head(r, tab_bias + 128 * hf, tab_g + 128 * (part < 2 ? part : 0), alpha2, qp, part, p.M, p.N, row,
+                 row_ok, m0 + 32 * q, n, slab, lane);
       }
     } else {
     // -------------------------------------------------------------- epilogue
