@@ -407,17 +407,6 @@ SVDQ_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_byt
 }
 
 // ------------------------------------------------------------------ conversions
-// Two fp32 -> one byte of two E2M1 codes (lo goes to bits 0-3), RNE, satfinite.
-SVDQ_DEV uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .b8 b;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
-      "cvt.u32.u8 %0, b;\n\t}"
-      : "=r"(out)
-      : "f"(lo), "f"(hi));
-  return out;
-}
 // fp32 -> E4M3 byte (RNE, satfinite), returned in the low 8 bits.
 SVDQ_DEV uint32_t cvt_e4m3(float v) {
   uint16_t out;
