@@ -35,6 +35,14 @@
  *    scheduled while the previous work on the stream finishes, and waits for
  *    that work's completion before it touches global memory.  Setting the
  *    environment variable SVDQ_PDL=0 launches plainly (read at every call).
+ *  - Kernel choice (environment, read at every call; results are the same
+ *    either way, bit for bit up to the summation order of fp32 low-rank
+ *    partials): the NVFP4 GEMMs run on CTA pairs (256 x 256 tiles on two
+ *    SMs) for the plain and QKV epilogues and one CTA per 128 x 256 tile for
+ *    the GELU-MLP epilogue; SVDQ_NVFP4_GEMM_KERNEL=pair or =single forces
+ *    one kind for every call.  NVFP4 activation quantization uses the
+ *    TMA-fed kernel; SVDQ_NVFP4_QUANT_KERNEL=copy selects the per-thread-copy
+ *    kernel.
  */
 #ifndef SVDQ_H
 #define SVDQ_H
