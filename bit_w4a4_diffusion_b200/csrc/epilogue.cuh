@@ -33,20 +33,22 @@ SVDQ_DEV float ex2_approx(float x) {
 // Phi(v) = erfc/2 for v < 0 and 1 - erfc/2 for v >= 0 keeps the small
 // negative tail free of cancellation.
 // Two elements at a time on the packed fp32x2 pipe (each lane of a packed
-// operation rounds like its scalar counterpart).
+// operation rounds like its scalar counterpart).  The polynomial carries the
+// 1/2 of Phi = erfc/2 in its coefficients: halving every coefficient halves
+// each rounded step exactly, so q below is exactly half the polynomial.
 SVDQ_DEV float2 f2(float a) { return make_float2(a, a); }
 SVDQ_DEV float2 gelu2(float2 v) {
   const float2 x = __fmul2_rn(make_float2(fabsf(v.x), fabsf(v.y)), f2(0.70710678118654752f));
   const float2 den = __ffma2_rn(f2(0.3275911f), x, f2(1.0f));
   const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
-  float2 q = __ffma2_rn(f2(1.061405429f), t, f2(-1.453152027f));
-  q = __ffma2_rn(q, t, f2(1.421413741f));
-  q = __ffma2_rn(q, t, f2(-0.284496736f));
-  q = __ffma2_rn(q, t, f2(0.254829592f));
-  q = __fmul2_rn(q, t);
+  float2 q = __ffma2_rn(f2(0.5f * 1.061405429f), t, f2(0.5f * -1.453152027f));
+  q = __ffma2_rn(q, t, f2(0.5f * 1.421413741f));
+  q = __ffma2_rn(q, t, f2(0.5f * -0.284496736f));
+  q = __ffma2_rn(q, t, f2(0.5f * 0.254829592f));
+  q = __fmul2_rn(q, t);                                                       // erfc(x) / (2 exp(-x^2))
   const float2 arg = __fmul2_rn(__fmul2_rn(x, x), f2(-1.4426950408889634f));  // -x^2 log2(e)
   const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));         // exp(-x^2)
-  const float2 half_erfc = __fmul2_rn(__fmul2_rn(f2(0.5f), q), e);
+  const float2 half_erfc = __fmul2_rn(q, e);
   const float2 upper = __fadd2_rn(f2(1.0f), make_float2(-half_erfc.x, -half_erfc.y));
   const float2 phi = make_float2(v.x < 0.f ? half_erfc.x : upper.x, v.y < 0.f ? half_erfc.y : upper.y);
   return __fmul2_rn(v, phi);
