@@ -108,8 +108,27 @@ void mul_At(const uint16_t* W, const double* lam, int N, int K, const double* Y,
   });
 }
 
-// In place: the columns of V [rows, l] (row-major) become an orthonormal
-// basis of their span (Householder QR, thin Q).
+// Applies the Householder reflection I - 2 v v^T / vn (v acting on rows
+// j..rows-1) to columns c0..l-1 of X [rows, l] (row-major): per column,
+// d = 2 (v . x) / vn, then x -= d v.  The columns are independent, so all
+// the dot products are taken in one pass over the rows and all the updates
+// in a second one (contiguous rows, each column's sum still over rows in
+// increasing order).
+void reflect(double* X, int rows, int l, int j, int c0, const std::vector<double>& v, double vn) {
+  std::vector<double> d(l - c0, 0.0);
+  for (int i = j; i < rows; ++i) {
+    const double vi = v[i - j];
+    const double* xi = X + (size_t)i * l;
+    for (int c = c0; c < l; ++c) d[c - c0] += vi * xi[c];
+  }
+  for (double& t : d) t = 2.0 * t / vn;
+  for (int i = j; i < rows; ++i) {
+    const double vi = v[i - j];
+    double* xi = X + (size_t)i * l;
+    for (int c = c0; c < l; ++c) xi[c] -= d[c - c0] * vi;
+  }
+}
+
 void orthonormalize(double* V, int rows, int l) {
   std::vector<double> R((size_t)rows * l);
   std::copy(V, V + (size_t)rows * l, R.begin());
@@ -124,14 +143,7 @@ void orthonormalize(double* V, int rows, int l) {
     v[0] -= alpha;
     double vn = 0.0;
     for (double t : v) vn += t * t;
-    if (vn > 0) {
-      for (int c = j; c < l; ++c) {
-        double d = 0.0;
-        for (int i = j; i < rows; ++i) d += v[i - j] * R[(size_t)i * l + c];
-        d = 2.0 * d / vn;
-        for (int i = j; i < rows; ++i) R[(size_t)i * l + c] -= d * v[i - j];
-      }
-    }
+    if (vn > 0) reflect(R.data(), rows, l, j, j, v, vn);
     hv[j] = std::move(v);
   }
   // Q = H_0 H_1 ... H_{l-1} applied to the first l columns of the identity
@@ -142,12 +154,7 @@ void orthonormalize(double* V, int rows, int l) {
     double vn = 0.0;
     for (double t : v) vn += t * t;
     if (vn == 0) continue;
-    for (int c = 0; c < l; ++c) {
-      double d = 0.0;
-      for (int i = j; i < rows; ++i) d += v[i - j] * V[(size_t)i * l + c];
-      d = 2.0 * d / vn;
-      for (int i = j; i < rows; ++i) V[(size_t)i * l + c] -= d * v[i - j];
-    }
+    reflect(V, rows, l, j, 0, v, vn);
   }
 }
 
