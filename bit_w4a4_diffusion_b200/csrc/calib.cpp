@@ -61,23 +61,54 @@ void parallel_for(int n, F&& f) {
   for (auto& th : pool) th.join();
 }
 
+// The row-block kernels of the two products are compiled for AVX2 and for
+// the baseline x86-64 target; the dynamic loader picks one by the host CPU.
+// Both give the same bits: the host code is built without multiply-add
+// contraction, and the element order of every sum is the loop order below.
+#if defined(__x86_64__) && defined(__GNUC__) && !defined(__clang__)
+#define SVDQ_HOST_CLONES __attribute__((target_clones("avx2", "default")))
+#else
+#define SVDQ_HOST_CLONES
+#endif
+
+// P [K, l] += sum over rows n0..n1-1 of W[n, k] X[n, :] (rows in order).
+SVDQ_HOST_CLONES
+void mul_A_block(const uint16_t* W, int K, const double* X, int l, int n0, int n1, double* P) {
+  std::vector<double> wrow(K);
+  for (int n = n0; n < n1; ++n) {
+    for (int k = 0; k < K; ++k) wrow[k] = (double)bf16_to_f32(W[(size_t)n * K + k]);
+    const double* xr = X + (size_t)n * l;
+    for (int k = 0; k < K; ++k) {
+      const double w = wrow[k];
+      if (w == 0.0) continue;
+      double* pr = P + (size_t)k * l;
+      for (int c = 0; c < l; ++c) pr[c] += w * xr[c];
+    }
+  }
+}
+
+// Z [n, :] = sum over k of W[n, k] ly[k, :] (k in order), rows n0..n1-1.
+SVDQ_HOST_CLONES
+void mul_At_block(const uint16_t* W, int K, const double* ly, int l, int n0, int n1, double* Z) {
+  std::vector<double> acc(l);
+  for (int n = n0; n < n1; ++n) {
+    std::fill(acc.begin(), acc.end(), 0.0);
+    for (int k = 0; k < K; ++k) {
+      const double w = (double)bf16_to_f32(W[(size_t)n * K + k]);
+      if (w == 0.0) continue;
+      const double* yr = ly + (size_t)k * l;
+      for (int c = 0; c < l; ++c) acc[c] += w * yr[c];
+    }
+    std::copy(acc.begin(), acc.end(), Z + (size_t)n * l);
+  }
+}
+
 // Y [K, l] = A X with A = (W diag(lam))^T, W [N, K] bf16, X [N, l].
 void mul_A(const uint16_t* W, const double* lam, int N, int K, const double* X, int l, double* Y) {
   std::vector<double> part((size_t)kBlocks * K * l, 0.0);
   parallel_for(kBlocks, [&](int b) {
     const int n0 = (int)((long long)N * b / kBlocks), n1 = (int)((long long)N * (b + 1) / kBlocks);
-    double* P = part.data() + (size_t)b * K * l;
-    std::vector<double> wrow(K);
-    for (int n = n0; n < n1; ++n) {
-      for (int k = 0; k < K; ++k) wrow[k] = (double)bf16_to_f32(W[(size_t)n * K + k]);
-      const double* xr = X + (size_t)n * l;
-      for (int k = 0; k < K; ++k) {
-        const double w = wrow[k];
-        if (w == 0.0) continue;
-        double* pr = P + (size_t)k * l;
-        for (int c = 0; c < l; ++c) pr[c] += w * xr[c];
-      }
-    }
+    mul_A_block(W, K, X, l, n0, n1, part.data() + (size_t)b * K * l);
   });
   for (int k = 0; k < K; ++k)
     for (int c = 0; c < l; ++c) {
@@ -94,17 +125,7 @@ void mul_At(const uint16_t* W, const double* lam, int N, int K, const double* Y,
     for (int c = 0; c < l; ++c) ly[(size_t)k * l + c] = lam[k] * Y[(size_t)k * l + c];
   parallel_for(kBlocks, [&](int b) {
     const int n0 = (int)((long long)N * b / kBlocks), n1 = (int)((long long)N * (b + 1) / kBlocks);
-    std::vector<double> acc(l);
-    for (int n = n0; n < n1; ++n) {
-      std::fill(acc.begin(), acc.end(), 0.0);
-      for (int k = 0; k < K; ++k) {
-        const double w = (double)bf16_to_f32(W[(size_t)n * K + k]);
-        if (w == 0.0) continue;
-        const double* yr = ly.data() + (size_t)k * l;
-        for (int c = 0; c < l; ++c) acc[c] += w * yr[c];
-      }
-      std::copy(acc.begin(), acc.end(), Z + (size_t)n * l);
-    }
+    mul_At_block(W, K, ly.data(), l, n0, n1, Z);
   });
 }
 
