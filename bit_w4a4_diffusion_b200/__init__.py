@@ -41,6 +41,7 @@ def _load():
         "svdq_version": (I, []),
         "svdq_set_timeout_ns": (None, [U]),
         "svdq_get_timeout_ns": (U, []),
+        "svdq_device_status": (I, [P, I, P]),
         "svdq_act_scale_bytes": (LL, [I, I, I]),
         "svdq_weight_scale_bytes": (LL, [I, I, I]),
         "svdq_workspace_bytes": (LL, [I, I, I, I]),
@@ -124,6 +125,24 @@ def workspace_bytes(precision, M, K, rank=SVDQ_RANK):
 
 def set_timeout_ns(ns):
     lib.svdq_set_timeout_ns(int(ns))
+
+
+def device_status(clear=True, stream=None):
+    """The library's own device status word on the current device: the code
+    of a bounded wait that gave up in a call made with ``dev_status=None``
+    (0 if none since the last clear).  Waits for ``stream``."""
+    v = ctypes.c_int(0)
+    _check(lib.svdq_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    return int(v.value)
+
+
+def check_device_status(stream=None):
+    """Raise SvdqError(5) if a call made with ``dev_status=None`` timed out on
+    the device since the last check (the word is cleared either way)."""
+    code = device_status(clear=True, stream=stream)
+    if code != 0:
+        raise SvdqError(5, f"a device-side wait gave up (code {code}); outputs of the calls since the last "
+                           "check are not valid")
 
 
 def get_timeout_ns():

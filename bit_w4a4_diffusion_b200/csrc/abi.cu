@@ -98,6 +98,47 @@ int check_cuda(cudaError_t e, const char* what) {
   return SVDQ_OK;
 }
 
+// The library's own device status word: every launch whose caller passes no
+// dev_status reports a wait that gave up here, so that such a call is never
+// mistaken for a good one; svdq_device_status() reads and clears it.  A
+// file-scope device variable exists once in each context that loads this
+// module.
+__device__ int g_lib_status;
+
+struct SymbolSlot {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
+SymbolSlot g_status_slot[kMaxDevices];
+std::mutex g_status_mu;
+
+// Device address of g_lib_status in the current context.
+int lib_status_word(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  const unsigned long long ctx = svdq::current_context_id();
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  SymbolSlot& s = g_status_slot[dev];
+  if (s.ptr == nullptr || ctx == 0 || s.ctx_id != ctx) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_lib_status);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(status word): %s", cudaGetErrorString(e));
+    s.ptr = p;
+    s.ctx_id = ctx;
+  }
+  *out = static_cast<int*>(s.ptr);
+  return SVDQ_OK;
+}
+
+// The caller's status word, or the library's when the caller gives none.
+int resolve_status(int** dev_status) {
+  if (*dev_status != nullptr) return SVDQ_OK;
+  return lib_status_word(dev_status);
+}
+
 }  // namespace
 
 namespace svdq {
@@ -108,6 +149,31 @@ int record_error(int status, const char* fmt, ...) {
   vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
   va_end(ap);
   return status;
+}
+
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
 }
 
 bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
@@ -146,6 +212,25 @@ int svdq_version(void) { return SVDQ_VERSION; }
 void svdq_set_timeout_ns(unsigned long long ns) { g_timeout_ns.store(ns, std::memory_order_relaxed); }
 unsigned long long svdq_get_timeout_ns(void) { return g_timeout_ns.load(std::memory_order_relaxed); }
 
+int svdq_device_status(int* value, int clear, void* stream) {
+  if (!value) return fail(SVDQ_ERR_INVALID_ARG, "null value pointer");
+  int sms = 0;
+  if (int s = check_device(&sms)) return s;
+  int* word = nullptr;
+  if (int s = lib_status_word(&word)) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (int s = check_cuda(cudaMemcpyAsync(&host, word, sizeof(int), cudaMemcpyDeviceToHost, st), "status read"))
+    return s;
+  if (int s = check_cuda(cudaStreamSynchronize(st), "status read")) return s;
+  if (clear && host != 0) {
+    if (int s = check_cuda(cudaMemsetAsync(word, 0, sizeof(int), st), "status clear")) return s;
+    if (int s = check_cuda(cudaStreamSynchronize(st), "status clear")) return s;
+  }
+  *value = host;
+  return SVDQ_OK;
+}
+
 long long svdq_act_scale_bytes(int precision, int M, int K) {
   if (M < 0 || K <= 0) return -1;
   const int64_t mp = round_up(M > 0 ? M : 1, 256);
@@ -174,9 +259,9 @@ static bool use_copy_quantizer() {
   return v && strcmp(v, "copy") == 0;
 }
 
-int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
-                      const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,
-                      void* lora_act, void* stream) {
+static int quantize_act_impl(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
+                             const void* lora_down, float act_scale, float weight_scale, void* act_codes,
+                             void* act_scales, void* lora_act, int* dev_status, void* stream) {
   if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
     return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
   if (M <= 0 || K <= 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d must be positive", M, K);
@@ -194,6 +279,7 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
                 act_scale, weight_scale);
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
   QuantActParams p{};
   p.M = M;
   p.K = K;
@@ -225,11 +311,18 @@ int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, cons
     ok &= encode_tmap_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, lora_down, K, SVDQ_RANK, (uint64_t)K * 2, 64, 32,
                          CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the quantize kernel");
-    return check_cuda(launch_quantize_nvfp4(p, tx, tl, nullptr, svdq_timeout_ns(), static_cast<cudaStream_t>(stream), pdl_on()),
+    return check_cuda(launch_quantize_nvfp4(p, tx, tl, dev_status, svdq_timeout_ns(), static_cast<cudaStream_t>(stream), pdl_on()),
                       "quantize_nvfp4 launch");
   }
   return check_cuda(launch_quantize_act(p, precision == SVDQ_NVFP4, static_cast<cudaStream_t>(stream), pdl_on()),
                     "quantize_act launch");
+}
+
+int svdq_quantize_act(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
+                      const void* lora_down, float act_scale, float weight_scale, void* act_codes, void* act_scales,
+                      void* lora_act, void* stream) {
+  return quantize_act_impl(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, act_codes,
+                           act_scales, lora_act, nullptr, stream);
 }
 
 // NVFP4 GEMM kernel per epilogue kind.  SVDQ_NVFP4_GEMM_KERNEL=pair or
@@ -366,6 +459,7 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
   if (precision == SVDQ_NVFP4 && !(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
   if (precision == SVDQ_INT4)
     return gemm_int4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, y, dev_status,
                           static_cast<cudaStream_t>(stream), pdl_on(), sms);
@@ -387,15 +481,17 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   uint8_t* codes = ws;
   uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
   uint8_t* lora = scales + round_up(svdq_act_scale_bytes(precision, M, K), 256);
-  if (int s = svdq_quantize_act(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
-                                scales, lora, stream))
-    return s;
+  // Every argument is checked before the first launch.
   if (!w_codes || !w_scales || !lora_up || !y) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || !aligned16(y) ||
       (bias && !aligned16(bias)))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
+  if (int s = quantize_act_impl(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
+                                scales, lora, dev_status, stream))
+    return s;
   if (precision == SVDQ_INT4)
     return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
                           static_cast<cudaStream_t>(stream), pdl_on(), sms);
@@ -498,6 +594,7 @@ int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_cod
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (int s = gelu_quant_prepare(M, N, next_act_scales, work, st)) return s;
   return launch_gelu_quant(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha,
@@ -549,12 +646,13 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // The memsets go first so that quantize -> fused GEMM -> down GEMM form one
   // chain of programmatic dependent launches.
   if (int s = gelu_quant_prepare(M, N, h_scales, work, st)) return s;
-  if (int s = svdq_quantize_act(SVDQ_NVFP4, M, K, rank, x, up_inv_smooth, up_lora_down, up_act_scale,
-                                up_weight_scale, a_codes, a_scales, a_lora, stream))
+  if (int s = quantize_act_impl(SVDQ_NVFP4, M, K, rank, x, up_inv_smooth, up_lora_down, up_act_scale,
+                                up_weight_scale, a_codes, a_scales, a_lora, dev_status, stream))
     return s;
   if (int s = launch_gelu_quant(M, N, K, a_codes, a_scales, a_lora, up_w_codes, up_w_scales, up_lora_up, up_bias,
                                 up_alpha, down_inv_smooth, down_lora_down, down_act_scale, down_weight_scale, h_codes,
@@ -605,6 +703,7 @@ int svdq_w4a4_gemm_qkv_norm_rope(int M, int N, int K, int rank, const void* act_
   if (!(alpha > 0.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be positive");
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
   const QkvParams q = qkv_params(heads, gamma_q, gamma_k, rope_cos, rope_sin, y);
   return gemm_nvfp4_impl(M, N, K, act_codes, act_scales, lora_act, w_codes, w_scales, lora_up, bias, alpha, y,
                          dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms, nullptr, &q);
@@ -630,11 +729,12 @@ int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int ra
   uint8_t* codes = ws;
   uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
   uint8_t* lora = scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, K), 256);
-  if (int s = svdq_quantize_act(SVDQ_NVFP4, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
-                                scales, lora, stream))
-    return s;
   int sms = 0;
   if (int s = check_device(&sms)) return s;
+  if (int s = resolve_status(&dev_status)) return s;
+  if (int s = quantize_act_impl(SVDQ_NVFP4, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
+                                scales, lora, dev_status, stream))
+    return s;
   const QkvParams q = qkv_params(heads, gamma_q, gamma_k, rope_cos, rope_sin, y);
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms, nullptr, &q);

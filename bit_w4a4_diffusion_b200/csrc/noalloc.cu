@@ -23,27 +23,38 @@ namespace {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SVDQ_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;   // context the address belongs to
+  void* ptr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address must come
-// from cudaGetSymbolAddress, once per device, with that device current.
+// from cudaGetSymbolAddress, with that device current.  It is looked up once
+// per device and context: a device reset (or another driver context) loads
+// the module again, possibly at another address, so the cached address is
+// dropped whenever the current context's id differs from the one it was
+// taken in.
 int scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return svdq::record_error(SVDQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices)
     return svdq::record_error(SVDQ_ERR_UNSUPPORTED_DEVICE, "device index %d out of range", dev);
+  const unsigned long long ctx = svdq::current_context_id();
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (slot.ptr == nullptr || ctx == 0 || slot.ctx_id != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return svdq::record_error(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-    g_scratch_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return SVDQ_OK;
 }
 

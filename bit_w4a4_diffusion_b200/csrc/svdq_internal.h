@@ -143,6 +143,12 @@ cudaError_t launch_awq(const AwqParams& p, int num_sms, cudaStream_t stream, boo
 // Records a message for svdq_last_error() and returns `status`.
 int record_error(int status, const char* fmt, ...);
 
+// Unique id (cuCtxGetId) of the calling thread's current CUDA context, or 0
+// when no context is current or the driver cannot tell.  Ids are never
+// reused within a process, so a device address cached under one id is
+// known to be stale once the id changes (for example after cudaDeviceReset).
+unsigned long long current_context_id();
+
 // Tensor-map encoding through the driver entry point (no libcuda link needed).
 bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);

@@ -25,10 +25,14 @@
  *    before launch are returned synchronously, nothing is launched then.
  *  - Return value: an svdq_status.  svdq_last_error() gives a thread-local
  *    message for the last failure.  No C++ exception crosses this boundary.
- *  - `dev_status` (may be NULL) is a device int32 the GEMM kernels set to a
- *    nonzero code when one of their bounded internal waits gives up; the
- *    kernel then drains its copies, frees its tensor memory and exits.  The
- *    caller reads it after synchronizing and should clear it beforehand.
+ *  - `dev_status` is a device int32 the kernels set to a nonzero code when
+ *    one of their bounded internal waits gives up; the kernel then drains
+ *    its copies, frees its tensor memory and exits, and the outputs of that
+ *    call are not valid.  The caller reads it after synchronizing and should
+ *    clear it beforehand.  When the caller passes NULL (and for
+ *    svdq_quantize_act, which takes no status argument) the kernels report
+ *    to the library's own status word on the current device instead, which
+ *    svdq_device_status() reads; a timed-out call is never silent.
  *  - Device calls require a compute-capability 10.0 GPU (B200) as the
  *    current device, else SVDQ_ERR_UNSUPPORTED_DEVICE.  There is no fallback.
  *  - Every kernel is launched with programmatic dependent launch: it may be
@@ -79,6 +83,15 @@ int svdq_version(void);
  * launches made after the call, from any thread. */
 void svdq_set_timeout_ns(unsigned long long ns);
 unsigned long long svdq_get_timeout_ns(void);
+
+/* svdq_device_status: the library's own status word on the current device
+ * (the one kernels report to when their caller passed dev_status == NULL).
+ * Waits for `stream` to finish, stores the word in *value (host int; 0 when
+ * no wait has given up since the word was last cleared) and, if `clear` is
+ * nonzero, resets it to 0.  The word lives in a file-scope device variable of
+ * this library, one per device context; calls that race with kernels
+ * reporting to it on other streams see either value. */
+int svdq_device_status(int* value, int clear, void* stream);
 
 /* ------------------------------------------------------------------ layouts
  * Codes: 4-bit values, two per byte, element 2j in the low nibble of byte j
@@ -212,8 +225,9 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
  *    SVDQ_NOALLOC_SCRATCH_BYTES (e.g. M = 4096 tokens up to K = 12288);
  *    larger shapes return SVDQ_ERR_UNSUPPORTED_SHAPE with a message.
  *  - The first call on a device looks up the array's device address with
- *    cudaGetSymbolAddress (once per device, with that device current); make
- *    that first call before any stream capture.
+ *    cudaGetSymbolAddress (once per device and driver context, with that
+ *    device current; after a cudaDeviceReset the next call looks it up
+ *    again); make that first call before any stream capture.
  *  - All calls share the one array, which keeps the last call's contents;
  *    nothing in it needs to start at zero.  Calls whose kernels overlap on
  *    the GPU (different streams without ordering, or concurrent threads)

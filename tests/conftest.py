@@ -25,3 +25,20 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _library_status_word_stays_clean(request):
+    """After every GPU test, the library's own device status word (where
+    kernels called with dev_status=None report a wait that gave up) must
+    still read 0: no call in the test timed out unnoticed."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import bit_w4a4_diffusion_b200 as B
+    torch.cuda.synchronize()
+    code = B.device_status(clear=True)
+    assert code == 0, f"a kernel called without dev_status reported a timeout (code {code})"

@@ -156,6 +156,61 @@ def test_quantize_ties_and_signed_zero():
     assert np.all(lora.float().cpu().numpy() == 0)
 
 
+def _order_case_inputs(vals, K_mult=256):
+    """One long row of case values as 1/lambda (x = +-1, 0.5 then gives
+    x_hat = +-vals, vals / 2 exactly)."""
+    K = -(-vals.size // K_mult) * K_mult
+    inv = np.zeros(K, np.float32)
+    inv[:vals.size] = vals
+    x = np.zeros((3, K), np.float32)
+    x[0], x[1], x[2] = 1.0, -1.0, 0.5
+    bits, xv = wl.to_bf16(x)
+    assert np.array_equal(xv, x)
+    return K, inv, bits, xv
+
+
+@pytest.mark.parametrize("s_a", [0.0123457, 3.1e-5])
+def test_quantize_operation_order_cases(s_a):
+    """Inputs on which fl(v * fl(1/d)) and fl(v / d) give different E2M1
+    codes, or fl(a * fl(1/(6 s))) and fl(a / (6 s)) different E4M3 scale
+    bytes, under a tensor scale whose reciprocals are inexact: the device
+    codes and scales equal the oracle's (the reciprocal form) bit for bit."""
+    from tests import quant_order_cases as QC
+    B = _lib()
+    s = np.float32(s_a)
+    rows, where = QC.nvfp4_rows(s)
+    assert len(where) >= 48
+    K, inv, bits, xv = _order_case_inputs(rows.reshape(-1))
+    dev = "cuda"
+    codes, scales, lora = B.svdq_quantize_act("nvfp4", B.bits_to_bf16(bits, dev), torch.from_numpy(inv).to(dev),
+                                              torch.zeros((32, K), dtype=torch.float16, device=dev), float(s), 1.0)
+    torch.cuda.synchronize()
+    ref = O.quantize_activations("nvfp4", xv, inv, s)
+    assert np.array_equal(nibbles(codes.cpu().numpy()), ref["codes"])
+    assert np.array_equal(B.scales_to_rowmajor(scales.cpu().numpy(), 3, K), ref["scales"])
+    assert np.all(lora.float().cpu().numpy() == 0)
+
+
+def test_quantize_int4_operation_order_cases():
+    """INT4: inputs on which rint(fl(v * fl(1/sc))) and rint(fl(v / sc))
+    differ; the device codes and bf16 scales equal the oracle's."""
+    from tests import quant_order_cases as QC
+    B = _lib()
+    rows, where = QC.int4_rows(32)
+    assert len(where) >= 24
+    K, inv, bits, xv = _order_case_inputs(rows.reshape(-1))
+    dev = "cuda"
+    codes, scales, lora = B.svdq_quantize_act("int4", B.bits_to_bf16(bits, dev), torch.from_numpy(inv).to(dev),
+                                              torch.zeros((32, K), dtype=torch.bfloat16, device=dev), 1.0, 1.0)
+    torch.cuda.synchronize()
+    ref = O.quantize_activations("int4", xv, inv)
+    got = nibbles(codes.cpu().numpy()).astype(np.int16)
+    got = np.where(got >= 8, got - 16, got)
+    assert np.array_equal(got, ref["q"].astype(np.int16))
+    sc = scales.cpu().numpy().view(np.uint16).reshape(K // 64, -1)[:, :3].T
+    assert np.array_equal(wl.to_bf16(ref["sc"])[0], sc)
+
+
 FULL = ["qkv", "mlp_up", "mlp_down"]
 
 

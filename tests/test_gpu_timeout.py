@@ -158,3 +158,37 @@ def test_qkv_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
     ref = OQ.qkv_layer_f64(act, ref_pw, inp.L1, inp.L2, inp.bias, gq, gk, cos, sin, heads)
     assert_output_close(y.float().cpu().numpy(), ref, "QKV GEMM after a timed-out call")
+
+
+def test_timeout_through_the_default_binding_path_raises():
+    """A call that passes no dev_status (the binding's default) reports to
+    the library's own status word: a 1 ns wait limit makes the GEMM give up,
+    and the next status check raises SvdqError(5); the check clears the
+    word, and a normal call afterwards leaves it at 0."""
+    import bit_w4a4_diffusion_b200 as B
+    c = wl.scaled_case(wl.SVDQ_CASES["qkv"], M=640, N=2048)
+    inp = svdq_inputs(c)
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    s_a = float(inp.act_scale)
+    torch.cuda.synchronize()
+    assert B.device_status(clear=True) == 0
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_linear("nvfp4", x, w, s_a)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    with pytest.raises(B.SvdqError) as e:
+        B.check_device_status()
+    assert e.value.status == 5
+    assert B.device_status(clear=False) == 0
+    y = B.svdq_w4a4_linear("nvfp4", x, w, s_a)
+    torch.cuda.synchronize()
+    B.check_device_status()
+    ref_pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
+    y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, None)
+    assert_output_close(y.float().cpu().numpy(), y64, "layer after a timed-out call")
