@@ -118,3 +118,40 @@ def test_pack_rejects_out_of_fp16_range_factor():
     with pytest.raises(B.SvdqError):
         B.svdq_pack_weights("nvfp4", np.zeros((128, 256), np.uint16), np.ones(256, np.float32),
                             wl.to_bf16(L1)[0], np.zeros((32, 128), np.uint16))
+
+
+# The five workloads at their full weight shapes: the per-tensor scale s_w
+# depends on the whole residual, so a scaled-down shape does not stand in for
+# the full one.
+FULL = ["qkv", "mlp_up", "mlp_down", "int4_m1024"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_pack_weights_matches_oracle_full_size(name):
+    c = wl.SVDQ_CASES[name]
+    inp = svdq_inputs(c)
+    pk = B.svdq_pack_weights(c.precision, inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    ref = O.pack_weights(c.precision, inp.W, inp.lam, inp.L1, inp.L2)
+    assert np.array_equal(pk["inv_smooth"], ref["inv_lam"])
+    if c.precision == "nvfp4":
+        assert pk["weight_scale"][0] == ref["s_w"]
+        assert np.array_equal(_nibbles(pk["codes"]), ref["codes"])
+        assert np.array_equal(B.scales_to_rowmajor(pk["scales"], c.N, c.K), ref["scales"])
+    else:
+        q = _nibbles(pk["codes"]).astype(np.int8)
+        assert np.array_equal(np.where(q > 7, q - 16, q).astype(np.int8), ref["q"])
+        np_ = (c.N + 255) // 256 * 256
+        sc = pk["scales"].view(np.uint16).reshape(c.K // 64, np_)[:, :c.N].T
+        assert np.array_equal(wl.to_bf16(ref["sc"])[0], sc)
+
+
+@pytest.mark.slow
+def test_awq_pack_matches_oracle_full_size():
+    inp = wl.make_awq_inputs(1)                       # W [18432, 3072]
+    pk = B.awq_pack_weights(inp.W_bits)
+    q, sc, z = OA.awq_quantize(inp.W)
+    assert np.array_equal(_nibbles(pk["qweight"]), q)
+    assert np.array_equal(pk["scales"], wl.to_bf16(sc)[0])
+    zz = np.stack([pk["zeros"] & 0xF, pk["zeros"] >> 4], axis=-1).reshape(inp.N, -1)
+    assert np.array_equal(zz, z)
