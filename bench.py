@@ -525,24 +525,29 @@ def measure_qkv(B, wl, dev, heads=24):
             "layer_without_norm_rope_us": round(t_p, 2)}
 
 
-def block_layers(B, wl, dev, M):
+def block_layers(B, wl, dev, M, calibrate=None):
     """The linear layers of one DiT block at M tokens, hidden 3072: the
     adaptive-norm modulation (awq_w4a16, 1 row -> 6 x 3072), the fused QKV
     projection with RMSNorm and RoPE on Q and K (3072 -> 9216, 24 heads),
     the attention output projection
     (3072 -> 3072) and the GELU MLP (3072 -> 12288 -> 3072).  Attention,
     norms and residual adds are not part of this library; each layer reads
-    its own synthetic input.  Returns a function that enqueues the block
-    (out: dict of output tensors)."""
+    its own synthetic input.  `calibrate` produces each layer's smoothing,
+    low-rank factors and activation scale (the library's svdq_calibrate by
+    default).  Returns a function that enqueues the block (its `inputs`
+    attribute holds the host inputs of every layer and the workspace), the
+    dict of output tensors and the block's FLOP count."""
     import dataclasses
     import torch
-    q = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M), B.svdq_calibrate)
-    o = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, N=3072, name="attn_out"), B.svdq_calibrate)
-    iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1), B.svdq_calibrate)
-    idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05), B.svdq_calibrate)
+    cal = calibrate if calibrate is not None else B.svdq_calibrate
+    q = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M), cal)
+    o = wl.make_svdq_inputs(wl.scaled_case(wl.SVDQ_CASES["qkv"], M=M, N=3072, name="attn_out"), cal)
+    iu = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_up"], M=M), bias_std=0.1), cal)
+    idn = wl.make_svdq_inputs(dataclasses.replace(wl.scaled_case(wl.SVDQ_CASES["mlp_down"], M=M), bias_std=0.05),
+                              cal)
     a = wl.make_awq_inputs(1)
-    rq = [torch.from_numpy(np.ascontiguousarray(t.T if t.ndim == 2 else t)).to(dev)
-          for t in wl.make_rope_norm_inputs(M, 24)]
+    rope = wl.make_rope_norm_inputs(M, 24)
+    rq = [torch.from_numpy(np.ascontiguousarray(t.T if t.ndim == 2 else t)).to(dev) for t in rope]
     wq, wo, wu, wd = (B.to_device(B.svdq_pack_weights("nvfp4", i.W_bits, i.lam, i.L1_bits, i.L2_bits), dev)
                       for i in (q, o, iu, idn))
     wa = B.to_device(B.awq_pack_weights(a.W_bits), dev)
@@ -565,6 +570,8 @@ def block_layers(B, wl, dev, M):
         B.svdq_w4a4_linear("nvfp4", xs["o"], wo, float(o.act_scale), bias=bo, y=out["attn_out"], workspace=ws)
         B.svdq_w4a4_mlp_gelu(xs["u"], wu, float(iu.act_scale), wd, float(idn.act_scale), up_bias=bu,
                              down_bias=bd, y=out["mlp"], workspace=ws)
+    run.inputs = {"qkv": q, "attn_out": o, "mlp_up": iu, "mlp_down": idn, "awq": a, "rope": rope, "heads": 24,
+                  "workspace": ws}
     flop = 2.0 * M * 3072 * (9216 + 3072 + 2 * 12288) + 2.0 * 18432 * 3072
     return run, out, flop
 

@@ -79,6 +79,14 @@ def check_nvfp4_near_boundary(v_ref, s, codes, scales, delta):
     return float(np.mean(ref_codes != np.asarray(codes)))
 
 
+def identical_decision_rows(got_codes, got_scales, ref_codes, ref_scales):
+    """Rows whose NVFP4 codes [rows, K] and scale bytes [rows, K/16] equal
+    the reference's everywhere (boolean mask)."""
+    same_c = np.all(np.asarray(got_codes) == np.asarray(ref_codes), axis=1)
+    same_s = np.all(np.asarray(got_scales) == np.asarray(ref_scales), axis=1)
+    return same_c & same_s
+
+
 def svdq_inputs(case):
     """The seeded inputs of `case`, calibrated by the oracle (smoothing,
     rank-r factors, activation scale)."""

@@ -17,7 +17,8 @@ import torch
 import workloads as wl
 from oracle import mlp as OM
 from oracle import svdq as O
-from tests.helpers import check_nvfp4_near_boundary, nibbles, output_errors, svdq_inputs
+from tests.helpers import (assert_output_close, check_nvfp4_near_boundary, identical_decision_rows, nibbles,
+                           output_errors, svdq_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,13 +38,33 @@ MAX_FLIPPED = 2e-3       # fraction of codes allowed to differ from the oracle's
 # The MLP output inherits those flips: a hidden code that takes the
 # neighbouring E2M1 value moves its element by up to a third of the group's
 # max |h_hat| (the step from 4 to 6 at scale max/6), and that element's
-# column of the down layer's weight carries it into every output.  At the
-# 0.06% of flipped codes seen on the workloads below this gives a relative L2
-# difference of about 6e-3 and single outputs off by up to 0.12 rms(y) against
-# the oracle evaluated on its own codes; the bounds leave room for the allowed
-# fraction.  Exactness of the down layer itself is covered by the layer tests.
+# column of the down layer's weight carries it into every output of its row.
+# At the 0.06% of flipped codes seen on the workloads below this gives a
+# relative L2 difference of about 6e-3 and single outputs off by up to 0.12
+# rms(y) against the oracle evaluated on its own codes.  So the output is
+# checked twice:
+#  - on the rows whose hidden codes and scales all equal the oracle's, within
+#    the layer bound of every other output (helpers.assert_output_close:
+#    5e-3 relative L2, 2e-2 rms per element);
+#  - on all rows, within the bounds below, which leave room for the allowed
+#    fraction of flipped decisions.
 MLP_REL_L2_TOL = 1.5e-2
 MLP_MAX_ABS_TOL = 0.5    # in units of rms(y_ref)
+MIN_CLEAN_ROWS = 0.25    # fraction of rows with no flipped decision (tests with >= 129 rows)
+
+
+def _assert_mlp_output(y_gpu, y_ref, hc, hs, h_ref, M, N, what, rows=None):
+    """Both output checks; returns the fraction of rows with identical
+    hidden decisions."""
+    B = _lib()
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    got_c = nibbles(hc.cpu().numpy())[sel]
+    got_s = B.scales_to_rowmajor(hs.cpu().numpy(), M, N)[sel]
+    clean = identical_decision_rows(got_c, got_s, h_ref["codes"], h_ref["scales"])
+    _assert_mlp_close(y_gpu, y_ref, what)
+    if np.any(clean):
+        assert_output_close(y_gpu[clean], y_ref[clean], f"{what}, rows with identical hidden decisions")
+    return float(np.mean(clean))
 
 
 def _assert_mlp_close(y_gpu, y_ref, what):
@@ -151,8 +172,10 @@ def test_fused_gelu_quant_matches_oracle(M, K, N, kernel, monkeypatch):
     assert int(status.item()) == 0
     ref_d = O.pack_weights("nvfp4", idn.W, idn.lam, idn.L1, idn.L2)
     y64 = O.linear_f64("nvfp4", h, ref_d, idn.L1, idn.L2, idn.bias)
-    _assert_mlp_close(y.float().cpu().numpy(), y64, f"MLP {M}x{K}x{N}")
-    _assert_mlp_close(y2.float().cpu().numpy(), y64, f"one-call MLP {M}x{K}x{N}")
+    clean = _assert_mlp_output(y.float().cpu().numpy(), y64, hc, hs, h, M, N, f"MLP {M}x{K}x{N}")
+    _assert_mlp_output(y2.float().cpu().numpy(), y64, hc, hs, h, M, N, f"one-call MLP {M}x{K}x{N}")
+    if M >= 129:
+        assert clean >= MIN_CLEAN_ROWS, f"only {clean:.2f} of the rows have the oracle's hidden decisions"
     # The two paths differ only through the atomic order of the low-rank sums.
     d = (y2.float() - y.float()).abs().max().item()
     assert d <= 1e-2 * y.float().abs().max().item()
@@ -210,4 +233,7 @@ def test_mlp_full_size_sampled():
     v, h = _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl, rows=rows)
     ref_d = O.pack_weights("nvfp4", idn.W, idn.lam, idn.L1, idn.L2)
     y64 = O.linear_f64("nvfp4", h, ref_d, idn.L1, idn.L2, idn.bias)
-    _assert_mlp_close(y.float().cpu().numpy()[rows], y64, "MLP full size (sampled rows)")
+    # 12288 hidden codes per row: most rows carry a few flipped decisions,
+    # so the layer bound applies only to the sampled rows that have none.
+    _assert_mlp_output(y.float().cpu().numpy()[rows], y64, hc, hs, h, up_case.M, up_case.N,
+                       "MLP full size (sampled rows)", rows=rows)
