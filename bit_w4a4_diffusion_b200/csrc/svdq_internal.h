@@ -71,6 +71,43 @@ struct QkvParams {
   uint16_t* y;            // bf16 [M, N]
 };
 
+// The whole NVFP4 layer in one kernel (svdq_w4a4_linear on CTA pairs): the
+// GEMM's epilogue warps quantize x themselves, one unit of 128 rows x K/splits
+// columns at a time, taken in order from a global queue while their
+// accumulator is not ready; each CTA's producer waits for its 128-row block
+// to be complete before it loads that block's codes, scales and low-rank
+// activation.  The low-rank partial sums of a unit go to their own slot of
+// u_part; the last unit of a row block adds the slots in slot order (so the
+// result does not depend on which CTA ran which unit), writes lora_act and
+// raises the block's ready word.
+struct FusedQuantParams {
+  const uint16_t* x;          // bf16 [M, K]
+  const float* inv_smooth;    // fp32 [K]
+  const uint16_t* l1t;        // fp16 [32, K] (lora_down)
+  float act_scale;            // s_a
+  float lora_scale;           // 2^e / (s_a s_w): folded into lora_act
+  float lr_in_scale;          // 2^-e applied before the fp16 conversion
+  uint8_t* codes;             // [M, K/2]
+  uint8_t* scales;            // tiled e4m3, rows padded to 256
+  uint16_t* lora_act;         // bf16 [M, 64] = [hi | lo]
+  float* u_part;              // fp32 [splits][row_blocks * 128][32]
+  int* sync;                  // control words (layout below): zero at launch, left zero
+  int splits;                 // units per 128-row block (each K / splits columns)
+  int row_blocks;             // rows padded to 256, / 128
+};
+
+// Control words of the fused layer kernel, int32 offsets into
+// FusedQuantParams::sync (a 64 KiB region): the unit queue, the count of
+// CTAs that finished, per row block the count of finished units and the
+// ready word, each group on its own cache lines.
+constexpr int kSyncQueue = 0;
+constexpr int kSyncExit = 32;
+constexpr int kSyncCount = 64;
+constexpr int kSyncMaxRowBlocks = 8128;
+constexpr int kSyncReady = kSyncCount + kSyncMaxRowBlocks;
+constexpr long long kSyncBytes = 65536;
+static_assert((kSyncReady + kSyncMaxRowBlocks) * 4 <= kSyncBytes, "control words fit the region");
+
 struct GemmNvfp4Params {
   int M, N, K;
   const uint8_t* act_scales;  // tiled e4m3, rows padded to 256
@@ -81,6 +118,7 @@ struct GemmNvfp4Params {
   unsigned long long timeout_ns;
   GeluQuantParams gq;         // used by the GELU-MLP epilogue only
   QkvParams qk;               // used by the QKV epilogue only
+  FusedQuantParams fq;        // used by the fused layer kernel only
 };
 
 struct GemmTmaps {
@@ -110,6 +148,11 @@ cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPair
                                         bool pdl);
 cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                        bool pdl);
+// The fused layer kernel (p.fq set; t.a / t.sfa / t.la map the buffers the
+// kernel itself fills).  tm_x maps x [M, K] bf16 in 256 x 128 boxes, used only
+// to prefetch x into L2.
+cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
+                                    cudaStream_t stream, bool pdl);
 
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;
