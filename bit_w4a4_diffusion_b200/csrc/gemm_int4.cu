@@ -15,7 +15,16 @@
 // in its own TMEM buffer (two, ping-pong) and the epilogue warps fold it into
 // fp32 registers while the tensor core computes the next group: the epilogue
 // ALU work is what bounds this kernel (the reason the docs expect int4 to be
-// slower than nvfp4 on Blackwell).
+// slower than nvfp4 on Blackwell).  Two devices keep that work to two packed
+// FMAs per pair of elements:
+//  - a partial buffer is preset (tcgen05.st) to the int32 pattern of the
+//    float C = 1.5 * 2^23 before its group's MMAs accumulate onto it, so the
+//    exact sum P (|P| <= 64 * 7 * 7 < 2^22) comes out as the bits of the
+//    float C + P: no integer-to-float conversion;
+//  - the unpack warps stage each group's scales in fp32 together with
+//    -s_w * C (exact: an 8-bit significand times 1.5 * 2^23), so that
+//    fl(s_w * f - s_w * C) = fl(s_w * P) with f = C + P, and then
+//    acc = fl(s_a * that + acc), as before.
 //
 // Structure: persistent CTAs, 128x128 output tiles, 14 warps:
 //   warp 0      producer: TMA of the packed int4 codes and bulk copies of the
@@ -44,7 +53,11 @@ constexpr int B4_BYTES = BN * KS / 2;        // 8 KB
 constexpr int A8_BYTES = BM * KS;            // 16 KB int8 (also u' bf16 [128 x 64])
 constexpr int B8_BYTES = BN * KS;            // 16 KB int8 (also [L2^T|L2^T] bf16 [128 x 64])
 constexpr int SC_BYTES = 2 * (BM + BN) * 2;  // bf16 scales of two groups, A then B
-constexpr int STAGE_BYTES = A8_BYTES + B8_BYTES + A4_BYTES + B4_BYTES + 1024;  // scales padded to 1 KB
+constexpr int SCF_BYTES = 2 * (BM + 2 * BN) * 4;   // fp32 of two groups: s_a [128], s_w [128], -s_w C [128]
+constexpr int STAGE_BYTES = A8_BYTES + B8_BYTES + A4_BYTES + B4_BYTES + 1024 + SCF_BYTES;  // bf16 scales in 1 KB
+static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of SWIZZLE_128B");
+constexpr uint32_t kPresetBits = 0x4B400000u;    // the float 1.5 * 2^23 (ulp 1 over [2^23, 2^24))
+constexpr float kPreset = 12582912.0f;
 constexpr int UNPACK_WARPS = 4, EPI_WARPS = 8;
 constexpr int EPI_COLS = 4 * BN / EPI_WARPS;   // columns per epilogue warp (4 warps per lane quarter)
 constexpr int NHALF = EPI_COLS / 32;           // 32-column TMEM loads per warp
@@ -76,6 +89,13 @@ constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 
 SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 
+SVDQ_DEV float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
 
 // Eight packed int4 (two's complement, element 2j in the low nibble of byte
 // j) -> eight int8 in element order (two 32-bit words).
@@ -100,6 +120,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto b4 = [&](int s) { return smem + s * STAGE_BYTES + A8_BYTES + B8_BYTES + A4_BYTES; };
   auto scl = [&](int s) {
     return reinterpret_cast<uint16_t*>(smem + s * STAGE_BYTES + A8_BYTES + B8_BYTES + A4_BYTES + B4_BYTES);
+  };
+  // fp32 scales of the stage's two groups: [h][s_a 128 | s_w 128 | -s_w C 128].
+  auto scf = [&](int s) {
+    return reinterpret_cast<float*>(smem + s * STAGE_BYTES + A8_BYTES + B8_BYTES + A4_BYTES + B4_BYTES + 1024);
   };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -246,15 +270,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else {
             for (int h = 0; h < 2; ++h, ++pcount) {
               const int pb = pcount & 1;
-              if (pcount >= 2 &&
-                  !mbar_wait_warp(smem_u32(&ctl->part_empty[pb]), ((pcount - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+              // Use pcount / 2 of buffer pb: the epilogue has preset it.
+              if (!mbar_wait_warp(smem_u32(&ctl->part_empty[pb]), (pcount >> 1) & 1, wctx, kDevTimeoutMma)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
               const uint32_t d = tmem + TMEM_PART + pb * BN;
               if (elect_one()) {
-                mma_i8(d, sw128_desc(sa + 64 * h), sw128_desc(sb + 64 * h), IDESC_I8, 0u);
+                mma_i8(d, sw128_desc(sa + 64 * h), sw128_desc(sb + 64 * h), IDESC_I8, 1u);
                 mma_i8(d, sw128_desc(sa + 64 * h + 32), sw128_desc(sb + 64 * h + 32), IDESC_I8, 1u);
                 tc_commit(smem_u32(&ctl->part_full[pb]));
               }
@@ -309,6 +333,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
             fence_proxy_async_smem();
+            // The epilogue's fp32 scales of both groups: row t of A, column t of B.
+            const uint16_t* sc = scl(stage);
+            float* sf = scf(stage);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float sw = __bfloat162float(__ushort_as_bfloat16(sc[2 * BM + h * BN + t]));
+              sf[h * (BM + 2 * BN) + t] = __bfloat162float(__ushort_as_bfloat16(sc[h * BM + t]));
+              sf[h * (BM + 2 * BN) + BM + t] = sw;
+              sf[h * (BM + 2 * BN) + BM + BN + t] = __fmul_rn(sw, -kPreset);   // exact
+            }
           }
           // The stop decision is taken inside the barrier (an OR over all
           // unpack threads), so that no unpack warp can go on to the next
@@ -335,6 +369,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0, pcount = 0;
     bool ok = true;
     int it = 0;
+    // This warp's columns of partial buffer pb.
+    auto part_addr = [&](int pb) {
+      return tmem + ((uint32_t)(32 * q) << 16) + TMEM_PART + pb * BN + EPI_COLS * ch;
+    };
+    // Preset this warp's columns of buffer pb to C and hand it to the MMA warp.
+    auto preset_release = [&](int pb) {
+      const uint32_t a = part_addr(pb);
+#pragma unroll
+      for (int c8 = 0; c8 < EPI_COLS / 8; ++c8) tmem_st_32x32b_x8_fill(a + 8 * c8, kPresetBits);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->part_empty[pb]));
+    };
+    preset_release(0);
+    preset_release(1);
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
       const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
       float2 acc[EPI_COLS / 2];   // columns (2 i, 2 i + 1) of this thread's EPI_COLS
@@ -342,13 +392,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.f, 0.f);
       for (int kt = 0; kt < slices && ok; ++kt) {
         if (kt > 0) {
-          // Acquire the slice's scales (landed by bulk copy) directly.
-          const bool sc_ok = mbar_wait(smem_u32(&ctl->full[stage]), phase, wctx, kDevTimeoutEpilogue);
+          // The slice's fp32 scales, staged by the unpack warps.
+          const bool sc_ok = mbar_wait(smem_u32(&ctl->opnd[stage]), phase, wctx, kDevTimeoutEpilogue);
           if (!__all_sync(0xffffffffu, sc_ok)) {
             ok = false;
             break;
           }
-          const uint16_t* sc = scl(stage);
+          const float* sf = scf(stage);
           for (int h = 0; h < 2; ++h, ++pcount) {
             const int pb = pcount & 1;
             const bool got = mbar_wait(smem_u32(&ctl->part_full[pb]), (pcount >> 1) & 1, wctx, kDevTimeoutEpilogue);
@@ -357,37 +407,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const float sa1 = __bfloat162float(__ushort_as_bfloat16(sc[h * BM + row]));
+            const float* sfh = sf + h * (BM + 2 * BN);
+            const float sa1 = sfh[row];
             const float2 sa = make_float2(sa1, sa1);
-            const float2 unbias = make_float2(-12582912.0f, -12582912.0f);
-            const uint16_t* sw = sc + 2 * BM + h * BN + EPI_COLS * ch;
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_PART + pb * BN + EPI_COLS * ch;
+            const float* swp = sfh + BM + EPI_COLS * ch;     // s_w of this warp's columns
+            const float* ncp = swp + BN;                     // -s_w C
+            const uint32_t taddr = part_addr(pb);
+            // 16 columns per TMEM load (a 32-column block and its sixteen
+            // scale vectors would not fit beside the accumulator).
 #pragma unroll
-            for (int half = 0; half < NHALF; ++half) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(taddr + 32 * half, r);
+            for (int qc = 0; qc < EPI_COLS / 16; ++qc) {
+              uint32_t r[16];
+              tmem_ld_32x32b_x16(taddr + 16 * qc, r);
               tmem_ld_wait(r);
-              if (half == NHALF - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl->part_empty[pb]));
-              }
+              if (qc == EPI_COLS / 16 - 1) preset_release(pb);   // every column is in registers
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
-                const uint4 w8 = *reinterpret_cast<const uint4*>(sw + 32 * half + 8 * v);
-                const uint32_t ws[4] = {w8.x, w8.y, w8.z, w8.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  // Two columns at a time with the packed fp32x2 instructions:
-                  // |P| <= 64 * 7 * 7 < 2^22, exact int -> float through the
-                  // 1.5 * 2^23 bias; then acc += s_a * (s_w * P).
-                  const float2 sw2 = make_float2(__uint_as_float(ws[i] << 16), __uint_as_float(ws[i] & 0xFFFF0000u));
-                  const float2 pf = __fadd2_rn(make_float2(__int_as_float((int)r[8 * v + 2 * i] + 0x4B400000),
-                                                           __int_as_float((int)r[8 * v + 2 * i + 1] + 0x4B400000)),
-                                               unbias);
-                  const int j = 16 * half + 4 * v + i;
-                  acc[j] = __ffma2_rn(sa, __fmul2_rn(sw2, pf), acc[j]);
-                }
+                const float4 w4 = ld_shared_f4(smem_u32(swp + 16 * qc + 4 * v));
+                const float4 n4 = ld_shared_f4(smem_u32(ncp + 16 * qc + 4 * v));
+                // r holds the bits of C + P: fl(s_w (C + P) - s_w C) = fl(s_w P).
+                const float2 t0 = __ffma2_rn(make_float2(w4.x, w4.y),
+                                             make_float2(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])),
+                                             make_float2(n4.x, n4.y));
+                const float2 t1 = __ffma2_rn(make_float2(w4.z, w4.w),
+                                             make_float2(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])),
+                                             make_float2(n4.z, n4.w));
+                const int j = 8 * qc + 2 * v;
+                acc[j] = __ffma2_rn(sa, t0, acc[j]);
+                acc[j + 1] = __ffma2_rn(sa, t1, acc[j + 1]);
               }
             }
           }
@@ -407,27 +454,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int lb = it & 1;
       const int m = m0 + row;
       const uint32_t laddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_LR + lb * BN + EPI_COLS * ch;
+      // 16 columns per TMEM load, as in the group drain.
 #pragma unroll
-      for (int half = 0; half < NHALF; ++half) {
-        uint32_t l[32];
-        tmem_ld_32x32b_x32(laddr + 32 * half, l);
+      for (int qc = 0; qc < EPI_COLS / 16; ++qc) {
+        uint32_t l[16];
+        tmem_ld_32x32b_x16(laddr + 16 * qc, l);
         tmem_ld_wait(l);
-        if (half == NHALF - 1) {
+        if (qc == EPI_COLS / 16 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctl->lr_empty[lb]));
         }
-        const int nb = n0 + EPI_COLS * ch + 32 * half;
+        const int nb = n0 + EPI_COLS * ch + 16 * qc;
         if (m < p.M && nb < p.N) {
           uint16_t* yrow = p.y + (size_t)m * p.N + nb;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 2; ++v) {
             uint32_t pk[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int j = 8 * v + 2 * i;
-              float y0 = __fadd_rn(acc[16 * half + j / 2].x, __uint_as_float(l[j]));
-              float y1 = __fadd_rn(acc[16 * half + j / 2].y, __uint_as_float(l[j + 1]));
+              float y0 = __fadd_rn(acc[8 * qc + j / 2].x, __uint_as_float(l[j]));
+              float y1 = __fadd_rn(acc[8 * qc + j / 2].y, __uint_as_float(l[j + 1]));
               if (p.bias) {
                 y0 = __fadd_rn(y0, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j])));
                 y1 = __fadd_rn(y1, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j + 1])));

@@ -44,6 +44,19 @@ SVDQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase.
+SVDQ_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Same, but the thread stays suspended at most about `hint_ns` nanoseconds
 // waiting for the phase (the suspend-time hint of mbarrier.try_wait).
 SVDQ_DEV bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
@@ -131,6 +144,11 @@ SVDQ_DEV bool named_bar_any(uint32_t id, uint32_t nthreads, bool flag) {
       : "r"((uint32_t)flag), "r"(id), "r"(nthreads)
       : "memory");
   return any != 0;
+}
+
+// Named barrier `id` over `nthreads` threads.
+SVDQ_DEV void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -274,6 +292,13 @@ SVDQ_DEV void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 SVDQ_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 32 lanes x 8 consecutive 32-bit columns, all set to the same word v (a
+// wider store of one repeated value takes that many registers).
+SVDQ_DEV void tmem_st_32x32b_x8_fill(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
+               : "memory");
+}
+SVDQ_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Wait for outstanding tcgen05.ld, naming the destination registers as
 // in/out operands so that no use of them can be scheduled before the wait.
 SVDQ_DEV void tmem_ld_wait(uint32_t (&r)[32]) {
@@ -380,6 +405,16 @@ SVDQ_DEV void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uin
 // shared memory at the descriptor's offset into its own tensor memory).
 SVDQ_DEV void tmem_cp_pair_32x128_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Wait for outstanding tcgen05.ld into a 16-register block (as above).
+SVDQ_DEV void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
 }
 
 // Register-only fence: no use of r can be scheduled above this point.  Placed

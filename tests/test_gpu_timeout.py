@@ -54,7 +54,10 @@ def test_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
 
 def test_int4_gemm_wait_timeout_reports_and_recovers():
     import bit_w4a4_diffusion_b200 as B
-    c = wl.scaled_case(wl.SVDQ_CASES["int4_m1024"], M=1024)
+    # M = 4096: enough tiles per CTA that some wait outlasts the device
+    # clock's resolution (the kernel is fast enough that at M = 1024 every
+    # wait can end before the clock ticks).
+    c = wl.SVDQ_CASES["int4_m4096"]
     inp = svdq_inputs(c)
     pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
     w = B.to_device(pk)
