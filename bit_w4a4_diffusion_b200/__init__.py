@@ -45,6 +45,7 @@ def _load():
         "svdq_act_scale_bytes": (LL, [I, I, I]),
         "svdq_weight_scale_bytes": (LL, [I, I, I]),
         "svdq_workspace_bytes": (LL, [I, I, I, I]),
+        "svdq_workspace_offsets": (I, [I, I, I, I, P]),
         "svdq_scales_to_rowmajor": (I, [I, I, P, P]),
         "svdq_scales_from_rowmajor": (I, [I, I, P, P]),
         "svdq_pack_weights": (I, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
@@ -120,7 +121,18 @@ def weight_scale_bytes(precision, N, K):
 
 
 def workspace_bytes(precision, M, K, rank=SVDQ_RANK):
+    """Bytes of a layer workspace.  Its first 64 KiB are control words that
+    must be zero before the first call on it (allocate it zeroed); every call
+    leaves them zero."""
     return int(lib.svdq_workspace_bytes(_prec(precision), M, K, rank))
+
+
+def workspace_offsets(precision, M, K, rank=SVDQ_RANK):
+    """Byte offsets in a layer workspace: control words, act codes, act
+    scales, lora_act, low-rank partial sums, end."""
+    off = np.zeros(6, np.int64)
+    _check(lib.svdq_workspace_offsets(_prec(precision), M, K, rank, off.ctypes.data))
+    return [int(v) for v in off]
 
 
 def set_timeout_ns(ns):
@@ -284,7 +296,7 @@ def svdq_w4a4_linear(precision, x, w, act_scale, bias=None, y=None, workspace=No
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = torch.empty(workspace_bytes(p, M, K, rank), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(workspace_bytes(p, M, K, rank), dtype=torch.uint8, device=x.device)
     wscale = w["weight_scale_f"]
     _check(lib.svdq_w4a4_linear(p, M, N, K, rank, _ptr(x), _ptr(w["inv_smooth"]), _ptr(w["lora_down"]),
                                 float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), wscale, _ptr(w["lora_up"]),
@@ -354,7 +366,7 @@ def svdq_w4a4_mlp_gelu(x, w_up, up_act_scale, w_down, down_act_scale, up_bias=No
     if y is None:
         y = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = torch.empty(max(mlp_workspace_bytes(M, K, N, rank), 1), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(max(mlp_workspace_bytes(M, K, N, rank), 1), dtype=torch.uint8, device=x.device)
     _check(lib.svdq_w4a4_mlp_gelu(M, K, N, rank, _ptr(x), _ptr(w_up["inv_smooth"]), _ptr(w_up["lora_down"]),
                                   float(up_act_scale), _ptr(w_up["codes"]), _ptr(w_up["scales"]),
                                   w_up["weight_scale_f"], _ptr(w_up["lora_up"]), _ptr(up_bias),
@@ -392,7 +404,7 @@ def svdq_w4a4_qkv_norm_rope_linear(x, w, act_scale, heads, gamma_q, gamma_k, rop
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = torch.empty(workspace_bytes(SVDQ_NVFP4, M, K, rank), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(workspace_bytes(SVDQ_NVFP4, M, K, rank), dtype=torch.uint8, device=x.device)
     _check(lib.svdq_w4a4_qkv_norm_rope_linear(M, K, int(heads), int(head_dim), rank, _ptr(x), _ptr(w["inv_smooth"]),
                                               _ptr(w["lora_down"]), float(act_scale), _ptr(w["codes"]),
                                               _ptr(w["scales"]), w["weight_scale_f"], _ptr(w["lora_up"]), _ptr(bias),

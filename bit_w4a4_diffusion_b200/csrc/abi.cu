@@ -139,6 +139,15 @@ int resolve_status(int** dev_status) {
   return lib_status_word(dev_status);
 }
 
+// Units per 128-row block of the fused layer kernel: the largest divisor of
+// K / 256 up to 12 (each unit quantizes K / splits columns).
+int fused_splits(int K) {
+  const int kb = K / 256;
+  for (int sp = 12; sp > 1; --sp)
+    if (kb % sp == 0) return sp;
+  return 1;
+}
+
 }  // namespace
 
 namespace svdq {
@@ -241,13 +250,31 @@ long long svdq_act_scale_bytes(int precision, int M, int K) {
 
 long long svdq_weight_scale_bytes(int precision, int N, int K) { return svdq_act_scale_bytes(precision, N, K); }
 
+int svdq_workspace_offsets(int precision, int M, int K, int rank, long long* offsets) {
+  if (!offsets) return fail(SVDQ_ERR_INVALID_ARG, "null offsets");
+  if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
+    return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
+  if (M <= 0 || K <= 0 || K % 256 != 0 || rank != SVDQ_RANK)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d rank=%d", M, K, rank);
+  const long long codes = kSyncBytes;
+  const long long scales = codes + round_up((int64_t)M * (K / 2), 256);
+  const long long lora = scales + round_up(svdq_act_scale_bytes(precision, M, K), 256);
+  const long long upart = lora + round_up((int64_t)M * 2 * rank * 2, 256);
+  const long long end =
+      upart + (precision == SVDQ_NVFP4 ? round_up((int64_t)fused_splits(K) * round_up(M, 256) * 32 * 4, 256) : 0);
+  offsets[0] = 0;
+  offsets[1] = codes;
+  offsets[2] = scales;
+  offsets[3] = lora;
+  offsets[4] = upart;
+  offsets[5] = end;
+  return SVDQ_OK;
+}
+
 long long svdq_workspace_bytes(int precision, int M, int K, int rank) {
-  if (M <= 0 || K <= 0 || rank != SVDQ_RANK) return -1;
-  const long long codes = round_up((int64_t)M * (K / 2), 256);
-  const long long scales = round_up(svdq_act_scale_bytes(precision, M, K), 256);
-  const long long lora = round_up((int64_t)M * 2 * rank * 2, 256);
-  if (scales < 0) return -1;
-  return codes + scales + lora;
+  long long off[6];
+  if (svdq_workspace_offsets(precision, M, K, rank, off) != SVDQ_OK) return -1;
+  return off[5];
 }
 
 // NVFP4 activation quantizer: the TMA-fed kernel unless
@@ -467,6 +494,87 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
                          dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);
 }
 
+static bool nvfp4_scale_ok(float s);
+
+// The NVFP4 layer runs as the quantize kernel followed by the GEMM unless
+// SVDQ_LAYER_KERNEL=fused asks for the one-kernel layer (quantizer units
+// inside the CTA-pair GEMM; read at every call), which also needs the pair
+// GEMM and M within the control region's row blocks.  Measured on B200 at
+// the DiT MLP up-projection (4096 x 3072 -> 12288): 96 us one kernel against
+// 81.5 us for the two kernels, whose GEMM alone takes 72 us: the quantizer's
+// arithmetic (about 14 instructions per element) takes issue slots from the
+// GEMM's MMA warp.
+static bool use_layer_kernel(int M) {
+  const char* v = getenv("SVDQ_LAYER_KERNEL");
+  if (!(v && strcmp(v, "fused") == 0)) return false;
+  if (!use_pair_gemm(false)) return false;
+  return round_up(M, 256) / 128 <= kSyncMaxRowBlocks;
+}
+
+// x's quantized form is produced inside the GEMM kernel, in the workspace.
+static int layer_nvfp4_impl(int M, int N, int K, const void* x, const float* inv_smooth, const void* lora_down,
+                            float act_scale, const void* w_codes, const void* w_scales, float weight_scale,
+                            const void* lora_up, const void* bias, void* y, uint8_t* ws, const long long* off,
+                            int* dev_status, cudaStream_t stream, bool pdl) {
+  uint8_t* codes = ws + off[1];
+  uint8_t* scales = ws + off[2];
+  uint8_t* lora = ws + off[3];
+  GemmPairTmaps u;
+  CUtensorMap tx, tl;
+  const uint64_t sfa_rows = (uint64_t)round_up(M, 256) * (K / 16) / 256;
+  const uint64_t sfb_rows = (uint64_t)round_up(N, 256) * (K / 16) / 256;
+  bool ok = true;
+  ok &= encode_tmap_2d(&u.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, M, K / 2, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora, 2 * SVDQ_RANK, M, 2 * SVDQ_RANK * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_up, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
+                       CU_TENSOR_MAP_SWIZZLE_32B);
+  ok &= encode_tmap_2d(&u.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, 256, sfa_rows, 256, 256, 8,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_tmap_2d(&u.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_scales, 256, sfb_rows, 256, 256, 8,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, (uint64_t)K * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, lora_down, K, SVDQ_RANK, (uint64_t)K * 2, 64, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the fused layer kernel");
+  GemmNvfp4Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.act_scales = scales;
+  p.w_scales = static_cast<const uint8_t*>(w_scales);
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.alpha = act_scale * weight_scale;
+  p.dev_status = dev_status;
+  p.timeout_ns = svdq_timeout_ns();
+  // x_hat enters the fp16 down-projection as x_hat * 2^-e (as in the
+  // quantize kernel: 2688 s_a maps into [2^12, 2^13)).
+  int ex = 0;
+  frexpf(2688.0f * act_scale, &ex);
+  const int e = ex - 1 - 12;
+  FusedQuantParams& q = p.fq;
+  q.x = static_cast<const uint16_t*>(x);
+  q.inv_smooth = inv_smooth;
+  q.l1t = static_cast<const uint16_t*>(lora_down);
+  q.act_scale = act_scale;
+  q.lr_in_scale = ldexpf(1.0f, -e);
+  q.lora_scale = ldexpf(1.0f, e) / (act_scale * weight_scale);
+  q.codes = codes;
+  q.scales = scales;
+  q.lora_act = reinterpret_cast<uint16_t*>(lora);
+  q.u_part = reinterpret_cast<float*>(ws + off[4]);
+  q.sync = reinterpret_cast<int*>(ws);
+  q.splits = fused_splits(K);
+  q.row_blocks = (int)(round_up(M, 256) / 128);
+  return check_cuda(launch_layer_nvfp4_pair(p, u, tx, tl, stream, pdl), "fused layer kernel launch");
+}
+
 int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
                      const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
                      float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
@@ -477,10 +585,12 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   if (workspace_bytes < need)
     return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  long long off[6];
+  if (int s = svdq_workspace_offsets(precision, M, K, rank, off)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* codes = ws;
-  uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
-  uint8_t* lora = scales + round_up(svdq_act_scale_bytes(precision, M, K), 256);
+  uint8_t* codes = ws + off[1];
+  uint8_t* scales = ws + off[2];
+  uint8_t* lora = ws + off[3];
   // Every argument is checked before the first launch.
   if (!w_codes || !w_scales || !lora_up || !y) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || !aligned16(y) ||
@@ -489,6 +599,16 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   int sms = 0;
   if (int s = check_device(&sms)) return s;
   if (int s = resolve_status(&dev_status)) return s;
+  if (precision == SVDQ_NVFP4 && use_layer_kernel(M)) {
+    if (!x || !inv_smooth || !lora_down) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(x) || !aligned16(inv_smooth) || !aligned16(lora_down))
+      return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+    if (!nvfp4_scale_ok(act_scale) || !nvfp4_scale_ok(weight_scale))
+      return fail(SVDQ_ERR_INVALID_ARG, "NVFP4 tensor scales must lie in [2^-100, 2^100) (act %g, weight %g)",
+                  act_scale, weight_scale);
+    return layer_nvfp4_impl(M, N, K, x, inv_smooth, lora_down, act_scale, w_codes, w_scales, weight_scale, lora_up,
+                            bias, y, ws, off, dev_status, static_cast<cudaStream_t>(stream), pdl_on());
+  }
   if (int s = quantize_act_impl(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
                                 scales, lora, dev_status, stream))
     return s;
@@ -625,14 +745,19 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
   if (workspace_bytes < need)
     return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  // [the up layer's workspace | the down layer's workspace | the work buffer]
+  long long oa[6], oh[6];
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, K, rank, oa)) return s;
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, N, rank, oh)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* a_codes = ws;
-  uint8_t* a_scales = a_codes + round_up((int64_t)M * (K / 2), 256);
-  uint8_t* a_lora = a_scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, K), 256);
-  uint8_t* h_codes = a_lora + round_up((int64_t)M * 2 * rank * 2, 256);
-  uint8_t* h_scales = h_codes + round_up((int64_t)M * (N / 2), 256);
-  uint8_t* h_lora = h_scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, N), 256);
-  uint8_t* work = h_lora + round_up((int64_t)M * 2 * rank * 2, 256);
+  uint8_t* a_codes = ws + oa[1];
+  uint8_t* a_scales = ws + oa[2];
+  uint8_t* a_lora = ws + oa[3];
+  uint8_t* hws = ws + oa[5];
+  uint8_t* h_codes = hws + oh[1];
+  uint8_t* h_scales = hws + oh[2];
+  uint8_t* h_lora = hws + oh[3];
+  uint8_t* work = hws + oh[5];
   const float up_alpha = up_act_scale * up_weight_scale;
   if (int s = check_gelu_quant_args(M, N, K, rank, up_alpha, down_inv_smooth, down_lora_down, down_act_scale,
                                     down_weight_scale, h_codes, h_scales, h_lora, work,
@@ -725,10 +850,12 @@ int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int ra
   if (!w_codes || !w_scales || !lora_up) return fail(SVDQ_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || (bias && !aligned16(bias)))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  long long off[6];
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, K, rank, off)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* codes = ws;
-  uint8_t* scales = codes + round_up((int64_t)M * (K / 2), 256);
-  uint8_t* lora = scales + round_up(svdq_act_scale_bytes(SVDQ_NVFP4, M, K), 256);
+  uint8_t* codes = ws + off[1];
+  uint8_t* scales = ws + off[2];
+  uint8_t* lora = ws + off[3];
   int sms = 0;
   if (int s = check_device(&sms)) return s;
   if (int s = resolve_status(&dev_status)) return s;

@@ -63,6 +63,7 @@
 #include <cstdint>
 
 #include "epilogue.cuh"
+#include "fused_quant.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -111,16 +112,28 @@ struct SmemCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int unit;        // fused layer kernel: the quantizer unit the epilogue warps took
+  int last;        // ... and whether it was the last unit of its row block
+  uint64_t qfull[2];   // fused layer kernel: a quantizer chunk landed in buffer b
 };
 
 // The fused epilogues keep per-tile column tables after the staging area:
-// GELU 1/lambda (fp32) + bias (bf16), QKV gamma_q | gamma_k (fp32) + bias.
+// GELU 1/lambda (fp32) + bias (bf16), QKV gamma_q | gamma_k (fp32) + bias;
+// the fused layer kernel keeps its quantizer's 1/d table (256 fp32) there.
 constexpr int TABLE_BYTES = BN * 4 + BN * 2;
-template <int kEpi>
+static_assert(TABLE_BYTES >= 256 * 4, "room for the quantizer's reciprocal table");
+// The fused layer kernel keeps 4 GEMM stages and gives the fifth's room to
+// the quantizer's two chunk buffers (fused_quant.cuh).
+template <bool kQuant>
+constexpr int stages() { return kQuant ? 4 : STAGES; }
+template <int kEpi, bool kQuant>
 constexpr size_t smem_bytes() {
-  return 1024 + STAGES * STAGE_BYTES + EPI_BYTES + (kEpi != EPI_PLAIN ? TABLE_BYTES : 0) + sizeof(SmemCtl);
+  return 1024 + stages<kQuant>() * STAGE_BYTES + EPI_BYTES + (kQuant ? 2 * QC_BUF_BYTES : 0) +
+         (kEpi != EPI_PLAIN || kQuant ? TABLE_BYTES : 0) + sizeof(SmemCtl);
 }
-static_assert(smem_bytes<EPI_GELU>() <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
+static_assert(QC_BUF_BYTES % 1024 == 0 && EPI_BYTES % 1024 == 0, "chunk buffers keep the SWIZZLE_128B alignment");
+static_assert(smem_bytes<EPI_GELU, false>() <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
+static_assert(smem_bytes<EPI_PLAIN, true>() <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 // Instruction descriptors for M = 256 (the pair), N = 256.
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
@@ -134,19 +147,25 @@ SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); 
 SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 SVDQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-template <int kEpi>
+template <int kEpi, bool kQuant>
 __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                            const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_sfa,
-                           const __grid_constant__ CUtensorMap tm_sfb, const GemmNvfp4Params p) {
+                           const __grid_constant__ CUtensorMap tm_sfb, const __grid_constant__ CUtensorMap tm_x,
+                           const __grid_constant__ CUtensorMap tm_l1, const GemmNvfp4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kStages = stages<kQuant>();
   uint8_t* stage_base = smem;
-  uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
+  uint8_t* epi_base = smem + kStages * STAGE_BYTES;
   constexpr bool kGelu = kEpi == EPI_GELU, kQkv = kEpi == EPI_QKV, kFused = kEpi != EPI_PLAIN;
   static_assert(!kFused || kGelu || kQkv, "epilogue kind");
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(epi_base + EPI_BYTES + (kFused ? TABLE_BYTES : 0));
+  static_assert(!kQuant || !kFused, "the fused layer kernel has the plain epilogue");
+  // Fused layer kernel: the quantizer's chunk buffers, then its 1/d table.
+  uint8_t* q_base = epi_base + EPI_BYTES;
+  uint8_t* table_base = q_base + (kQuant ? 2 * QC_BUF_BYTES : 0);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(table_base + (kFused || kQuant ? TABLE_BYTES : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();     // 0: leader (issues the MMAs), 1: peer
@@ -161,11 +180,24 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
   // [i T / G, (i + 1) T / G) of tiles numbered N-block fastest, so that its
   // consecutive tiles share an M-block and the epilogue can carry the
   // low-rank partial of those rows from tile to tile.
+  // Fused layer kernel: round robin over tiles numbered N-block fastest, so
+  // that the first wave needs only the first M-blocks of x quantized.
+  constexpr bool kNFast = kGelu || kQuant;
   const int t_begin = kGelu ? (int)((long long)pair * num_tiles / num_pairs) : pair;
   const int t_end = kGelu ? (int)((long long)(pair + 1) * num_tiles / num_pairs) : num_tiles;
   const int t_step = kGelu ? 1 : num_pairs;
-  auto tile_m0 = [&](int tile) { return (kGelu ? tile / tiles_n : tile % tiles_m) * 2 * BM + (int)rank * BM; };
-  auto tile_n0 = [&](int tile) { return (kGelu ? tile % tiles_n : tile / tiles_m) * BN; };
+  auto tile_m0 = [&](int tile) { return (kNFast ? tile / tiles_n : tile % tiles_m) * 2 * BM + (int)rank * BM; };
+  auto tile_n0 = [&](int tile) { return (kNFast ? tile % tiles_n : tile / tiles_m) * BN; };
+  float* rcp_tab = reinterpret_cast<float*>(table_base);   // fused layer kernel only
+  if constexpr (kQuant) {
+    // The reciprocal each group's codes are scaled by, for every scale byte
+    // the quantizer can produce (0 marks an all-zero group), as in the
+    // quantize kernel.
+    if (threadIdx.x < 256) {
+      const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), p.fq.act_scale);
+      rcp_tab[threadIdx.x] = d != 0.f ? __frcp_rn(d) : 0.f;
+    }
+  }
 
   // Every CTA initialises the same barrier set; only CTA 0's full[],
   // acc_empty and drain barriers are used.
@@ -177,6 +209,8 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     mbar_init(smem_u32(&ctl->acc_full), 1);
     mbar_init(smem_u32(&ctl->acc_empty), 2 * EPI_WARPS);
     mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->qfull[0]), 1);
+    mbar_init(smem_u32(&ctl->qfull[1]), 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -200,64 +234,166 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  // Inputs produced by the preceding quantize kernel become visible here.
+  // Inputs produced by the preceding kernel become visible here.
   pdl_wait();
   // The next kernel on the stream may be scheduled from now on; it waits for
   // this grid's completion before it reads anything.
   pdl_launch_dependents();
 
   WaitCtx wctx{&ctl->abort_flag, p.dev_status, p.timeout_ns};
+  const int total_units = kQuant ? p.fq.row_blocks * p.fq.splits : 0;
+  if constexpr (kQuant) {
+    // (No L2 prefetch of x: issued at kernel entry it competes for HBM with
+    // the first units' own chunk loads, which decide when the GEMM starts.)
+    if (threadIdx.x == 0) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_l1);
+    }
+  }
 
   // ---------------------------------------------------------------- roles
   auto role_producer = [&]() {
     {
       // ------------------------------------------------------------ producer
       // The whole warp runs the loop; one elected lane issues the copies.
+      // Loads of a K slice split into the weight side (B codes and scales, or
+      // [L2^T|L2^T] for the low-rank slice) and the activation side (A codes
+      // and scales, or lora_act).  In the fused layer kernel the activation
+      // side of a 128-row block exists only once the block's ready word is
+      // set: at the first tile of a new row block the producer issues the
+      // weight side of up to kStages slices, waits for the word, then issues
+      // their activation side.
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;  // CTA 0: per stage, load outstanding and its parity
       bool ok = true;
       const uint64_t pol = policy_evict_last();   // every operand is re-read by other tiles
       const int kch = p.K / 64;
+      // Fused layer kernel: the last row block seen ready, and the ready word
+      // of the next tile's row block, read (acquire) one tile ahead so that
+      // its latency hides behind the filled ring.
+      int ready_rb = -1, ahead_rb = -1, ahead_val = 0;
+      auto stage_ptr = [&](int st) { return stage_base + st * STAGE_BYTES; };
+      auto full_addr = [&](int st) {
+        const uint32_t local = smem_u32(&ctl->full[st]);
+        return rank == 0 ? local : mapa_shared(local, 0);
+      };
+      auto issue_weight = [&](int st, int kt, int n0, int nb) {
+        uint8_t* sa = stage_ptr(st);
+        uint8_t* sb = sa + A_BYTES;
+        uint8_t* ssfb = sb + B_BYTES + SFA_BYTES;
+        const uint32_t full = full_addr(st);
+        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[st]), kt == 0 ? 2 * (A_BYTES + B_BYTES)
+                                                                              : 2 * STAGE_BYTES);
+        if (kt == 0) {
+          tma_load_2d_pair(smem_u32(sb), &tm_lb, 0, nb, full, pol);
+        } else {
+          const int kb = kt - 1;
+          tma_load_2d_pair(smem_u32(sb), &tm_b, kb * BK_BYTES, nb, full, pol);
+          // Scales: 256-byte rows of the tiled layout, 2 KB (8 rows) per
+          // 128-row block and K slice.
+          tma_load_2d_pair(smem_u32(ssfb), &tm_sfb, 0, ((n0 / 128) * kch + kb * 4) * 2, full, pol);
+          tma_load_2d_pair(smem_u32(ssfb + SFA_BYTES), &tm_sfb, 0, ((n0 / 128 + 1) * kch + kb * 4) * 2, full, pol);
+        }
+      };
+      auto issue_act = [&](int st, int kt, int m0) {
+        uint8_t* sa = stage_ptr(st);
+        uint8_t* ssfa = sa + A_BYTES + B_BYTES;
+        const uint32_t full = full_addr(st);
+        if (kt == 0) {
+          tma_load_2d_pair(smem_u32(sa), &tm_la, 0, m0, full, pol);
+        } else {
+          const int kb = kt - 1;
+          tma_load_2d_pair(smem_u32(sa), &tm_a, kb * BK_BYTES, m0, full, pol);
+          tma_load_2d_pair(smem_u32(ssfa), &tm_sfa, 0, ((m0 / 128) * kch + kb * 4) * 2, full, pol);
+        }
+      };
+      auto advance = [&]() {
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      };
       for (int tile = t_begin; tile < t_end && ok; tile += t_step) {
         const int m0 = tile_m0(tile);                                  // this CTA's A rows
         const int n0 = tile_n0(tile);                                  // the tile's B rows
         const int nb = n0 + (int)rank * BN_HALF;                       // this CTA's half of them
-        for (int kt = 0; kt < slices; ++kt) {
+        int kt0 = 0;
+        if (kQuant && (m0 >> 7) != ready_rb) {
+          const int rb = m0 >> 7;
+          int v = (rb == ahead_rb) ? ahead_val : 0;
+          if (v == 0) {
+            if (lane == 0) v = ld_acquire_gpu(p.fq.sync + kSyncReady + rb);
+            v = __shfl_sync(0xffffffffu, v, 0);
+          }
+          if (v != 0) {
+            // The rows were written through the generic proxy by other SMs;
+            // the TMA reads them through the async proxy.
+            fence_proxy_async_global();
+            ready_rb = rb;
+          }
+        }
+        if (kQuant && tile + t_step < t_end) {
+          const int nrb = tile_m0(tile + t_step) >> 7;
+          if (nrb != ahead_rb && nrb != ready_rb) {
+            int v = 0;
+            if (lane == 0) v = ld_acquire_gpu(p.fq.sync + kSyncReady + nrb);
+            ahead_val = __shfl_sync(0xffffffffu, v, 0);
+            ahead_rb = nrb;
+          }
+        }
+        if (kQuant && (m0 >> 7) != ready_rb) {
+          // Not ready yet: the weight side of the first slices, then the wait.
+          const int rb = m0 >> 7;
+          const int P = slices < kStages ? slices : kStages;
+          const int st0 = stage;
+          for (int kt = 0; kt < P; ++kt) {
+            if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
+              ok = false;
+              break;
+            }
+            if (elect_one()) issue_weight(stage, kt, n0, nb);
+            __syncwarp();
+            advance();
+          }
+          if (!ok) {
+            // The weight side of the stages issued so far is in flight; their
+            // barriers complete only with the activation side, which the
+            // drain below does not wait for: give it the (possibly stale)
+            // rows so that every armed stage completes.
+            kt0 = -1;
+          } else {
+            bool got = true;
+            if (lane == 0) got = flag_wait(p.fq.sync + kSyncReady + rb, wctx, kDevTimeoutProducer);
+            got = __shfl_sync(0xffffffffu, got, 0) != 0;
+            // The rows were written through the generic proxy by other SMs;
+            // the TMA reads them through the async proxy.
+            fence_proxy_async_global();
+            if (!got) ok = false;
+            ready_rb = got ? rb : ready_rb;
+            kt0 = P;
+          }
+          // Activation side of the stages just armed (also after a timeout,
+          // so that no armed barrier is left without its bytes).
+          const int armed = kt0 < 0 ? (stage - st0 + kStages) % kStages : P;   // < kStages when the loop broke
+          if (elect_one())
+            for (int i = 0; i < armed; ++i) issue_act((st0 + i) % kStages, i, m0);
+          __syncwarp();
+          if (!ok) break;
+        }
+        for (int kt = kt0; kt < slices; ++kt) {
           if (!mbar_wait_warp(smem_u32(&ctl->empty[stage]), phase ^ 1, wctx, kDevTimeoutProducer)) {
             ok = false;
             break;
           }
-          uint8_t* sa = stage_base + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          uint8_t* ssfa = sb + B_BYTES;
-          uint8_t* ssfb = ssfa + SFA_BYTES;
-          const uint32_t full_local = smem_u32(&ctl->full[stage]);
-          const uint32_t full = rank == 0 ? full_local : mapa_shared(full_local, 0);
-          if (!elect_one()) {
-          } else if (kt == 0) {
-            if (rank == 0) mbar_arrive_expect_tx(full_local, 2 * (A_BYTES + B_BYTES));
-            tma_load_2d_pair(smem_u32(sa), &tm_la, 0, m0, full, pol);
-            tma_load_2d_pair(smem_u32(sb), &tm_lb, 0, nb, full, pol);
-          } else {
-            const int kb = kt - 1;
-            if (rank == 0) mbar_arrive_expect_tx(full_local, 2 * STAGE_BYTES);
-            tma_load_2d_pair(smem_u32(sa), &tm_a, kb * BK_BYTES, m0, full, pol);
-            tma_load_2d_pair(smem_u32(sb), &tm_b, kb * BK_BYTES, nb, full, pol);
-            // Scales: 256-byte rows of the tiled layout, 2 KB (8 rows) per
-            // 128-row block and K slice.
-            tma_load_2d_pair(smem_u32(ssfa), &tm_sfa, 0, ((m0 / 128) * kch + kb * 4) * 2, full, pol);
-            tma_load_2d_pair(smem_u32(ssfb), &tm_sfb, 0, ((n0 / 128) * kch + kb * 4) * 2, full, pol);
-            tma_load_2d_pair(smem_u32(ssfb + SFA_BYTES), &tm_sfb, 0, ((n0 / 128 + 1) * kch + kb * 4) * 2, full,
-                             pol);
+          if (elect_one()) {
+            issue_weight(stage, kt, n0, nb);
+            issue_act(stage, kt, m0);
           }
           __syncwarp();
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          advance();
         }
       }
       // CTA 0 never leaves with copies in flight into the pair's shared
@@ -265,7 +401,7 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
       if (rank == 0) {
         volatile int never = 0;
         WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < kStages; ++s)
           if (issued_mask & (1u << s))
             mbar_wait(smem_u32(&ctl->full[s]), (issued_phase >> s) & 1, drain_ctx, kDevTimeoutDrain);
       }
@@ -322,7 +458,7 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
           // copies and MMAs reading it are done.
           if (leader) tc_commit_pair_mc(smem_u32(&ctl->empty[stage]), PAIR_MASK);
           __syncwarp();
-          if (++stage == STAGES) {
+          if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
@@ -353,14 +489,146 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     const uint32_t acc_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * EPI_COLS);
     uint32_t acc_phase = 0;
     int chunk_seq = 0;
+    // Fused layer kernel: quantizer units (fused_quant.cuh) while this CTA's
+    // accumulator is not ready (until_acc) or until the queue is empty.  All
+    // eight warps take every decision together (named barriers 2 and 3), so
+    // that they work on one unit at a time and stay in step.  A unit's
+    // 64-column chunks come through the two TMA-fed buffers: thread 0 issues
+    // the first two when it takes the unit and chunk c + 2 once every warp is
+    // done with chunk c.  A CTA's first unit is unit blockIdx.x, known without
+    // the queue, so that its loads start at kernel entry; the queue hands out
+    // units from gridDim.x on.
+    constexpr int NT = EPI_WARPS * 32;
+    bool units_left = kQuant;
+    const int span = p.K / (kQuant ? p.fq.splits : 1), nch = span / QC_COLS;
+    uint32_t qseq = 0;                       // chunk loads issued by this CTA so far (uniform)
+    uint32_t q_issued_mask = 0, q_issued_phase = 0;   // thread 0: last load per buffer, for the drain
+    const uint32_t qb0 = smem_u32(q_base);
+    auto issue_chunk = [&](int rb, int k, uint32_t seq) {   // thread 0
+      const int b = (int)(seq & 1);
+      const uint32_t buf = qb0 + (uint32_t)b * QC_BUF_BYTES;
+      const uint32_t bar = smem_u32(&ctl->qfull[b]);
+      fence_proxy_async_smem();   // the buffer's generic reads (chunk seq - 2) before the async-proxy writes
+      mbar_arrive_expect_tx(bar, QC_TX_BYTES);
+      tma_load_2d(buf, &tm_x, k, rb * 128, bar);
+      tma_load_2d(buf + QC_X_BYTES, &tm_l1, k, 0, bar);
+      bulk_load(buf + QC_X_BYTES + QC_L_BYTES, p.fq.inv_smooth + k, QC_I_BYTES, bar);
+      q_issued_mask |= 1u << b;
+      q_issued_phase = (q_issued_phase & ~(1u << b)) | (((seq >> 1) & 1) << b);
+    };
+    const float q_inv_six_s = kQuant ? __frcp_rn(__fmul_rn(6.0f, p.fq.act_scale)) : 0.f;
+    const float2 q_xs2 = make_float2(p.fq.lr_in_scale, p.fq.lr_in_scale);
+    auto issue_first_chunks = [&](int u) {   // thread 0
+      if (u < total_units) {
+        const int rb = u / p.fq.splits, k0 = (u - rb * p.fq.splits) * span;
+        issue_chunk(rb, k0, qseq);
+        if (nch > 1) issue_chunk(rb, k0 + QC_COLS, qseq + 1);
+      }
+    };
+    bool first_unit = kQuant;
+    if (kQuant && threadIdx.x == 0) {
+      ctl->unit = (int)blockIdx.x;
+      issue_first_chunks((int)blockIdx.x);
+    }
+    auto run_units = [&](bool until_acc) {
+      while (units_left) {
+        const bool stop = until_acc && mbar_test_wait(smem_u32(&ctl->acc_full), acc_phase);
+        if (named_bar_any(2, NT, stop || *reinterpret_cast<volatile int*>(&ctl->abort_flag) != 0)) return;
+        if (threadIdx.x == 0 && !first_unit) {
+          const int u = atomicAdd(p.fq.sync + kSyncQueue, 1) + (int)gridDim.x;
+          ctl->unit = u;
+          issue_first_chunks(u);
+        }
+        first_unit = false;
+        named_bar_sync(3, NT);
+        const int u = ctl->unit;
+        if (u >= total_units) {
+          units_left = false;
+          return;
+        }
+        const int rb = u / p.fq.splits, sp = u - rb * p.fq.splits, k0 = sp * span;
+        // The lane's rows within the unit: 16 w + perm(g), + 8.
+        const int g = lane >> 2, c = lane & 3;
+        const int r0 = 16 * warp + quant_perm(g);
+        QuantLane L;
+        L.row0 = rb * 128 + r0;
+        L.K = p.K;
+        L.c = c;
+        L.ok0 = L.row0 < p.M;
+        L.ok1 = L.row0 + 8 < p.M;
+        L.code0 = p.fq.codes + (size_t)L.row0 * (p.K / 2) + 4 * c;
+        L.xr0 = nullptr;
+        L.inv = nullptr;
+        L.l1t = nullptr;
+        float qacc[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) qacc[j][e] = 0.f;
+        bool ok = true;
+        for (int ch = 0; ch < nch; ++ch) {
+          const uint32_t seq = qseq + ch;
+          const int b = (int)(seq & 1);
+          const bool got = mbar_wait(smem_u32(&ctl->qfull[b]), (seq >> 1) & 1, wctx, kDevTimeoutEpilogue);
+          if (named_bar_any(3, NT, !got)) {
+            ok = false;
+            break;
+          }
+          quant_chunk(qb0 + (uint32_t)b * QC_BUF_BYTES, k0 + QC_COLS * ch, L, r0, rcp_tab, q_inv_six_s, q_xs2,
+                      p.fq.scales, qacc);
+          named_bar_sync(3, NT);   // every warp is done with buffer b
+          if (threadIdx.x == 0 && ch + 2 < nch) issue_chunk(rb, k0 + QC_COLS * (ch + 2), seq + 2);
+        }
+        if (!ok) {
+          units_left = false;
+          return;
+        }
+        qseq += nch;
+        // The warp's low-rank partial: row r0 (r0 + 8), ranks 8 j + c and 8 j + 4 + c.
+        {
+          const size_t mp = (size_t)p.fq.row_blocks * 128;
+          float* u0 = p.fq.u_part + ((size_t)sp * mp + L.row0) * 32 + c;
+          float* u1 = u0 + 8 * 32;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            __stcg(u0 + 8 * j, qacc[j][0]);
+            __stcg(u0 + 8 * j + 4, qacc[j][1]);
+            __stcg(u1 + 8 * j, qacc[j][2]);
+            __stcg(u1 + 8 * j + 4, qacc[j][3]);
+          }
+        }
+        // Publish the unit: the barrier orders every thread's stores before
+        // thread 0's fence and count (one count per unit).
+        named_bar_sync(3, NT);
+        if (threadIdx.x == 0)
+          ctl->last = atomic_add_acq_rel_gpu(p.fq.sync + kSyncCount + rb, 1) == p.fq.splits - 1;
+        named_bar_sync(3, NT);
+        if (ctl->last) {
+          // The last unit of the block: every other unit's partials are
+          // visible (thread 0 saw all counts, then fenced, then the barrier);
+          // add them up, then raise the block's ready word.
+          reduce_row_block(p.fq, p.M, rb, threadIdx.x);
+          named_bar_sync(3, NT);
+          if (threadIdx.x == 0) {
+            fence_proxy_async_global();
+            st_release_gpu(p.fq.sync + kSyncReady + rb, 1);
+          }
+        }
+      }
+    };
     for (int tile = t_begin; tile < t_end; tile += t_step) {
+      if constexpr (kQuant) run_units(true);
       const int m0 = tile_m0(tile);
       const int nw = tile_n0(tile) + h * EPI_COLS;   // this warp's first column
       // Lane l holds the bias of columns nw + 4 l .. nw + 4 l + 3.
       uint2 bias4 = make_uint2(0, 0);
       if (p.bias != nullptr && nw + 4 * lane < p.N) bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + nw) + lane);
       const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
-      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
+      if constexpr (kQuant) {
+        if (named_bar_any(2, NT, !got)) break;   // decided by all eight warps
+      } else {
+        if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform decision
+      }
       tc_fence_after();
       uint32_t r[4][32];
 #pragma unroll
@@ -419,6 +687,18 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
       }
       acc_phase ^= 1;
     }
+    // Units nobody has taken yet (other CTAs' tiles may wait for them).
+    if constexpr (kQuant) {
+      run_units(false);
+      // Never leave with a chunk load in flight into shared memory.
+      if (threadIdx.x == 0) {
+        volatile int never = 0;
+        WaitCtx drain_ctx{&never, p.dev_status, kDrainLimitNs};
+        for (int b = 0; b < 2; ++b)
+          if (q_issued_mask & (1u << b))
+            mbar_wait(smem_u32(&ctl->qfull[b]), (q_issued_phase >> b) & 1, drain_ctx, kDevTimeoutDrain);
+      }
+    }
     if (lane == 0) bulk_wait<0>();
   };
   // Release of the accumulator by one epilogue warp: CTA 0's warps arrive
@@ -463,8 +743,8 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     const int et = threadIdx.x;  // 0..255 over the epilogue warps
     const GeluQuantParams& gq = p.gq;
     const uint32_t hbase = smem_u32(epi_base + warp * 1024);
-    float* tab_inv = reinterpret_cast<float*>(epi_base + EPI_BYTES);
-    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + BN * 4);
+    float* tab_inv = reinterpret_cast<float*>(table_base);
+    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(table_base + BN * 4);
     const float2 lr2 = make_float2(gq.lr_in_scale, gq.lr_in_scale);
     const float2 alpha2 = make_float2(p.alpha, p.alpha);
     const float inv_six_s = __frcp_rn(__fmul_rn(6.0f, gq.s_d));
@@ -543,8 +823,8 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     const int et = threadIdx.x;  // 0..255 over the epilogue warps
     const QkvParams& qp = p.qk;
     const float2 alpha2 = make_float2(p.alpha, p.alpha);
-    float* tab_g = reinterpret_cast<float*>(epi_base + EPI_BYTES);                  // gamma_q | gamma_k
-    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(epi_base + EPI_BYTES + 1024);  // 256 bf16
+    float* tab_g = reinterpret_cast<float*>(table_base);                  // gamma_q | gamma_k
+    uint16_t* tab_bias = reinterpret_cast<uint16_t*>(table_base + 1024);  // 256 bf16
     const uint32_t slab = smem_u32(epi_base + warp * 1024);
     tab_g[et] = et < 128 ? __ldg(qp.gamma_q + et) : __ldg(qp.gamma_k + et - 128);
     uint32_t acc_phase = 0;
@@ -608,24 +888,45 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, TMEM_COLS);
   }
+  if constexpr (kQuant) {
+    // Every role of this CTA is done with the control words.  The last CTA
+    // to get here returns them to zero for the next call on this workspace
+    // (the next kernel on the stream reads them only after this grid ends).
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.fq.sync + kSyncExit, 1) == (int)gridDim.x - 1) {
+        __threadfence();
+        int* sy = p.fq.sync;
+        sy[kSyncQueue] = 0;
+        sy[kSyncExit] = 0;
+        for (int rb = 0; rb < p.fq.row_blocks; ++rb) {
+          sy[kSyncCount + rb] = 0;
+          sy[kSyncReady + rb] = 0;
+        }
+        __threadfence();
+      }
+    }
+  }
 }
 
 }  // namespace
 
 namespace {
-template <int kEpi>
-cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
+template <int kEpi, bool kQuant>
+cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
+                             const CUtensorMap& tm_l1, cudaStream_t stream, bool pdl) {
   static int max_pairs = -1;
+  auto kernel = gemm_nvfp4_pair_kernel<kEpi, kQuant>;
+  constexpr size_t smem = smem_bytes<kEpi, kQuant>();
   if (max_pairs < 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<kEpi>());
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (kEpi != EPI_PLAIN) {
       // The epilogue warpgroups' setmaxnreg.inc waits until the third
       // warpgroup has released enough registers: only launch if the compiled
       // register count makes the split add up.
       cudaFuncAttributes fa;
-      e = cudaFuncGetAttributes(&fa, gemm_nvfp4_pair_kernel<kEpi>);
+      e = cudaFuncGetAttributes(&fa, kernel);
       if (e != cudaSuccess) return e;
       if (fa.numRegs * num_threads<kEpi>() < 256 * FUSED_EPI_REGS + 128 * FUSED_CTL_REGS)
         return cudaErrorInvalidConfiguration;
@@ -633,7 +934,7 @@ cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, c
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2);
     q.blockDim = dim3(num_threads<kEpi>());
-    q.dynamicSmemBytes = smem_bytes<kEpi>();
+    q.dynamicSmemBytes = smem;
     cudaLaunchAttribute ca[1];
     ca[0].id = cudaLaunchAttributeClusterDimension;
     ca[0].val.clusterDim.x = 2;
@@ -642,7 +943,7 @@ cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, c
     q.attrs = ca;
     q.numAttrs = 1;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kEpi>, &q);
+    e = cudaOccupancyMaxActiveClusters(&n, kernel, &q);
     if (e != cudaSuccess) return e;
     if (n < 1) return cudaErrorInvalidConfiguration;
     max_pairs = n;
@@ -652,7 +953,7 @@ cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(num_threads<kEpi>());
-  cfg.dynamicSmemBytes = smem_bytes<kEpi>();
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -663,22 +964,27 @@ cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, c
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel<kEpi>, t.a, t.b, t.la, t.lb, t.y, t.sfa, t.sfb, p);
+  return cudaLaunchKernelEx(&cfg, kernel, t.a, t.b, t.la, t.lb, t.y, t.sfa, t.sfb, tm_x, tm_l1, p);
 }
 }  // namespace
 
 cudaError_t launch_gemm_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
-  return launch_pair_impl<EPI_PLAIN>(p, t, stream, pdl);
+  return launch_pair_impl<EPI_PLAIN, false>(p, t, t.a, t.a, stream, pdl);
 }
 
 cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                         bool pdl) {
-  return launch_pair_impl<EPI_GELU>(p, t, stream, pdl);
+  return launch_pair_impl<EPI_GELU, false>(p, t, t.a, t.a, stream, pdl);
 }
 
 cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                        bool pdl) {
-  return launch_pair_impl<EPI_QKV>(p, t, stream, pdl);
+  return launch_pair_impl<EPI_QKV, false>(p, t, t.a, t.a, stream, pdl);
+}
+
+cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
+                                    const CUtensorMap& tm_l1, cudaStream_t stream, bool pdl) {
+  return launch_pair_impl<EPI_PLAIN, true>(p, t, tm_x, tm_l1, stream, pdl);
 }
 
 }  // namespace svdq

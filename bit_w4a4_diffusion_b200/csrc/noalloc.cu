@@ -81,9 +81,11 @@ int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const
                               M, K, need, (long long)SVDQ_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   if (int s = scratch_for_current_device(&scratch)) return s;
-  // Nothing in the scratch has to start at zero: the quantize kernel writes
-  // every byte the GEMM then reads (all code rows < M, every scale row up to
-  // the 256-row padding, every low-rank row < M) before the GEMM starts.
+  // The scratch's first 64 KiB are the layer kernel's control words: zero
+  // when the module is loaded (a file-scope device array starts zeroed) and
+  // left zero by every call.  The rest needs no clearing: the layer writes
+  // every byte it reads (code rows < M, scale rows up to the 256-row padding,
+  // low-rank rows < M and the partial sums) before reading it.
   return svdq_w4a4_linear(precision, M, N, K, rank, x, inv_smooth, lora_down, act_scale, w_codes, w_scales,
                           weight_scale, lora_up, bias, y, scratch, need, dev_status, stream);
 }

@@ -149,10 +149,10 @@ cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPair
 cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                        bool pdl);
 // The fused layer kernel (p.fq set; t.a / t.sfa / t.la map the buffers the
-// kernel itself fills).  tm_x maps x [M, K] bf16 in 256 x 128 boxes, used only
-// to prefetch x into L2.
+// kernel itself fills).  tm_x maps x [M, K] bf16 and tm_l1 L1^T [32, K] fp16,
+// both in 64 x 128 / 64 x 32 SWIZZLE_128B boxes (the quantizer's chunks).
 cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
-                                    cudaStream_t stream, bool pdl);
+                                    const CUtensorMap& tm_l1, cudaStream_t stream, bool pdl);
 
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;

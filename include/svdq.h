@@ -198,13 +198,35 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
                    const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
                    const void* bias, float alpha, void* y, int* dev_status, void* stream);
 
-/* svdq_w4a4_linear: the whole layer, svdq_quantize_act then svdq_w4a4_gemm on
- * `stream` (the GEMM is launched with programmatic dependent launch so its
- * prologue overlaps the quantize kernel's tail).  `workspace` is a device
- * buffer of at least svdq_workspace_bytes(precision, M, K, rank) bytes that
- * holds the quantized activations between the two kernels; calls that share
- * a workspace must not overlap in time. */
+/* svdq_w4a4_linear: the whole layer, y = svdq_w4a4_gemm(svdq_quantize_act(x))
+ * on `stream`: svdq_quantize_act then svdq_w4a4_gemm, the GEMM launched with
+ * programmatic dependent launch so that its prologue overlaps the quantize
+ * kernel's tail.
+ *  - With SVDQ_LAYER_KERNEL=fused in the environment (read at every call;
+ *    NVFP4 on the CTA-pair GEMM only): ONE kernel, whose epilogue warps
+ *    quantize x themselves, 128 rows x K/splits columns at a time (splits =
+ *    the largest divisor of K/256 up to 12), while their accumulator is not
+ *    ready; each CTA's TMA producer waits (bounded, like every wait of the
+ *    library) for its 128 rows to be complete.  Codes and scales are those
+ *    of svdq_quantize_act bit for bit; the low-rank activation sums the same
+ *    products in a different (fixed) order, so y can differ from quantize +
+ *    gemm in its last bits, and is the same on every run.  It is slower than
+ *    the two kernels on B200 (the quantizer's arithmetic competes with the
+ *    GEMM's MMA issue) and kept for comparison.
+ * `workspace` is a device buffer of at least svdq_workspace_bytes(precision,
+ * M, K, rank) bytes laid out as svdq_workspace_offsets gives:
+ *   [0]  control words of the one-kernel layer, a fixed 64 KiB at offset 0;
+ *        when that layer runs they MUST BE ZERO before the first call on a
+ *        workspace (e.g. a workspace from cudaMemset or torch.zeros), and
+ *        every call leaves them zero again (the kernel's last CTA resets
+ *        them), so a workspace can be reused by calls of any shape without
+ *        clearing it; the two-kernel path does not touch them;
+ *   [1]  act codes [M, K/2];  [2] act scales;  [3] lora_act bf16 [M, 2r];
+ *   [4]  fp32 low-rank partial sums (NVFP4); [5] the end (= the size).
+ * Calls that share a workspace must not overlap in time.  The one-kernel
+ * layer takes M up to 1040384 (larger M runs as two kernels). */
 long long svdq_workspace_bytes(int precision, int M, int K, int rank);
+int svdq_workspace_offsets(int precision, int M, int K, int rank, long long* offsets /* [6], host */);
 int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
                      const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
                      float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
@@ -222,16 +244,19 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
  * GPU that loads the library, until the process exits.  It never calls
  * cudaMalloc, cudaFree or any allocating routine.
  *  - Limit: svdq_workspace_bytes(precision, M, K, rank) must not exceed
- *    SVDQ_NOALLOC_SCRATCH_BYTES (e.g. M = 4096 tokens up to K = 12288);
- *    larger shapes return SVDQ_ERR_UNSUPPORTED_SHAPE with a message.
+ *    SVDQ_NOALLOC_SCRATCH_BYTES (e.g. M = 4096 tokens up to K = 9216, or
+ *    2048 tokens up to K = 12288, for NVFP4); larger shapes return
+ *    SVDQ_ERR_UNSUPPORTED_SHAPE with a message.
  *  - The first call on a device looks up the array's device address with
  *    cudaGetSymbolAddress (once per device and driver context, with that
  *    device current; after a cudaDeviceReset the next call looks it up
  *    again); make that first call before any stream capture.
- *  - All calls share the one array, which keeps the last call's contents;
- *    nothing in it needs to start at zero.  Calls whose kernels overlap on
- *    the GPU (different streams without ordering, or concurrent threads)
- *    race on it: order them on one stream.
+ *  - All calls share the one array, which keeps the last call's contents.
+ *    Its first 64 KiB are the layer kernel's control words (see
+ *    svdq_w4a4_linear): the array is zero when the module loads and every
+ *    call leaves those words zero again.  Calls whose kernels overlap on the
+ *    GPU (different streams without ordering, or concurrent threads) race on
+ *    it: order them on one stream.
  * Arguments, layouts and errors are those of svdq_w4a4_linear without the
  * workspace pair. */
 #define SVDQ_NOALLOC_SCRATCH_BYTES (32ll << 20)

@@ -58,10 +58,6 @@ def test_block_graph_and_pdl_invariance(M):
     del g
 
 
-def _ru(a, b):
-    return (a + b - 1) // b * b
-
-
 @pytest.mark.parametrize("M", [129, 384])
 def test_block_layers_match_oracle(M):
     """Each layer of the graph-replayed block against its oracle: the AWQ
@@ -116,12 +112,12 @@ def test_block_layers_match_oracle(M):
     pk_u = B.svdq_pack_weights("nvfp4", iu.W_bits, iu.lam, iu.L1_bits, iu.L2_bits)
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
     ws = inp["workspace"]
-    off = _ru(M * K // 2, 256) + _ru(B.act_scale_bytes("nvfp4", M, K), 256) + _ru(M * 128, 256)
-    hc = ws[off:off + M * N // 2].view(M, N // 2)
-    off += _ru(M * N // 2, 256)
-    hs = ws[off:off + B.act_scale_bytes("nvfp4", M, N)]
-    off += _ru(B.act_scale_bytes("nvfp4", M, N), 256)
-    hl = ws[off:off + M * 128].view(torch.bfloat16).view(M, 64)
+    # the MLP's workspace: [up layer's | down layer's | work]
+    base = B.workspace_bytes("nvfp4", M, K)
+    oh = B.workspace_offsets("nvfp4", M, N)
+    hc = ws[base + oh[1]:base + oh[1] + M * N // 2].view(M, N // 2)
+    hs = ws[base + oh[2]:base + oh[2] + B.act_scale_bytes("nvfp4", M, N)]
+    hl = ws[base + oh[3]:base + oh[3] + M * 128].view(torch.bfloat16).view(M, 64)
     v, h = _check_hidden(iu, idn, pk_u, pk_d, hc, hs, hl)
     ref_d = O.pack_weights("nvfp4", idn.W, idn.lam, idn.L1, idn.L2)
     y64 = O.linear_f64("nvfp4", h, ref_d, idn.L1, idn.L2, idn.bias)

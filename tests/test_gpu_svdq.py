@@ -72,6 +72,24 @@ def _layer(c):
     return inp, pk, w, bias
 
 
+def _check_layer_workspace(ws, c, codes, scales, lora):
+    """The layer's workspace after a call: activation codes and scales equal
+    the quantize kernel's bit for bit, the low-rank activation equal up to the
+    order of its fp32 sums, and the control words back at zero."""
+    B = _lib()
+    off = B.workspace_offsets("nvfp4", c.M, c.K)
+    wcodes = ws[off[1]:off[1] + c.M * c.K // 2].view(c.M, c.K // 2)
+    wscales = ws[off[2]:off[2] + B.act_scale_bytes("nvfp4", c.M, c.K)]
+    wlora = ws[off[3]:off[3] + c.M * 128].view(torch.bfloat16).view(c.M, 64)
+    assert torch.equal(wcodes, codes), "layer codes differ from the quantize kernel's"
+    assert torch.equal(wscales, scales), "layer scales differ from the quantize kernel's"
+    ua = wlora.double()[:, :32] + wlora.double()[:, 32:]
+    ub = lora.double()[:, :32] + lora.double()[:, 32:]
+    # fp32 sums of the same products in two orders (the oracle bound on u is 2e-3 max|u|)
+    assert (ua - ub).abs().max().item() <= 1e-4 * ub.abs().max().item() + 1e-30
+    assert int(ws[:off[1]].count_nonzero().item()) == 0, "control words not left at zero"
+
+
 SMALL = [
     ("tiny", {}),
     ("qkv", dict(M=300, N=1024)),          # ragged M, bias, weight outliers
@@ -82,12 +100,16 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("kernel", ["pair", "single"])
+@pytest.mark.parametrize("kernel", ["pair", "single", "fused"])
 @pytest.mark.parametrize("name,kw", SMALL)
 def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
-    """Both NVFP4 GEMM kernels: the one-CTA-per-tile kernel (the default) and
-    the CTA-pair kernel."""
-    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
+    """Both NVFP4 GEMM kernels: the CTA-pair kernel (the default) and the
+    one-CTA-per-tile kernel, with the layer as quantize + GEMM; and the
+    one-kernel layer (SVDQ_LAYER_KERNEL=fused), which quantizes x inside the
+    pair GEMM."""
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", "single" if kernel == "single" else "pair")
+    if kernel == "fused":
+        monkeypatch.setenv("SVDQ_LAYER_KERNEL", "fused")
     B = _lib()
     c = wl.SVDQ_CASES[name]
     if kw:
@@ -96,7 +118,8 @@ def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
     x, codes, scales, lora = _run_s1(inp, w)
     alpha = float(np.float32(np.float32(inp.act_scale) * np.float32(pk["weight_scale"][0])))
     y = B.svdq_w4a4_gemm("nvfp4", codes, scales, lora, w, alpha, bias=bias)
-    y2 = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias)
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    y2 = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
     torch.cuda.synchronize()
     _check_s1(inp, codes, scales, lora, pk)
     ref_pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
@@ -104,7 +127,13 @@ def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
     y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, inp.bias)
     yg = y.float().cpu().numpy()
     assert_output_close(yg, y64, f"{c.name} gemm")
-    assert torch.equal(y, y2), "svdq_w4a4_linear differs from quantize + gemm"
+    _check_layer_workspace(ws, c, codes, scales, lora)
+    if kernel != "fused":
+        # the two-kernel path: the layer is quantize + gemm, bit for bit
+        assert torch.equal(y, y2), "svdq_w4a4_linear differs from quantize + gemm"
+    else:
+        # one kernel: the low-rank sums run in another (fixed) order
+        assert_output_close(y2.float().cpu().numpy(), y64, f"{c.name} layer")
 
 
 @pytest.mark.parametrize("name,kw", SMALL)
@@ -214,20 +243,26 @@ def test_quantize_int4_operation_order_cases():
 FULL = ["qkv", "mlp_up", "mlp_down"]
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("kernel", ["single", "pair", "fused"])
 @pytest.mark.parametrize("name", FULL)
 def test_linear_full_size_sampled(name, kernel, monkeypatch):
     """Full workload shape (the launch configuration the benchmark times):
     all activation codes bit-exact, 48 sampled output rows within tolerance."""
-    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", kernel)
+    monkeypatch.setenv("SVDQ_NVFP4_GEMM_KERNEL", "single" if kernel == "single" else "pair")
+    if kernel == "fused":
+        monkeypatch.setenv("SVDQ_LAYER_KERNEL", "fused")
     B = _lib()
     c = wl.SVDQ_CASES[name]
     inp, pk, w, bias = _layer(c)
     x = B.bits_to_bf16(inp.x_bits, "cuda")
-    y = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias)
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    y = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
+    y_again = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
     _, codes, scales, lora = _run_s1(inp, w)
     torch.cuda.synchronize()
     ref = _check_s1(inp, codes, scales, lora, pk)
+    _check_layer_workspace(ws, c, codes, scales, lora)
+    assert torch.equal(y, y_again), "the layer is not deterministic"
     rng = np.random.default_rng(99)
     rows = np.sort(np.concatenate([[0, c.M - 1], rng.choice(np.arange(1, c.M - 1), 46, replace=False)]))
     act = {k: ref[k][rows] for k in ("codes", "scales", "x_hat")}

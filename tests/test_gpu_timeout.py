@@ -195,3 +195,40 @@ def test_timeout_through_the_default_binding_path_raises():
     act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
     y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, None)
     assert_output_close(y.float().cpu().numpy(), y64, "layer after a timed-out call")
+
+
+def test_fused_layer_wait_timeout_reports_and_recovers(monkeypatch):
+    """The one-kernel layer (SVDQ_LAYER_KERNEL=fused): its producers wait
+    (bounded) for row blocks that its epilogue warps quantize.  With a 1 ns
+    limit some wait gives up; the kernel reports it, drains its copies, and
+    its last CTA still returns the workspace's control words to zero, so the
+    next call on the same workspace is correct."""
+    import bit_w4a4_diffusion_b200 as B
+    monkeypatch.setenv("SVDQ_LAYER_KERNEL", "fused")
+    c = wl.scaled_case(wl.SVDQ_CASES["qkv"], M=640, N=2048)
+    inp = svdq_inputs(c)
+    pk = B.svdq_pack_weights("nvfp4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    bias = B.bits_to_bf16(inp.bias_bits, "cuda") if inp.bias_bits is not None else None
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    s_a = float(inp.act_scale)
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_linear("nvfp4", x, w, s_a, bias=bias, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+    off = B.workspace_offsets("nvfp4", c.M, c.K)
+    assert int(ws[:off[1]].count_nonzero().item()) == 0, "control words not left at zero"
+    status.zero_()
+    y = B.svdq_w4a4_linear("nvfp4", x, w, s_a, bias=bias, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("nvfp4", inp.x, ref_pw["inv_lam"], np.float32(inp.act_scale))
+    y64 = O.linear_f64("nvfp4", act, ref_pw, inp.L1, inp.L2, inp.bias)
+    assert_output_close(y.float().cpu().numpy(), y64, "one-kernel layer after a timed-out call")
