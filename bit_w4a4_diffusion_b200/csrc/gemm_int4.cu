@@ -12,8 +12,9 @@
 //                    + bias[n] )
 //
 // Every 64-group needs its own rescale, so each group's int32 partial lands
-// in its own TMEM buffer (two, ping-pong) and the epilogue warps fold it into
-// fp32 registers while the tensor core computes the next group: the epilogue
+// in its own TMEM buffer (four, in turn; the tile's low-rank result takes the
+// first one and starts the accumulator) and the epilogue warps fold it into
+// fp32 registers while the tensor core computes the next groups: the epilogue
 // ALU work is what bounds this kernel (the reason the docs expect int4 to be
 // slower than nvfp4 on Blackwell).  Two devices keep that work to two packed
 // FMAs per pair of elements:
@@ -60,20 +61,22 @@ constexpr uint32_t kPresetBits = 0x4B400000u;    // the float 1.5 * 2^23 (ulp 1 
 constexpr float kPreset = 12582912.0f;
 constexpr int UNPACK_WARPS = 4, EPI_WARPS = 8;
 constexpr int EPI_COLS = 4 * BN / EPI_WARPS;   // columns per epilogue warp (4 warps per lane quarter)
-constexpr int NHALF = EPI_COLS / 32;           // 32-column TMEM loads per warp
 constexpr int NUM_THREADS = (2 + UNPACK_WARPS + EPI_WARPS) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_PART = 0;     // two int32 partial buffers: columns 0 and 128
-constexpr int TMEM_LR = 256;     // two fp32 low-rank accumulators: columns 256 and 384
+// Four partial buffers of 128 columns (all of TMEM), used in turn by the
+// tile's low-rank result (fp32, the tile's first "group") and its 64-groups
+// (int32 on the preset C): the MMA can run up to three groups ahead of the
+// epilogue.
+constexpr int NPART = 4;
+constexpr int TMEM_PART = 0;
 constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 
 struct SmemCtl {
   uint64_t full[STAGES];     // producer -> unpack (int4 + scales landed)
   uint64_t opnd[STAGES];     // unpack / TMA -> MMA (int8 or bf16 operands ready)
   uint64_t empty[STAGES];    // MMA commit + epilogue warps -> producer
-  uint64_t part_full[2];     // MMA -> epilogue (group partial ready)
-  uint64_t part_empty[2];    // epilogue -> MMA
-  uint64_t lr_empty[2];      // epilogue -> MMA (low-rank accumulator drained)
+  uint64_t part_full[NPART];    // MMA -> epilogue (group partial ready)
+  uint64_t part_empty[NPART];   // epilogue -> MMA (buffer drained and preset)
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -139,10 +142,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&ctl->opnd[s]), 1);
       mbar_init(smem_u32(&ctl->empty[s]), 1 + EPI_WARPS);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NPART; ++b) {
       mbar_init(smem_u32(&ctl->part_full[b]), 1);
       mbar_init(smem_u32(&ctl->part_empty[b]), EPI_WARPS);
-      mbar_init(smem_u32(&ctl->lr_empty[b]), EPI_WARPS);
     }
     mbar_init(smem_u32(&ctl->drain), 1);
     ctl->abort_flag = 0;
@@ -240,11 +242,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t pcount = 0;  // group partials issued so far
+      uint32_t pcount = 0;  // partial-buffer uses so far (low-rank results and groups)
       bool ok = true;
-      int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-        const int lb = it & 1;
+      // Use pcount / NPART of buffer pcount % NPART: the epilogue has drained
+      // its previous use and preset it.
+      auto take_part = [&]() -> bool {
+        const bool got = mbar_wait_warp(smem_u32(&ctl->part_empty[pcount % NPART]), (pcount / NPART) & 1, wctx,
+                                        kDevTimeoutMma);
+        tc_fence_after();
+        return got;
+      };
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kt = 0; kt < slices && ok; ++kt) {
           if (!mbar_wait_warp(smem_u32(&ctl->opnd[stage]), phase, wctx, kDevTimeoutMma)) {
             ok = false;
@@ -253,29 +261,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(a8(stage)), sb = smem_u32(b8(stage));
           if (kt == 0) {
-            // Low-rank accumulator lb was last read by the epilogue two tiles ago.
-            if (it >= 2 &&
-                !mbar_wait_warp(smem_u32(&ctl->lr_empty[lb]), ((it - 2) >> 1) & 1, wctx, kDevTimeoutMma)) {
+            // The low-rank result (fp32, overwriting the preset).
+            if (!take_part()) {
               ok = false;
               break;
             }
-            tc_fence_after();
+            const uint32_t d = tmem + TMEM_PART + (pcount % NPART) * BN;
             if (elect_one()) {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
-                mma_bf16(tmem + TMEM_LR + lb * BN, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16,
-                         j > 0 ? 1u : 0u);
+                mma_bf16(d, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
+              tc_commit(smem_u32(&ctl->part_full[pcount % NPART]));
             }
             __syncwarp();
+            ++pcount;
           } else {
             for (int h = 0; h < 2; ++h, ++pcount) {
-              const int pb = pcount & 1;
-              // Use pcount / 2 of buffer pb: the epilogue has preset it.
-              if (!mbar_wait_warp(smem_u32(&ctl->part_empty[pb]), (pcount >> 1) & 1, wctx, kDevTimeoutMma)) {
+              const int pb = pcount % NPART;
+              if (!take_part()) {
                 ok = false;
                 break;
               }
-              tc_fence_after();
               const uint32_t d = tmem + TMEM_PART + pb * BN;
               if (elect_one()) {
                 mma_i8(d, sw128_desc(sa + 64 * h), sw128_desc(sb + 64 * h), IDESC_I8, 1u);
@@ -316,20 +322,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           // all 128 unpack threads take the same branch: the abort flag is shared
           if (ok) {
+            // 16-byte piece i = t + 128 j of the 8 KB packed tile is row i / 4,
+            // columns 32 (i % 4) .. + 31: a warp reads 512 contiguous bytes
+            // (no bank conflict; one thread per 64-byte row made every
+            // quarter-warp load hit two bank groups), and the two 16-byte
+            // int8 chunks it writes land, under the 128-byte swizzle, in
+            // chunk sets of opposite parity for the two rows of a
+            // quarter-warp (no conflict either).
             for (int op = 0; op < 2; ++op) {
-              const uint8_t* src = (op == 0 ? a4(stage) : b4(stage)) + t * (KS / 2);
-              uint8_t* dst = (op == 0 ? a8(stage) : b8(stage)) + t * KS;
+              const uint8_t* src = op == 0 ? a4(stage) : b4(stage);
+              uint8_t* dst = op == 0 ? a8(stage) : b8(stage);
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {  // 16 packed bytes -> two 16-byte int8 chunks
-                const uint4 w = *reinterpret_cast<const uint4*>(src + 16 * c);
+              for (int j = 0; j < 4; ++j) {
+                const int i = t + 128 * j;
+                const int r = i >> 2, c = i & 3;
+                const uint4 w = *reinterpret_cast<const uint4*>(src + 16 * i);
                 uint4 o0, o1;
                 unpack_int4x8(w.x, o0.x, o0.y);
                 unpack_int4x8(w.y, o0.z, o0.w);
                 unpack_int4x8(w.z, o1.x, o1.y);
                 unpack_int4x8(w.w, o1.z, o1.w);
-                const int ch0 = 2 * c, ch1 = 2 * c + 1;  // logical 16-byte chunks of the row
-                *reinterpret_cast<uint4*>(dst + 16 * (ch0 ^ (t & 7))) = o0;
-                *reinterpret_cast<uint4*>(dst + 16 * (ch1 ^ (t & 7))) = o1;
+                uint8_t* row = dst + r * KS;
+                *reinterpret_cast<uint4*>(row + 16 * ((2 * c) ^ (r & 7))) = o0;
+                *reinterpret_cast<uint4*>(row + 16 * ((2 * c + 1) ^ (r & 7))) = o1;
               }
             }
             fence_proxy_async_smem();
@@ -368,7 +383,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int stage = 0;
     uint32_t phase = 0, pcount = 0;
     bool ok = true;
-    int it = 0;
     // This warp's columns of partial buffer pb.
     auto part_addr = [&](int pb) {
       return tmem + ((uint32_t)(32 * q) << 16) + TMEM_PART + pb * BN + EPI_COLS * ch;
@@ -383,15 +397,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->part_empty[pb]));
     };
-    preset_release(0);
-    preset_release(1);
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+#pragma unroll
+    for (int b = 0; b < NPART; ++b) preset_release(b);
+    auto wait_part = [&](int pb) -> bool {
+      const bool got = mbar_wait(smem_u32(&ctl->part_full[pb]), (pcount / NPART) & 1, wctx, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      tc_fence_after();
+      return true;
+    };
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
       float2 acc[EPI_COLS / 2];   // columns (2 i, 2 i + 1) of this thread's EPI_COLS
-#pragma unroll
-      for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = make_float2(0.f, 0.f);
       for (int kt = 0; kt < slices && ok; ++kt) {
-        if (kt > 0) {
+        if (kt == 0) {
+          // The low-rank result starts the accumulator.
+          const int pb = pcount % NPART;
+          if (!wait_part(pb)) {
+            ok = false;
+            break;
+          }
+          const uint32_t taddr = part_addr(pb);
+#pragma unroll
+          for (int qc = 0; qc < EPI_COLS / 16; ++qc) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(taddr + 16 * qc, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[8 * qc + i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          }
+          preset_release(pb);
+          ++pcount;
+        } else {
           // The slice's fp32 scales, staged by the unpack warps.
           const bool sc_ok = mbar_wait(smem_u32(&ctl->opnd[stage]), phase, wctx, kDevTimeoutEpilogue);
           if (!__all_sync(0xffffffffu, sc_ok)) {
@@ -400,13 +437,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const float* sf = scf(stage);
           for (int h = 0; h < 2; ++h, ++pcount) {
-            const int pb = pcount & 1;
-            const bool got = mbar_wait(smem_u32(&ctl->part_full[pb]), (pcount >> 1) & 1, wctx, kDevTimeoutEpilogue);
-            if (!__all_sync(0xffffffffu, got)) {
+            const int pb = pcount % NPART;
+            if (!wait_part(pb)) {
               ok = false;
               break;
             }
-            tc_fence_after();
             const float* sfh = sf + h * (BM + 2 * BN);
             const float sa1 = sfh[row];
             const float2 sa = make_float2(sa1, sa1);
@@ -450,21 +485,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!ok) break;
-      // Low-rank accumulator (its MMAs completed before the last partial's).
-      const int lb = it & 1;
+      // y = bf16(acc + bias): the low-rank result is already in acc.
       const int m = m0 + row;
-      const uint32_t laddr = tmem + ((uint32_t)(32 * q) << 16) + TMEM_LR + lb * BN + EPI_COLS * ch;
-      // 16 columns per TMEM load, as in the group drain.
 #pragma unroll
       for (int qc = 0; qc < EPI_COLS / 16; ++qc) {
-        uint32_t l[16];
-        tmem_ld_32x32b_x16(laddr + 16 * qc, l);
-        tmem_ld_wait(l);
-        if (qc == EPI_COLS / 16 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&ctl->lr_empty[lb]));
-        }
         const int nb = n0 + EPI_COLS * ch + 16 * qc;
         if (m < p.M && nb < p.N) {
           uint16_t* yrow = p.y + (size_t)m * p.N + nb;
@@ -474,8 +498,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int j = 8 * v + 2 * i;
-              float y0 = __fadd_rn(acc[8 * qc + j / 2].x, __uint_as_float(l[j]));
-              float y1 = __fadd_rn(acc[8 * qc + j / 2].y, __uint_as_float(l[j + 1]));
+              float y0 = acc[8 * qc + j / 2].x, y1 = acc[8 * qc + j / 2].y;
               if (p.bias) {
                 y0 = __fadd_rn(y0, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j])));
                 y1 = __fadd_rn(y1, __bfloat162float(__ushort_as_bfloat16(p.bias[nb + j + 1])));
