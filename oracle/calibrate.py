@@ -7,7 +7,7 @@ Diffusers", section "SVDQuant and the Nunchaku engine": activation outliers
 are migrated into the weights, then the hardest part of each weight matrix
 is absorbed by a 16-bit low-rank branch obtained by decomposing it; the
 "Nunchaku Lite" docs' config example uses rank 32.  The pages give no
-formula; the reading (listed with the others in the design notes):
+formula; the reading taken here, where each choice is this module's own:
 
     lambda_j   = sqrt(max_i |x_ij| / max_n |W_nj|) in fp32, 1 where a max is 0
                  (migration strength 1/2 over the calibration batch x)

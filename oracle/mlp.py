@@ -5,8 +5,8 @@ the CPU-baseline leg of ``bench.py``, never by the product path).
 Page: "Nunchaku Lite" (Diffusers docs), section "Fused kernels": the original
 Nunchaku engine runs the MLP with a fused GELU kernel (its table credits the
 "GELU-MLP fusion" with 1.06x per step); Nunchaku Lite runs the same layers
-without it.  The pages give no formula.  The reading taken here (listed with
-the other readings in the design notes):
+without it.  The pages give no formula.  The reading taken here (the
+plainest composition of the two layers that never stores the up output):
 
     v     = up layer output before its bf16 rounding
           = Q(x_hat) Q(R_up)^T + x_hat L1_up L2_up + b_up        (fp64 here)

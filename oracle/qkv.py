@@ -6,9 +6,8 @@ Page: "Nunchaku Lite" (Diffusers docs), section "Fused kernels": the original
 Nunchaku engine combines the Q, K and V projections with RMSNorm and RoPE
 (its table credits the fusion with 1.27x per step); Nunchaku Lite runs the
 same layers without it.  The pages give neither a formula nor the head
-layout.  The reading taken here (listed with the other readings in the
-design notes) is the one of diffusion transformers with query/key
-normalization:
+layout.  The reading taken here is the one of diffusion transformers with
+query/key normalization:
 
     v        = the QKV layer's output before rounding, [M, 3 H d], columns
                [Q | K | V], head h of each part in columns [h d, (h + 1) d)

@@ -15,8 +15,9 @@ What the pages say (no formula, no code is printed there):
   ``svdq_w4a4`` with ``nvfp4`` (group 16) or ``int4`` (group 64), and the
   config example there uses ``rank: 32``.
 
-The layer computed here (the plainest reading, all readings listed in the
-design notes):
+The layer computed here (the plainest reading of the pages; where they are
+silent, the reading taken is stated in the docstring of the function that
+takes it):
 
     x_hat = x * inv_lambda                  (per input channel, one fp32 multiply)
     W_hat = W * lambda                      (per input channel, exact in fp64)
