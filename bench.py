@@ -262,7 +262,7 @@ def run_gpu(args, rank, world, local_rank):
     for i in range(nsets):
         w = B.to_device(pk, dev)
         sets.append(dict(w=w, x=x0.clone(), y=torch.empty((M, N), dtype=torch.bfloat16, device=dev),
-                         ws=torch.zeros(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev),
+                         ws=torch.zeros(B.workspace_bytes("nvfp4", M, N, K), dtype=torch.uint8, device=dev),
                          codes=torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
                          scales=torch.empty(B.act_scale_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev),
                          lora=torch.empty((M, 64), dtype=torch.bfloat16, device=dev)))
@@ -539,7 +539,7 @@ def measure_rows(B, wl, dev, peaks):
         ws = [B.to_device(pk, dev) for _ in range(nset)]
         x = B.bits_to_bf16(inp.x_bits, dev)
         ys = [torch.empty((M, c.N), dtype=torch.bfloat16, device=dev) for _ in range(nset)]
-        wsp = torch.zeros(B.workspace_bytes("int4", M, c.K), dtype=torch.uint8, device=dev)
+        wsp = torch.zeros(B.workspace_bytes("int4", M, c.N, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=ys[i], workspace=wsp) for i in range(nset)]
         t = _event_time_us(torch, fns, 40)
         int4[f"M={M}"] = {"us": round(t, 2), "TOPS": round(2.0 * M * c.N * c.K / t / 1e6, 1)}
@@ -564,7 +564,7 @@ def measure_read_reference(dev, peaks):
         nset = max(2, -(-2 * L2_BYTES // (mib * 2 ** 20)))
         bufs = [torch.randn(n, device=dev).to(torch.bfloat16) for _ in range(nset)]
         acc = torch.empty((), dtype=torch.float32, device=dev)
-        fns = [lambda i=i: torch.sum(bufs[i], dtype=torch.float32, out=acc) for i in range(nset)]
+        fns = [lambda i=i: torch.sum(bufs[i], dim=0, dtype=torch.float32, out=acc) for i in range(nset)]
         t = _event_time_us(torch, fns, 40)
         out[f"{mib} MiB"] = {"us": round(t, 2), "GB/s": round(mib * 2 ** 20 / t / 1e3, 1),
                              "hbm_frac": round(mib * 2 ** 20 / t / 1e3 / peaks["hbm_gbs"], 3)}
@@ -593,7 +593,7 @@ def measure_qkv(B, wl, dev, heads=24):
     bias = B.bits_to_bf16(inp.bias_bits, dev)
     s_a = float(inp.act_scale)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    wsp = torch.zeros(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
+    wsp = torch.zeros(B.workspace_bytes("nvfp4", M, N, K), dtype=torch.uint8, device=dev)
     hd = heads * 128
 
     gq16, gk16 = gq.to(torch.bfloat16), gk.to(torch.bfloat16)
@@ -660,7 +660,7 @@ def block_layers(B, wl, dev, M, calibrate=None):
            "qkv": torch.empty((M, 9216), dtype=torch.bfloat16, device=dev),
            "attn_out": torch.empty((M, 3072), dtype=torch.bfloat16, device=dev),
            "mlp": torch.empty((M, 3072), dtype=torch.bfloat16, device=dev)}
-    ws = torch.zeros(max(B.workspace_bytes("nvfp4", M, 3072), B.mlp_workspace_bytes(M, 3072, 12288)),
+    ws = torch.zeros(max(B.workspace_bytes("nvfp4", M, 9216, 3072), B.mlp_workspace_bytes(M, 3072, 12288)),
                      dtype=torch.uint8, device=dev)
 
     def run():
@@ -795,7 +795,7 @@ def run_profile_calls(row, calls):
         ws = [B.to_device(pk, dev) for _ in range(4)]
         x = B.bits_to_bf16(inp.x_bits, dev)
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
-        wsp = torch.zeros(B.workspace_bytes("int4", c.M, c.K), dtype=torch.uint8, device=dev)
+        wsp = torch.zeros(B.workspace_bytes("int4", c.M, c.N, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=y, workspace=wsp) for i in range(4)]
     elif row == "cublas_fp4":
         M, K, N = 4096, 3072, 12288
@@ -813,7 +813,7 @@ def run_profile_calls(row, calls):
         x = B.bits_to_bf16(inp.x_bits, dev)
         bias = B.bits_to_bf16(inp.bias_bits, dev) if inp.bias_bits is not None else None
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
-        wsp = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device=dev)
+        wsp = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.N, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_linear("nvfp4", x, ws[i], float(inp.act_scale), bias=bias, y=y, workspace=wsp)
                for i in range(4)]
     elif row == "qkv":
@@ -826,7 +826,7 @@ def run_profile_calls(row, calls):
         x = B.bits_to_bf16(inp.x_bits, dev)
         bias = B.bits_to_bf16(inp.bias_bits, dev)
         y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
-        wsp = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device=dev)
+        wsp = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.N, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_qkv_norm_rope_linear(x, ws[i], float(inp.act_scale), 24, *t, bias=bias, y=y,
                                                             workspace=wsp) for i in range(2)]
     else:
@@ -855,8 +855,8 @@ def measure_mlp(B, wl, dev):
     fused = [lambda i=i: B.svdq_w4a4_mlp_gelu(x, wus[i], s_u, wds[i], s_d, up_bias=b_u, down_bias=b_d, y=y,
                                               workspace=ws) for i in range(nset)]
     y_up = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ws_u = torch.zeros(B.workspace_bytes("nvfp4", M, K), dtype=torch.uint8, device=dev)
-    ws_d = torch.zeros(B.workspace_bytes("nvfp4", M, N), dtype=torch.uint8, device=dev)
+    ws_u = torch.zeros(B.workspace_bytes("nvfp4", M, N, K), dtype=torch.uint8, device=dev)
+    ws_d = torch.zeros(B.workspace_bytes("nvfp4", M, K, N), dtype=torch.uint8, device=dev)
 
     def unfused(i):
         B.svdq_w4a4_linear("nvfp4", x, wus[i], s_u, bias=b_u, y=y_up, workspace=ws_u)

@@ -44,8 +44,8 @@ def _load():
         "svdq_device_status": (I, [P, I, P]),
         "svdq_act_scale_bytes": (LL, [I, I, I]),
         "svdq_weight_scale_bytes": (LL, [I, I, I]),
-        "svdq_workspace_bytes": (LL, [I, I, I, I]),
-        "svdq_workspace_offsets": (I, [I, I, I, I, P]),
+        "svdq_workspace_bytes": (LL, [I, I, I, I, I]),
+        "svdq_workspace_offsets": (I, [I, I, I, I, I, P]),
         "svdq_scales_to_rowmajor": (I, [I, I, P, P]),
         "svdq_scales_from_rowmajor": (I, [I, I, P, P]),
         "svdq_pack_weights": (I, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
@@ -120,18 +120,19 @@ def weight_scale_bytes(precision, N, K):
     return int(lib.svdq_weight_scale_bytes(_prec(precision), N, K))
 
 
-def workspace_bytes(precision, M, K, rank=SVDQ_RANK):
-    """Bytes of a layer workspace.  Its first 64 KiB are control words that
-    must be zero before the first call on it (allocate it zeroed); every call
-    leaves them zero."""
-    return int(lib.svdq_workspace_bytes(_prec(precision), M, K, rank))
+def workspace_bytes(precision, M, N, K, rank=SVDQ_RANK):
+    """Bytes of the workspace of a layer [M, K] -> [M, N].  Its first 64 KiB
+    are control words that must be zero before the first call on it
+    (allocate it zeroed); every call leaves them zero."""
+    return int(lib.svdq_workspace_bytes(_prec(precision), M, N, K, rank))
 
 
-def workspace_offsets(precision, M, K, rank=SVDQ_RANK):
+def workspace_offsets(precision, M, N, K, rank=SVDQ_RANK):
     """Byte offsets in a layer workspace: control words, act codes, act
-    scales, lora_act, low-rank partial sums, end."""
+    scales, lora_act, the precision's own region (NVFP4: the one-kernel
+    layer's low-rank partial sums; INT4: the fp16 operands), end."""
     off = np.zeros(6, np.int64)
-    _check(lib.svdq_workspace_offsets(_prec(precision), M, K, rank, off.ctypes.data))
+    _check(lib.svdq_workspace_offsets(_prec(precision), M, N, K, rank, off.ctypes.data))
     return [int(v) for v in off]
 
 
@@ -296,7 +297,7 @@ def svdq_w4a4_linear(precision, x, w, act_scale, bias=None, y=None, workspace=No
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = torch.zeros(workspace_bytes(p, M, K, rank), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(workspace_bytes(p, M, N, K, rank), dtype=torch.uint8, device=x.device)
     wscale = w["weight_scale_f"]
     _check(lib.svdq_w4a4_linear(p, M, N, K, rank, _ptr(x), _ptr(w["inv_smooth"]), _ptr(w["lora_down"]),
                                 float(act_scale), _ptr(w["codes"]), _ptr(w["scales"]), wscale, _ptr(w["lora_up"]),
@@ -404,7 +405,7 @@ def svdq_w4a4_qkv_norm_rope_linear(x, w, act_scale, heads, gamma_q, gamma_k, rop
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = torch.zeros(workspace_bytes(SVDQ_NVFP4, M, K, rank), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(workspace_bytes(SVDQ_NVFP4, M, N, K, rank), dtype=torch.uint8, device=x.device)
     _check(lib.svdq_w4a4_qkv_norm_rope_linear(M, K, int(heads), int(head_dim), rank, _ptr(x), _ptr(w["inv_smooth"]),
                                               _ptr(w["lora_down"]), float(act_scale), _ptr(w["codes"]),
                                               _ptr(w["scales"]), w["weight_scale_f"], _ptr(w["lora_up"]), _ptr(bias),

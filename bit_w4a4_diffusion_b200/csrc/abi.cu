@@ -250,18 +250,37 @@ long long svdq_act_scale_bytes(int precision, int M, int K) {
 
 long long svdq_weight_scale_bytes(int precision, int N, int K) { return svdq_act_scale_bytes(precision, N, K); }
 
-int svdq_workspace_offsets(int precision, int M, int K, int rank, long long* offsets) {
+// The INT4 layer's fp16-operand region (workspace offset [4]), in bytes from
+// its start: A' [M, K] fp16, the scaled lora_act [M, 64] bf16, f_a [M] fp32,
+// W' [N, K] fp16, the scaled lora_up [N, 64] bf16, f_w [N] fp32, each
+// 256-byte aligned; o[6] is the region's size.
+static void int4_operand_offsets(int M, int N, int K, long long (&o)[7]) {
+  o[0] = 0;
+  o[1] = o[0] + round_up((int64_t)M * K * 2, 256);
+  o[2] = o[1] + round_up((int64_t)M * 64 * 2, 256);
+  o[3] = o[2] + round_up((int64_t)M * 4, 256);
+  o[4] = o[3] + round_up((int64_t)N * K * 2, 256);
+  o[5] = o[4] + round_up((int64_t)N * 64 * 2, 256);
+  o[6] = o[5] + round_up((int64_t)N * 4, 256);
+}
+
+int svdq_workspace_offsets(int precision, int M, int N, int K, int rank, long long* offsets) {
   if (!offsets) return fail(SVDQ_ERR_INVALID_ARG, "null offsets");
   if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
     return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
   if (M <= 0 || K <= 0 || K % 256 != 0 || rank != SVDQ_RANK)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d rank=%d", M, K, rank);
+  if (N < 0 || (precision == SVDQ_INT4 && (N == 0 || N % 128 != 0)))
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N=%d (INT4 needs a positive multiple of 128)", N);
   const long long codes = kSyncBytes;
   const long long scales = codes + round_up((int64_t)M * (K / 2), 256);
   const long long lora = scales + round_up(svdq_act_scale_bytes(precision, M, K), 256);
   const long long upart = lora + round_up((int64_t)M * 2 * rank * 2, 256);
+  long long int4_region[7];
+  int4_operand_offsets(M, N, K, int4_region);
   const long long end =
-      upart + (precision == SVDQ_NVFP4 ? round_up((int64_t)fused_splits(K) * round_up(M, 256) * 32 * 4, 256) : 0);
+      upart + (precision == SVDQ_NVFP4 ? round_up((int64_t)fused_splits(K) * round_up(M, 256) * 32 * 4, 256)
+                                       : int4_region[6]);
   offsets[0] = 0;
   offsets[1] = codes;
   offsets[2] = scales;
@@ -271,9 +290,9 @@ int svdq_workspace_offsets(int precision, int M, int K, int rank, long long* off
   return SVDQ_OK;
 }
 
-long long svdq_workspace_bytes(int precision, int M, int K, int rank) {
+long long svdq_workspace_bytes(int precision, int M, int N, int K, int rank) {
   long long off[6];
-  if (svdq_workspace_offsets(precision, M, K, rank, off) != SVDQ_OK) return -1;
+  if (svdq_workspace_offsets(precision, M, N, K, rank, off) != SVDQ_OK) return -1;
   return off[5];
 }
 
@@ -474,6 +493,63 @@ static int gemm_int4_impl(int M, int N, int K, const void* act_codes, const void
   return check_cuda(launch_gemm_int4(p, t, sms, stream, pdl), "gemm_int4 launch");
 }
 
+// The INT4 layer's product on the fp16 tensor pipe: both operands turned into
+// exact fp16 values (dequant_int4.cu) in the workspace region `region`, then
+// the CTA-pair GEMM with kind::f16 MMAs and one accumulator per tile.  The
+// i8 kernel (gemm_int4.cu) needs no scratch and stays the GEMM of
+// svdq_w4a4_gemm; SVDQ_INT4_LAYER_GEMM=i8 (read at every call) runs it in
+// the layer too, for comparison.  Both sum the same exact products in fp32.
+static bool use_int4_i8_gemm() {
+  const char* v = getenv("SVDQ_INT4_LAYER_GEMM");
+  return v && strcmp(v, "i8") == 0;
+}
+
+static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const void* act_scales,
+                              const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
+                              const void* bias, void* y, uint8_t* region, int* dev_status, cudaStream_t stream,
+                              bool pdl) {
+  long long o[7];
+  int4_operand_offsets(M, N, K, o);
+  uint16_t* a16 = reinterpret_cast<uint16_t*>(region + o[0]);
+  uint16_t* la = reinterpret_cast<uint16_t*>(region + o[1]);
+  float* fa = reinterpret_cast<float*>(region + o[2]);
+  uint16_t* w16 = reinterpret_cast<uint16_t*>(region + o[3]);
+  uint16_t* lb = reinterpret_cast<uint16_t*>(region + o[4]);
+  float* fw = reinterpret_cast<float*>(region + o[5]);
+  GemmPairTmaps u;
+  bool ok = true;
+  ok &= encode_tmap_2d(&u.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a16, (uint64_t)K * 2, M, (uint64_t)K * 2, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w16, (uint64_t)K * 2, N, (uint64_t)K * 2, 128, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, 2 * SVDQ_RANK, M, 2 * SVDQ_RANK * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lb, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_tmap_2d(&u.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
+                       CU_TENSOR_MAP_SWIZZLE_32B);
+  if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the fp16-operand INT4 GEMM");
+  u.sfa = u.a;   // not read
+  u.sfb = u.a;
+  DequantInt4Params da{M, K, (int)round_up(M, 256), static_cast<const uint8_t*>(act_codes),
+                       static_cast<const uint16_t*>(act_scales), static_cast<const uint16_t*>(lora_act), a16, la, fa};
+  DequantInt4Params dw{N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
+                       static_cast<const uint16_t*>(w_scales), static_cast<const uint16_t*>(lora_up), w16, lb, fw};
+  if (int s = check_cuda(launch_dequant_int4(dw, stream, pdl), "dequant_int4 (weights) launch")) return s;
+  if (int s = check_cuda(launch_dequant_int4(da, stream, pdl), "dequant_int4 (activations) launch")) return s;
+  GemmNvfp4Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.alpha = 1.0f;
+  p.dev_status = dev_status;
+  p.timeout_ns = svdq_timeout_ns();
+  p.row_factor = fa;
+  p.col_factor = fw;
+  return check_cuda(launch_gemm_f16_pair(p, u, stream, pdl), "gemm_f16_pair (INT4) launch");
+}
+
 int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act_codes, const void* act_scales,
                    const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
                    const void* bias, float alpha, void* y, int* dev_status, void* stream) {
@@ -581,12 +657,12 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
                      long long workspace_bytes, int* dev_status, void* stream) {
   if (int s = check_gemm_args(precision, M, N, K, rank)) return s;
   if (!workspace) return fail(SVDQ_ERR_INVALID_ARG, "null workspace");
-  const long long need = svdq_workspace_bytes(precision, M, K, rank);
+  const long long need = svdq_workspace_bytes(precision, M, N, K, rank);
   if (workspace_bytes < need)
     return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   long long off[6];
-  if (int s = svdq_workspace_offsets(precision, M, K, rank, off)) return s;
+  if (int s = svdq_workspace_offsets(precision, M, N, K, rank, off)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* codes = ws + off[1];
   uint8_t* scales = ws + off[2];
@@ -612,9 +688,13 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   if (int s = quantize_act_impl(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
                                 scales, lora, dev_status, stream))
     return s;
-  if (precision == SVDQ_INT4)
-    return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
-                          static_cast<cudaStream_t>(stream), pdl_on(), sms);
+  if (precision == SVDQ_INT4) {
+    if (use_int4_i8_gemm())
+      return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
+                            static_cast<cudaStream_t>(stream), pdl_on(), sms);
+    return gemm_int4_f16_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, ws + off[4],
+                              dev_status, static_cast<cudaStream_t>(stream), pdl_on());
+  }
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);
 }
@@ -723,8 +803,8 @@ int svdq_w4a4_gemm_gelu_quant(int M, int N, int K, int rank, const void* act_cod
 }
 
 long long svdq_mlp_workspace_bytes(int M, int K, int N_hidden, int rank) {
-  const long long a = svdq_workspace_bytes(SVDQ_NVFP4, M, K, rank);
-  const long long h = svdq_workspace_bytes(SVDQ_NVFP4, M, N_hidden, rank);
+  const long long a = svdq_workspace_bytes(SVDQ_NVFP4, M, N_hidden, K, rank);
+  const long long h = svdq_workspace_bytes(SVDQ_NVFP4, M, K, N_hidden, rank);
   const long long w = svdq_gelu_quant_work_bytes(M);
   if (a < 0 || h < 0 || w < 0) return -1;
   return a + h + w;
@@ -747,8 +827,8 @@ int svdq_w4a4_mlp_gelu(int M, int K, int N_hidden, int rank, const void* x, cons
   if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   // [the up layer's workspace | the down layer's workspace | the work buffer]
   long long oa[6], oh[6];
-  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, K, rank, oa)) return s;
-  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, N, rank, oh)) return s;
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, N, K, rank, oa)) return s;
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, K, N, rank, oh)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* a_codes = ws + oa[1];
   uint8_t* a_scales = ws + oa[2];
@@ -843,7 +923,7 @@ int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int ra
   const int N = 3 * heads * head_dim;
   if (int s = check_qkv_args(M, N, K, rank, heads, head_dim, gamma_q, gamma_k, rope_cos, rope_sin, y)) return s;
   if (!workspace) return fail(SVDQ_ERR_INVALID_ARG, "null workspace");
-  const long long need = svdq_workspace_bytes(SVDQ_NVFP4, M, K, rank);
+  const long long need = svdq_workspace_bytes(SVDQ_NVFP4, M, N, K, rank);
   if (workspace_bytes < need)
     return fail(SVDQ_ERR_INVALID_ARG, "workspace of %lld bytes is smaller than the %lld needed", workspace_bytes, need);
   if (!aligned16(workspace)) return fail(SVDQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
@@ -851,7 +931,7 @@ int svdq_w4a4_qkv_norm_rope_linear(int M, int K, int heads, int head_dim, int ra
   if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(lora_up) || (bias && !aligned16(bias)))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   long long off[6];
-  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, K, rank, off)) return s;
+  if (int s = svdq_workspace_offsets(SVDQ_NVFP4, M, N, K, rank, off)) return s;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* codes = ws + off[1];
   uint8_t* scales = ws + off[2];

@@ -59,6 +59,13 @@
 //   acc_empty   CTA 0 only; the 16 epilogue warps of both CTAs arrive on it
 // Every mbarrier wait is bounded; on timeout the kernel records a status code,
 // drains what it can observe, and both CTAs meet at the final cluster barrier.
+//
+// The same pipeline also runs the INT4 layer's product on fp16 operands
+// (EPI_F16; the operands come from dequant_int4.cu, exact fp16 values of the
+// dequantized codes, each row scaled by a power of two): the K slices are 64
+// fp16 elements (128 bytes, one 64-group) with four kind::f16 MMAs each and
+// no block scales, the low-rank slice is the same, and the epilogue applies
+// the rows' and columns' powers of two: y = bf16(D f_a[m] f_w[n] + bias).
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -84,9 +91,11 @@ static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of S
 constexpr int EPI_WARPS = 8;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int EPI_PLAIN = 0, EPI_GELU = 1, EPI_QKV = 2;
+constexpr int EPI_PLAIN = 0, EPI_GELU = 1, EPI_QKV = 2, EPI_F16 = 3;
 template <int kEpi>
-constexpr int num_threads() { return kEpi == EPI_PLAIN ? (MMA_WARP + 1) * 32 : 12 * 32; }
+constexpr bool fused_epi() { return kEpi == EPI_GELU || kEpi == EPI_QKV; }
+template <int kEpi>
+constexpr int num_threads() { return fused_epi<kEpi>() ? 12 * 32 : (MMA_WARP + 1) * 32; }
 // Fused epilogues: launched at 168 registers per thread; the third warpgroup
 // (producer, MMA, two idle warps) drops to 72 and the two epilogue
 // warpgroups rise to 216.
@@ -129,7 +138,7 @@ constexpr int stages() { return kQuant ? 4 : STAGES; }
 template <int kEpi, bool kQuant>
 constexpr size_t smem_bytes() {
   return 1024 + stages<kQuant>() * STAGE_BYTES + EPI_BYTES + (kQuant ? 2 * QC_BUF_BYTES : 0) +
-         (kEpi != EPI_PLAIN || kQuant ? TABLE_BYTES : 0) + sizeof(SmemCtl);
+         (fused_epi<kEpi>() || kQuant ? TABLE_BYTES : 0) + sizeof(SmemCtl);
 }
 static_assert(QC_BUF_BYTES % 1024 == 0 && EPI_BYTES % 1024 == 0, "chunk buffers keep the SWIZZLE_128B alignment");
 static_assert(smem_bytes<EPI_GELU, false>() <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
@@ -139,6 +148,8 @@ static_assert(smem_bytes<EPI_PLAIN, true>() <= 232448, "fits the 227 KB opt-in s
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 constexpr uint32_t IDESC_BF16 =
     (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+// kind::f16 with fp16 A and B (format 0), fp32 D.
+constexpr uint32_t IDESC_F16 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
 SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
 SVDQ_DEV uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
@@ -159,9 +170,10 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
   constexpr int kStages = stages<kQuant>();
   uint8_t* stage_base = smem;
   uint8_t* epi_base = smem + kStages * STAGE_BYTES;
-  constexpr bool kGelu = kEpi == EPI_GELU, kQkv = kEpi == EPI_QKV, kFused = kEpi != EPI_PLAIN;
-  static_assert(!kFused || kGelu || kQkv, "epilogue kind");
-  static_assert(!kQuant || !kFused, "the fused layer kernel has the plain epilogue");
+  constexpr bool kGelu = kEpi == EPI_GELU, kFused = fused_epi<kEpi>();
+  constexpr bool kF16 = kEpi == EPI_F16;
+  static_assert(kEpi >= EPI_PLAIN && kEpi <= EPI_F16, "epilogue kind");
+  static_assert(!kQuant || kEpi == EPI_PLAIN, "the fused layer kernel has the plain epilogue");
   // Fused layer kernel: the quantizer's chunk buffers, then its 1/d table.
   uint8_t* q_base = epi_base + EPI_BYTES;
   uint8_t* table_base = q_base + (kQuant ? 2 * QC_BUF_BYTES : 0);
@@ -173,7 +185,7 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
   const int tiles_m = (p.M + 2 * BM - 1) / (2 * BM);
   const int tiles_n = (p.N + BN - 1) / BN;
   const int num_tiles = tiles_m * tiles_n;
-  const int k_tiles = p.K / 256;
+  const int k_tiles = kF16 ? p.K / 64 : p.K / 256;
   const int slices = k_tiles + 1;  // + the low-rank slice (slice 0, no block scales)
   // Tile schedule.  Plain and QKV epilogues: round robin over tiles numbered
   // M-block fastest.  GELU-MLP epilogue: cluster i takes the contiguous run
@@ -283,10 +295,12 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
         uint8_t* sb = sa + A_BYTES;
         uint8_t* ssfb = sb + B_BYTES + SFA_BYTES;
         const uint32_t full = full_addr(st);
-        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[st]), kt == 0 ? 2 * (A_BYTES + B_BYTES)
-                                                                              : 2 * STAGE_BYTES);
+        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&ctl->full[st]), kt == 0 || kF16 ? 2 * (A_BYTES + B_BYTES)
+                                                                                      : 2 * STAGE_BYTES);
         if (kt == 0) {
           tma_load_2d_pair(smem_u32(sb), &tm_lb, 0, nb, full, pol);
+        } else if (kF16) {
+          tma_load_2d_pair(smem_u32(sb), &tm_b, (kt - 1) * BK_BYTES, nb, full, pol);
         } else {
           const int kb = kt - 1;
           tma_load_2d_pair(smem_u32(sb), &tm_b, kb * BK_BYTES, nb, full, pol);
@@ -305,7 +319,7 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
         } else {
           const int kb = kt - 1;
           tma_load_2d_pair(smem_u32(sa), &tm_a, kb * BK_BYTES, m0, full, pol);
-          tma_load_2d_pair(smem_u32(ssfa), &tm_sfa, 0, ((m0 / 128) * kch + kb * 4) * 2, full, pol);
+          if (!kF16) tma_load_2d_pair(smem_u32(ssfa), &tm_sfa, 0, ((m0 / 128) * kch + kb * 4) * 2, full, pol);
         }
       };
       auto advance = [&]() {
@@ -437,6 +451,11 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               mma_bf16_pair(tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_BF16, j > 0 ? 1u : 0u);
+          } else if (kF16) {
+            // 64 fp16 elements: four K = 16 steps of 32 bytes in the swizzled rows.
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_bf16_pair(tmem, sw128_desc(sa + 32 * j), sw128_desc(sb + 32 * j), IDESC_F16, 1u);
           } else {
             // Scales smem -> this stage's TMEM buffer in both CTAs: per K64
             // chunk j, SFA (4 columns) and the SFB of the tile's two 128-row
@@ -623,6 +642,15 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
       // Lane l holds the bias of columns nw + 4 l .. nw + 4 l + 3.
       uint2 bias4 = make_uint2(0, 0);
       if (p.bias != nullptr && nw + 4 * lane < p.N) bias4 = __ldg(reinterpret_cast<const uint2*>(p.bias + nw) + lane);
+      // fp16-operand kernel: the row's power of two (this lane's row) and,
+      // in lane l, those of columns nw + 4 l .. + 3.
+      float f_row = 0.f;
+      float4 f_col4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (kF16) {
+        const int row = m0 + 32 * q + lane;
+        if (row < p.M) f_row = __ldg(p.row_factor + row);
+        if (nw + 4 * lane < p.N) f_col4 = __ldg(reinterpret_cast<const float4*>(p.col_factor + nw) + lane);
+      }
       const bool got = mbar_wait(smem_u32(&ctl->acc_full), acc_phase, wctx, kDevTimeoutEpilogue);
       if constexpr (kQuant) {
         if (named_bar_any(2, NT, !got)) break;   // decided by all eight warps
@@ -660,11 +688,26 @@ __global__ void __launch_bounds__(num_threads<kEpi>(), 1)
             bw[2 * j] = __shfl_sync(0xffffffffu, bias4.x, c0 / 4 + j);
             bw[2 * j + 1] = __shfl_sync(0xffffffffu, bias4.y, c0 / 4 + j);
           }
+          // Per column, the factor D is multiplied by: alpha, or for the
+          // fp16-operand kernel f_a[row] f_w[col] (a power of two, so the
+          // fma below still rounds once).
+          float fc[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) fc[j] = p.alpha;
+          if constexpr (kF16) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              fc[4 * j] = __fmul_rn(f_row, __shfl_sync(0xffffffffu, f_col4.x, c0 / 4 + j));
+              fc[4 * j + 1] = __fmul_rn(f_row, __shfl_sync(0xffffffffu, f_col4.y, c0 / 4 + j));
+              fc[4 * j + 2] = __fmul_rn(f_row, __shfl_sync(0xffffffffu, f_col4.z, c0 / 4 + j));
+              fc[4 * j + 3] = __fmul_rn(f_row, __shfl_sync(0xffffffffu, f_col4.w, c0 / 4 + j));
+            }
+          }
           uint32_t packed[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float y0 = __fmaf_rn(p.alpha, __uint_as_float(r[i][hh * 16 + 2 * k]), bf16_lo(bw[k]));
-            const float y1 = __fmaf_rn(p.alpha, __uint_as_float(r[i][hh * 16 + 2 * k + 1]), bf16_hi(bw[k]));
+            const float y0 = __fmaf_rn(fc[2 * k], __uint_as_float(r[i][hh * 16 + 2 * k]), bf16_lo(bw[k]));
+            const float y1 = __fmaf_rn(fc[2 * k + 1], __uint_as_float(r[i][hh * 16 + 2 * k + 1]), bf16_hi(bw[k]));
             __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
             packed[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
@@ -921,7 +964,7 @@ cudaError_t launch_pair_impl(const GemmNvfp4Params& p, const GemmPairTmaps& t, c
   if (max_pairs < 0) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (kEpi != EPI_PLAIN) {
+    if (fused_epi<kEpi>()) {
       // The epilogue warpgroups' setmaxnreg.inc waits until the third
       // warpgroup has released enough registers: only launch if the compiled
       // register count makes the split add up.
@@ -980,6 +1023,10 @@ cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPair
 cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                        bool pdl) {
   return launch_pair_impl<EPI_QKV, false>(p, t, t.a, t.a, stream, pdl);
+}
+
+cudaError_t launch_gemm_f16_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl) {
+  return launch_pair_impl<EPI_F16, false>(p, t, t.a, t.a, stream, pdl);
 }
 
 cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,

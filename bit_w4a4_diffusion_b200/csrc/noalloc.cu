@@ -68,7 +68,7 @@ int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const
                              const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
                              float weight_scale, const void* lora_up, const void* bias, void* y, int* dev_status,
                              void* stream) {
-  const long long need = svdq_workspace_bytes(precision, M, K, rank);
+  const long long need = svdq_workspace_bytes(precision, M, N, K, rank);
   if (need < 0) {
     // Let the regular entry point produce its precise shape / argument error.
     return svdq_w4a4_linear(precision, M, N, K, rank, x, inv_smooth, lora_down, act_scale, w_codes, w_scales,
@@ -76,16 +76,17 @@ int svdq_w4a4_linear_noalloc(int precision, int M, int N, int K, int rank, const
   }
   if (need > (long long)SVDQ_NOALLOC_SCRATCH_BYTES)
     return svdq::record_error(SVDQ_ERR_UNSUPPORTED_SHAPE,
-                              "M=%d K=%d needs %lld bytes of scratch; the built-in scratch holds %lld bytes "
+                              "M=%d N=%d K=%d needs %lld bytes of scratch; the built-in scratch holds %lld bytes "
                               "(use svdq_w4a4_linear with a workspace)",
-                              M, K, need, (long long)SVDQ_NOALLOC_SCRATCH_BYTES);
+                              M, N, K, need, (long long)SVDQ_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   if (int s = scratch_for_current_device(&scratch)) return s;
   // The scratch's first 64 KiB are the layer kernel's control words: zero
   // when the module is loaded (a file-scope device array starts zeroed) and
   // left zero by every call.  The rest needs no clearing: the layer writes
-  // every byte it reads (code rows < M, scale rows up to the 256-row padding,
-  // low-rank rows < M and the partial sums) before reading it.
+  // every byte it uses (code rows < M, scale rows up to the 256-row padding,
+  // low-rank rows < M, the partial sums, and for INT4 the fp16 operand rows
+  // < M and < N with their powers of two) before reading it.
   return svdq_w4a4_linear(precision, M, N, K, rank, x, inv_smooth, lora_down, act_scale, w_codes, w_scales,
                           weight_scale, lora_up, bias, y, scratch, need, dev_status, stream);
 }

@@ -390,8 +390,8 @@ SVDQ_DEV void mma_nvfp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
-// D (+)= A * B^T over the pair, M = 256, bf16 operands, fp32 accumulate; no
-// output lane disabled.
+// D (+)= A * B^T over the pair, M = 256, 16-bit operands (bf16 or fp16, as
+// the instruction descriptor says), fp32 accumulate; no output lane disabled.
 SVDQ_DEV void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
   const uint32_t z = 0;
   asm volatile(

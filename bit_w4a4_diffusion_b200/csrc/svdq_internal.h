@@ -119,6 +119,8 @@ struct GemmNvfp4Params {
   GeluQuantParams gq;         // used by the GELU-MLP epilogue only
   QkvParams qk;               // used by the QKV epilogue only
   FusedQuantParams fq;        // used by the fused layer kernel only
+  const float* row_factor;    // fp16-operand (INT4) kernel: y = bf16(D f_row[m] f_col[n] + b)
+  const float* col_factor;
 };
 
 struct GemmTmaps {
@@ -148,11 +150,32 @@ cudaError_t launch_gemm_nvfp4_pair_gelu(const GemmNvfp4Params& p, const GemmPair
                                         bool pdl);
 cudaError_t launch_gemm_nvfp4_pair_qkv(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream,
                                        bool pdl);
+// The INT4 product on fp16 operands (dequant_int4.cu): t.a / t.b map the fp16
+// [M, K] / [N, K] operands as bytes (128-byte boxes of 64 elements), t.la /
+// t.lb the scaled low-rank operands; t.sfa / t.sfb are unused.
+cudaError_t launch_gemm_f16_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, cudaStream_t stream, bool pdl);
 // The fused layer kernel (p.fq set; t.a / t.sfa / t.la map the buffers the
 // kernel itself fills).  tm_x maps x [M, K] bf16 and tm_l1 L1^T [32, K] fp16,
 // both in 64 x 128 / 64 x 32 SWIZZLE_128B boxes (the quantizer's chunks).
 cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
                                     const CUtensorMap& tm_l1, cudaStream_t stream, bool pdl);
+
+// INT4 rows -> exact fp16 operands for the fp16 tensor pipe (dequant_int4.cu):
+// out[r, k] = fp16(s[r, k/64] 2^-E[r] q[r, k]) with K permuted within every
+// 8-code word as (0, 2, 4, 6, 1, 3, 5, 7), lora_out = lora_in 2^-E[r],
+// factor[r] = 2^E[r].
+struct DequantInt4Params {
+  int R, K, R_pad;
+  const uint8_t* codes;       // [R, K/2]
+  const uint16_t* scales;     // bf16 [K/64][R_pad]
+  const uint16_t* lora_in;    // bf16 [R, 64] or null
+  uint16_t* out;              // fp16 [R, K]
+  uint16_t* lora_out;         // bf16 [R, 64] (unused when lora_in is null)
+  float* factor;              // fp32 [R]
+};
+
+size_t dequant_int4_smem_bytes(int K);
+cudaError_t launch_dequant_int4(const DequantInt4Params& p, cudaStream_t stream, bool pdl);
 
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;

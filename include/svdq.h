@@ -202,6 +202,16 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  * on `stream`: svdq_quantize_act then svdq_w4a4_gemm, the GEMM launched with
  * programmatic dependent launch so that its prologue overlaps the quantize
  * kernel's tail.
+ *  - INT4: the product runs on the fp16 tensor pipe instead of svdq_w4a4_gemm's
+ *    i8 kernel (which has no scratch): both operands are first turned into
+ *    fp16 values in the workspace, exactly sa*qa and sw*qw (an 8-bit scale
+ *    significand times a code of at most 3 bits fits fp16's 11), each row
+ *    scaled by a power of two 2^-E (E = floor(log2 of the row's largest
+ *    scale) - 12, clamped to [-100, 100]) and undone in the epilogue; exact
+ *    for every group within 2^29 of its row's largest scale.  Same products,
+ *    summed in fp32 in another order, so y can differ from quantize + gemm in
+ *    its last bits.  SVDQ_INT4_LAYER_GEMM=i8 in the environment (read at
+ *    every call) runs svdq_w4a4_gemm's kernel instead.
  *  - With SVDQ_LAYER_KERNEL=fused in the environment (read at every call;
  *    NVFP4 on the CTA-pair GEMM only): ONE kernel, whose epilogue warps
  *    quantize x themselves, 128 rows x K/splits columns at a time (splits =
@@ -214,7 +224,7 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  *    the two kernels on B200 (the quantizer's arithmetic competes with the
  *    GEMM's MMA issue) and kept for comparison.
  * `workspace` is a device buffer of at least svdq_workspace_bytes(precision,
- * M, K, rank) bytes laid out as svdq_workspace_offsets gives:
+ * M, N, K, rank) bytes laid out as svdq_workspace_offsets gives:
  *   [0]  control words of the one-kernel layer, a fixed 64 KiB at offset 0;
  *        when that layer runs they MUST BE ZERO before the first call on a
  *        workspace (e.g. a workspace from cudaMemset or torch.zeros), and
@@ -222,11 +232,17 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  *        them), so a workspace can be reused by calls of any shape without
  *        clearing it; the two-kernel path does not touch them;
  *   [1]  act codes [M, K/2];  [2] act scales;  [3] lora_act bf16 [M, 2r];
- *   [4]  fp32 low-rank partial sums (NVFP4); [5] the end (= the size).
+ *   [4]  NVFP4: the one-kernel layer's fp32 low-rank partial sums; INT4: the
+ *        fp16 operands of the product (A' [M, K], the scaled lora_act
+ *        [M, 2r], the rows' powers of two [M], then W' [N, K], the scaled
+ *        lora_up [N, 2r] and [N], each 256-byte aligned);
+ *   [5]  the end (= the size).
+ * N (the layer's output width) sizes only the INT4 region; NVFP4 accepts any
+ * N >= 0.
  * Calls that share a workspace must not overlap in time.  The one-kernel
  * layer takes M up to 1040384 (larger M runs as two kernels). */
-long long svdq_workspace_bytes(int precision, int M, int K, int rank);
-int svdq_workspace_offsets(int precision, int M, int K, int rank, long long* offsets /* [6], host */);
+long long svdq_workspace_bytes(int precision, int M, int N, int K, int rank);
+int svdq_workspace_offsets(int precision, int M, int N, int K, int rank, long long* offsets /* [6], host */);
 int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x, const float* inv_smooth,
                      const void* lora_down, float act_scale, const void* w_codes, const void* w_scales,
                      float weight_scale, const void* lora_up, const void* bias, void* y, void* workspace,
@@ -243,7 +259,7 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
  * SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB) that the CUDA driver reserves on every
  * GPU that loads the library, until the process exits.  It never calls
  * cudaMalloc, cudaFree or any allocating routine.
- *  - Limit: svdq_workspace_bytes(precision, M, K, rank) must not exceed
+ *  - Limit: svdq_workspace_bytes(precision, M, N, K, rank) must not exceed
  *    SVDQ_NOALLOC_SCRATCH_BYTES (e.g. M = 4096 tokens up to K = 9216, or
  *    2048 tokens up to K = 12288, for NVFP4); larger shapes return
  *    SVDQ_ERR_UNSUPPORTED_SHAPE with a message.

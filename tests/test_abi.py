@@ -43,8 +43,16 @@ def test_sizes():
     assert B.act_scale_bytes("nvfp4", 300, 1024) == 512 * 1024 // 16
     assert B.act_scale_bytes("int4", 300, 1024) == 512 * 1024 // 64 * 2
     assert B.act_scale_bytes(7, 300, 1024) == -1
-    assert B.workspace_bytes("nvfp4", 4096, 3072) >= 4096 * 1536 + 4096 * 192 + 4096 * 128
-    assert B.workspace_bytes("nvfp4", 4096, 3072, rank=16) == -1
+    assert B.workspace_bytes("nvfp4", 4096, 12288, 3072) >= 4096 * 1536 + 4096 * 192 + 4096 * 128
+    assert B.workspace_bytes("nvfp4", 4096, 12288, 3072, rank=16) == -1
+    # NVFP4 workspaces do not depend on N; INT4 ones hold the fp16 operands
+    # A' [M, K] and W' [N, K] besides the quantized activations.
+    assert B.workspace_bytes("nvfp4", 4096, 0, 3072) == B.workspace_bytes("nvfp4", 4096, 12288, 3072)
+    base = B.workspace_offsets("int4", 4096, 3072, 3072)
+    assert base[5] - base[4] >= (4096 + 3072) * 3072 * 2 + (4096 + 3072) * (128 + 4)
+    assert B.workspace_bytes("int4", 4096, 6144, 3072) - B.workspace_bytes("int4", 4096, 3072, 3072) == 3072 * 3072 * 2 + 3072 * 132
+    assert B.workspace_bytes("int4", 4096, 0, 3072) == -1
+    assert B.workspace_bytes("int4", 4096, 100, 3072) == -1
 
 
 FAKE = 1 << 20   # never dereferenced: every call below fails validation first
@@ -94,8 +102,8 @@ def test_gelu_mlp_sizes():
     assert B.gelu_quant_work_bytes(4096) == 4096 * 32 * 4
     assert B.gelu_quant_work_bytes(301) == 301 * 128 + (-301 * 128) % 256
     assert B.gelu_quant_work_bytes(0) == -1
-    assert B.mlp_workspace_bytes(4096, 3072, 12288) == (B.workspace_bytes("nvfp4", 4096, 3072) +
-                                                         B.workspace_bytes("nvfp4", 4096, 12288) +
+    assert B.mlp_workspace_bytes(4096, 3072, 12288) == (B.workspace_bytes("nvfp4", 4096, 12288, 3072) +
+                                                         B.workspace_bytes("nvfp4", 4096, 3072, 12288) +
                                                          B.gelu_quant_work_bytes(4096))
 
 

@@ -113,8 +113,8 @@ def test_block_layers_match_oracle(M):
     pk_d = B.svdq_pack_weights("nvfp4", idn.W_bits, idn.lam, idn.L1_bits, idn.L2_bits)
     ws = inp["workspace"]
     # the MLP's workspace: [up layer's | down layer's | work]
-    base = B.workspace_bytes("nvfp4", M, K)
-    oh = B.workspace_offsets("nvfp4", M, N)
+    base = B.workspace_bytes("nvfp4", M, N, K)
+    oh = B.workspace_offsets("nvfp4", M, K, N)
     hc = ws[base + oh[1]:base + oh[1] + M * N // 2].view(M, N // 2)
     hs = ws[base + oh[2]:base + oh[2] + B.act_scale_bytes("nvfp4", M, N)]
     hl = ws[base + oh[3]:base + oh[3] + M * 128].view(torch.bfloat16).view(M, 64)

@@ -77,7 +77,7 @@ def _check_layer_workspace(ws, c, codes, scales, lora):
     the quantize kernel's bit for bit, the low-rank activation equal up to the
     order of its fp32 sums, and the control words back at zero."""
     B = _lib()
-    off = B.workspace_offsets("nvfp4", c.M, c.K)
+    off = B.workspace_offsets("nvfp4", c.M, c.N, c.K)
     wcodes = ws[off[1]:off[1] + c.M * c.K // 2].view(c.M, c.K // 2)
     wscales = ws[off[2]:off[2] + B.act_scale_bytes("nvfp4", c.M, c.K)]
     wlora = ws[off[3]:off[3] + c.M * 128].view(torch.bfloat16).view(c.M, 64)
@@ -118,7 +118,7 @@ def test_linear_small_matches_oracle(name, kw, kernel, monkeypatch):
     x, codes, scales, lora = _run_s1(inp, w)
     alpha = float(np.float32(np.float32(inp.act_scale) * np.float32(pk["weight_scale"][0])))
     y = B.svdq_w4a4_gemm("nvfp4", codes, scales, lora, w, alpha, bias=bias)
-    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
     y2 = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
     torch.cuda.synchronize()
     _check_s1(inp, codes, scales, lora, pk)
@@ -255,7 +255,7 @@ def test_linear_full_size_sampled(name, kernel, monkeypatch):
     c = wl.SVDQ_CASES[name]
     inp, pk, w, bias = _layer(c)
     x = B.bits_to_bf16(inp.x_bits, "cuda")
-    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
     y = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
     y_again = B.svdq_w4a4_linear("nvfp4", x, w, float(inp.act_scale), bias=bias, workspace=ws)
     _, codes, scales, lora = _run_s1(inp, w)

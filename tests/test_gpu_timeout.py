@@ -212,7 +212,7 @@ def test_fused_layer_wait_timeout_reports_and_recovers(monkeypatch):
     bias = B.bits_to_bf16(inp.bias_bits, "cuda") if inp.bias_bits is not None else None
     x = B.bits_to_bf16(inp.x_bits, "cuda")
     s_a = float(inp.act_scale)
-    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.K), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(B.workspace_bytes("nvfp4", c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     old = B.get_timeout_ns()
     try:
@@ -222,7 +222,7 @@ def test_fused_layer_wait_timeout_reports_and_recovers(monkeypatch):
     finally:
         B.set_timeout_ns(old)
     assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
-    off = B.workspace_offsets("nvfp4", c.M, c.K)
+    off = B.workspace_offsets("nvfp4", c.M, c.N, c.K)
     assert int(ws[:off[1]].count_nonzero().item()) == 0, "control words not left at zero"
     status.zero_()
     y = B.svdq_w4a4_linear("nvfp4", x, w, s_a, bias=bias, workspace=ws, dev_status=status)

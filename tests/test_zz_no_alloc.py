@@ -57,7 +57,7 @@ def test_noalloc_rejects_shapes_beyond_the_scratch():
     cap = B.lib.svdq_noalloc_scratch_bytes()
     assert cap == 32 * 2 ** 20
     M, K = 8192, 12288                         # needs about 58 MB of scratch
-    assert B.workspace_bytes("nvfp4", M, K) > cap
+    assert B.workspace_bytes("nvfp4", M, 256, K) > cap
     x = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     w = {"N": 256, "K": K, "rank": 32, "weight_scale_f": 1.0,
          **{k: torch.empty(16, dtype=torch.uint8, device="cuda")
