@@ -42,10 +42,13 @@
 // q exactly; one fp16 multiply by the scaled group scale gives the value
 // (exact, see above).  Two codes per packed f16x2 operation.
 //
-// One CTA of 256 threads per 16 rows: the rows' scales are staged in shared
-// memory (group-major, so a group's 16 row scales are one 32-byte read), the
-// row exponents come from them, then each thread turns 16 bytes of codes into
-// 64 bytes of fp16 at a time, consecutive threads along a row (coalesced).
+// One CTA of 128 threads per 8 rows, 16 threads per row: thread (r, l)
+// takes the 16-byte code chunks l, l + 16, l + 32, ... of row r (a row's 16
+// threads read 256 contiguous bytes per step), issuing the loads of up to
+// eight chunks before it converts any, so that enough bytes are in flight to
+// cover the memory latency.  The rows' scales are staged in shared memory
+// (group-major, so a group's 8 row scales are one 16-byte read) and each
+// row's largest scale is a max over its 16 threads.
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -55,8 +58,10 @@
 namespace svdq {
 namespace {
 
-constexpr int DQ_ROWS = 16;
-constexpr int DQ_THREADS = 256;
+constexpr int DQ_ROWS = 8;
+constexpr int DQ_TPR = 16;                         // threads per row
+constexpr int DQ_THREADS = DQ_ROWS * DQ_TPR;
+constexpr int DQ_BATCH = 8;                        // chunk loads in flight per thread
 
 SVDQ_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
@@ -99,68 +104,82 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
   extern __shared__ float dq_smem[];
   const int groups = p.K / 64;
   float* sc = dq_smem;                          // [groups][DQ_ROWS]
-  float* inv = dq_smem + groups * DQ_ROWS;      // [DQ_ROWS]: 2^-E[r]
   const int r0 = blockIdx.x * DQ_ROWS;
   const int tid = threadIdx.x;
+  const int r = tid / DQ_TPR, l = tid % DQ_TPR;
+  const int row = r0 + r;
+  const bool row_ok = row < p.R;
   pdl_wait();
   pdl_launch_dependents();
 
   // Scales of the CTA's rows (rows past R read the zero padding: R_pad is a
   // multiple of 256 and r0 + DQ_ROWS <= R_pad).
   for (int i = tid; i < groups * DQ_ROWS; i += DQ_THREADS) {
-    const int g = i / DQ_ROWS, r = i - g * DQ_ROWS;
-    sc[i] = __bfloat162float(__ushort_as_bfloat16(p.scales[(size_t)g * p.R_pad + r0 + r]));
+    const int g = i / DQ_ROWS, rr = i - g * DQ_ROWS;
+    sc[i] = __bfloat162float(__ushort_as_bfloat16(p.scales[(size_t)g * p.R_pad + r0 + rr]));
   }
   __syncthreads();
-  if (tid < DQ_ROWS) {
-    float mx = 0.f;
-    for (int g = 0; g < groups; ++g) mx = fmaxf(mx, sc[g * DQ_ROWS + tid]);
-    int e = 0;
-    if (mx > 0.f) {
-      const int biased = (__float_as_int(mx) >> 23) & 0xFF;   // 0 for an fp32 subnormal
-      e = (biased == 0 ? -126 : biased - 127) - 12;
-      e = e < -100 ? -100 : (e > 100 ? 100 : e);
-    }
-    inv[tid] = exp2i(-e);
-    if (r0 + tid < p.R) p.factor[r0 + tid] = exp2i(e);
-  }
-  __syncthreads();
-
-  // Codes: 16 bytes (32 codes, all in one 64-group) per step.
-  const int chunks = p.K / 32;
-  for (int i = tid; i < DQ_ROWS * chunks; i += DQ_THREADS) {
-    const int r = i / chunks, j = i - r * chunks;
-    const int row = r0 + r;
-    if (row >= p.R) break;   // rows are visited in order: the rest are past R too
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.codes + (size_t)row * (p.K / 2)) + j);
-    // The scaled group scale: exact in fp32 (a power-of-two factor), then in
-    // fp16 for every group within 2^29 of the row's largest.
-    const uint32_t s2 = f32_to_f16x2_dup(__fmul_rn(sc[(j >> 1) * DQ_ROWS + r], inv[r]));
-    uint32_t o[4][4];
-    dequant_word(w.x, s2, o[0]);
-    dequant_word(w.y, s2, o[1]);
-    dequant_word(w.z, s2, o[2]);
-    dequant_word(w.w, s2, o[3]);
-    uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.K) + 4 * j;
+  // The row's largest scale: each of its 16 threads takes every 16th group.
+  float mx = 0.f;
+  for (int g = l; g < groups; g += DQ_TPR) mx = fmaxf(mx, sc[g * DQ_ROWS + r]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+  for (int o = DQ_TPR / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  int e = 0;
+  if (mx > 0.f) {
+    const int biased = (__float_as_int(mx) >> 23) & 0xFF;   // 0 for an fp32 subnormal
+    e = (biased == 0 ? -126 : biased - 127) - 12;
+    e = e < -100 ? -100 : (e > 100 ? 100 : e);
   }
+  const float inv = exp2i(-e);
+  if (row_ok && l == 0) p.factor[row] = exp2i(e);
 
-  // The low-rank operand rows, scaled by the same power of two.
-  if (p.lora_in != nullptr) {
-    for (int i = tid; i < DQ_ROWS * 64; i += DQ_THREADS) {
-      const int r = i >> 6, c = i & 63;
-      const int row = r0 + r;
-      if (row >= p.R) break;
-      const float v = __bfloat162float(__ushort_as_bfloat16(p.lora_in[(size_t)row * 64 + c]));
-      p.lora_out[(size_t)row * 64 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, inv[r])));
+  if (row_ok) {
+    // Codes: 16 bytes (32 codes, all in one 64-group) per chunk.
+    const int chunks = p.K / 32;
+    const uint4* src = reinterpret_cast<const uint4*>(p.codes + (size_t)row * (p.K / 2));
+    uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.K);
+    for (int j0 = l; j0 < chunks; j0 += DQ_TPR * DQ_BATCH) {
+      uint4 w[DQ_BATCH];
+#pragma unroll
+      for (int b = 0; b < DQ_BATCH; ++b) {
+        const int j = j0 + DQ_TPR * b;
+        if (j < chunks) w[b] = __ldg(src + j);
+      }
+#pragma unroll
+      for (int b = 0; b < DQ_BATCH; ++b) {
+        const int j = j0 + DQ_TPR * b;
+        if (j < chunks) {
+          // The scaled group scale: exact in fp32 (a power-of-two factor),
+          // then in fp16 for every group within 2^29 of the row's largest.
+          const uint32_t s2 = f32_to_f16x2_dup(__fmul_rn(sc[(j >> 1) * DQ_ROWS + r], inv));
+          uint32_t o[4][4];
+          dequant_word(w[b].x, s2, o[0]);
+          dequant_word(w[b].y, s2, o[1]);
+          dequant_word(w[b].z, s2, o[2]);
+          dequant_word(w[b].w, s2, o[3]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[4 * j + q] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+        }
+      }
+    }
+    // The low-rank operand row, scaled by the same power of two: four
+    // values per thread.
+    if (p.lora_in != nullptr) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.lora_in + (size_t)row * 64) + l);
+      auto scale2 = [&](uint32_t b) {
+        const float lo = __fmul_rn(__uint_as_float(b << 16), inv);
+        const float hi = __fmul_rn(__uint_as_float(b & 0xFFFF0000u), inv);
+        return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+      };
+      reinterpret_cast<uint2*>(p.lora_out + (size_t)row * 64)[l] = make_uint2(scale2(v.x), scale2(v.y));
     }
   }
 }
 
 }  // namespace
 
-size_t dequant_int4_smem_bytes(int K) { return (size_t)((K / 64) * DQ_ROWS + DQ_ROWS) * sizeof(float); }
+size_t dequant_int4_smem_bytes(int K) { return (size_t)(K / 64) * DQ_ROWS * sizeof(float); }
 
 cudaError_t launch_dequant_int4(const DequantInt4Params& p, cudaStream_t stream, bool pdl) {
   const size_t smem = dequant_int4_smem_bytes(p.K);
