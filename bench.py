@@ -542,17 +542,20 @@ def measure_rows(B, wl, dev, peaks):
         wsp = torch.zeros(B.workspace_bytes("int4", M, c.N, c.K), dtype=torch.uint8, device=dev)
         fns = [lambda i=i: B.svdq_w4a4_linear("int4", x, ws[i], 1.0, y=ys[i], workspace=wsp) for i in range(nset)]
         t = _event_time_us(torch, fns, 40)
-        # The same layer with svdq_w4a4_gemm's i8 kernel (for comparison).
-        os.environ["SVDQ_INT4_LAYER_GEMM"] = "i8"
-        try:
-            t8 = _event_time_us(torch, fns, 40)
-        finally:
-            del os.environ["SVDQ_INT4_LAYER_GEMM"]
+        # The same layer with the other two GEMM options (for comparison).
+        alt = {}
+        for opt in ("dq", "i8"):
+            os.environ["SVDQ_INT4_LAYER_GEMM"] = opt
+            try:
+                alt[opt] = _event_time_us(torch, fns, 40)
+            finally:
+                del os.environ["SVDQ_INT4_LAYER_GEMM"]
         int4[f"M={M}"] = {"us": round(t, 2), "TOPS": round(2.0 * M * c.N * c.K / t / 1e6, 1),
-                          "i8_gemm_us": round(t8, 2)}
+                          "dq_in_gemm_us": round(alt["dq"], 2), "i8_gemm_us": round(alt["i8"], 2)}
         del ws, ys
-    int4["what"] = ("svdq_w4a4_linear INT4: quantize, fp16 operands of both sides, CTA-pair fp16 GEMM; "
-                    "i8_gemm_us: the same layer on the i8 kernel of svdq_w4a4_gemm")
+    int4["what"] = ("svdq_w4a4_linear INT4: quantize, both operands written out in fp16 (one launch), CTA-pair "
+                    "fp16 GEMM; dq_in_gemm_us: the GEMM building its fp16 operand tiles from the codes itself; "
+                    "i8_gemm_us: the i8 kernel of svdq_w4a4_gemm")
     rows["svdq_w4a4 int4 K=N=3072"] = int4
     rows["hbm_read_reference"] = measure_read_reference(dev, peaks)
     rows["mlp_gelu"] = measure_mlp(B, wl, dev)

@@ -23,7 +23,7 @@ NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-
 CXX_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-ffp-contract=off", "-pthread", "-I", INCLUDE,
              "-I", "/usr/local/cuda/include"]
 
-CU_SOURCES = ["abi.cu", "quantize_act.cu", "quantize_nvfp4.cu", "gemm_nvfp4.cu", "gemm_nvfp4_pair.cu", "gemm_int4.cu", "dequant_int4.cu", "awq_gemm.cu", "noalloc.cu"]
+CU_SOURCES = ["abi.cu", "quantize_act.cu", "quantize_nvfp4.cu", "gemm_nvfp4.cu", "gemm_nvfp4_pair.cu", "gemm_int4.cu", "gemm_int4_pair.cu", "dequant_int4.cu", "awq_gemm.cu", "noalloc.cu"]
 CXX_SOURCES = ["pack.cpp", "calib.cpp"]
 
 

@@ -493,21 +493,28 @@ static int gemm_int4_impl(int M, int N, int K, const void* act_codes, const void
   return check_cuda(launch_gemm_int4(p, t, sms, stream, pdl), "gemm_int4 launch");
 }
 
-// The INT4 layer's product on the fp16 tensor pipe: both operands turned into
-// exact fp16 values (dequant_int4.cu) in the workspace region `region`, then
-// the CTA-pair GEMM with kind::f16 MMAs and one accumulator per tile.  The
-// i8 kernel (gemm_int4.cu) needs no scratch and stays the GEMM of
-// svdq_w4a4_gemm; SVDQ_INT4_LAYER_GEMM=i8 (read at every call) runs it in
-// the layer too, for comparison.  Both sum the same exact products in fp32.
-static bool use_int4_i8_gemm() {
+// The INT4 layer's product on the fp16 tensor pipe, from exact fp16 values of
+// both operands (dequant_int4.cu).  By default both operands are written out
+// in fp16 to the workspace region first (one launch for both), then the NVFP4
+// pair kernel runs its fp16 path.  SVDQ_INT4_LAYER_GEMM (read at every call)
+// selects instead "dq": the CTA-pair kernel of gemm_int4_pair.cu, which
+// builds the fp16 operand tiles itself in shared memory, slice by slice, from
+// the codes (the same values and MMAs, so the same y bit for bit; slower on
+// B200: 229 against 105 us at M = 4096, K = N = 3072); or "i8":
+// svdq_w4a4_gemm's kernel (gemm_int4.cu, which needs no scratch).  All sum
+// the same exact products in fp32.
+enum class Int4LayerGemm { kF16Operands, kDequantInGemm, kI8 };
+static Int4LayerGemm int4_layer_gemm() {
   const char* v = getenv("SVDQ_INT4_LAYER_GEMM");
-  return v && strcmp(v, "i8") == 0;
+  if (v && strcmp(v, "i8") == 0) return Int4LayerGemm::kI8;
+  if (v && strcmp(v, "dq") == 0) return Int4LayerGemm::kDequantInGemm;
+  return Int4LayerGemm::kF16Operands;
 }
 
 static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const void* act_scales,
                               const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
                               const void* bias, void* y, uint8_t* region, int* dev_status, cudaStream_t stream,
-                              bool pdl) {
+                              bool pdl, bool in_gemm) {
   long long o[7];
   int4_operand_offsets(M, N, K, o);
   uint16_t* a16 = reinterpret_cast<uint16_t*>(region + o[0]);
@@ -516,6 +523,44 @@ static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const 
   uint16_t* w16 = reinterpret_cast<uint16_t*>(region + o[3]);
   uint16_t* lb = reinterpret_cast<uint16_t*>(region + o[4]);
   float* fw = reinterpret_cast<float*>(region + o[5]);
+  if (in_gemm) {
+    // The rows' powers of two and the scaled low-rank operands only; the GEMM
+    // builds the fp16 operand tiles from the codes.
+    GemmInt4DqTmaps t;
+    bool ok = true;
+    ok &= encode_tmap_2d(&t.a4, CU_TENSOR_MAP_DATA_TYPE_UINT8, act_codes, K / 2, M, K / 2, 32, 128,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= encode_tmap_2d(&t.b4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 32, 128,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= encode_tmap_2d(&t.la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, 2 * SVDQ_RANK, M, 2 * SVDQ_RANK * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= encode_tmap_2d(&t.lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lb, 2 * SVDQ_RANK, N, 2 * SVDQ_RANK * 2, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= encode_tmap_2d(&t.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, (uint64_t)N * 2, 16, 32,
+                         CU_TENSOR_MAP_SWIZZLE_32B);
+    if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the INT4 pair GEMM");
+    DequantInt4Params fw_p{N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
+                           static_cast<const uint16_t*>(w_scales), static_cast<const uint16_t*>(lora_up), nullptr, lb,
+                           fw};
+    DequantInt4Params fa_p{M, K, (int)round_up(M, 256), static_cast<const uint8_t*>(act_codes),
+                           static_cast<const uint16_t*>(act_scales), static_cast<const uint16_t*>(lora_act), nullptr,
+                           la, fa};
+    if (int s = check_cuda(launch_dequant_int4(fw_p, fa_p, stream, pdl), "INT4 row factors launch")) return s;
+    GemmInt4DqParams q{};
+    q.M = M;
+    q.N = N;
+    q.K = K;
+    q.M_pad = (int)round_up(M, 256);
+    q.N_pad = (int)round_up(N, 256);
+    q.act_scales = static_cast<const uint16_t*>(act_scales);
+    q.w_scales = static_cast<const uint16_t*>(w_scales);
+    q.bias = static_cast<const uint16_t*>(bias);
+    q.row_factor = fa;
+    q.col_factor = fw;
+    q.dev_status = dev_status;
+    q.timeout_ns = svdq_timeout_ns();
+    return check_cuda(launch_gemm_int4_pair(q, t, stream, pdl), "gemm_int4_pair launch");
+  }
   GemmPairTmaps u;
   bool ok = true;
   ok &= encode_tmap_2d(&u.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a16, (uint64_t)K * 2, M, (uint64_t)K * 2, 128, 128,
@@ -535,8 +580,7 @@ static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const 
                        static_cast<const uint16_t*>(act_scales), static_cast<const uint16_t*>(lora_act), a16, la, fa};
   DequantInt4Params dw{N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
                        static_cast<const uint16_t*>(w_scales), static_cast<const uint16_t*>(lora_up), w16, lb, fw};
-  if (int s = check_cuda(launch_dequant_int4(dw, stream, pdl), "dequant_int4 (weights) launch")) return s;
-  if (int s = check_cuda(launch_dequant_int4(da, stream, pdl), "dequant_int4 (activations) launch")) return s;
+  if (int s = check_cuda(launch_dequant_int4(dw, da, stream, pdl), "dequant_int4 launch")) return s;
   GemmNvfp4Params p{};
   p.M = M;
   p.N = N;
@@ -689,11 +733,13 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
                                 scales, lora, dev_status, stream))
     return s;
   if (precision == SVDQ_INT4) {
-    if (use_int4_i8_gemm())
+    const Int4LayerGemm g = int4_layer_gemm();
+    if (g == Int4LayerGemm::kI8)
       return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
                             static_cast<cudaStream_t>(stream), pdl_on(), sms);
     return gemm_int4_f16_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, ws + off[4],
-                              dev_status, static_cast<cudaStream_t>(stream), pdl_on());
+                              dev_status, static_cast<cudaStream_t>(stream), pdl_on(),
+                              g == Int4LayerGemm::kDequantInGemm);
   }
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);

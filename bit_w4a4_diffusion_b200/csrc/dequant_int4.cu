@@ -42,7 +42,9 @@
 // q exactly; one fp16 multiply by the scaled group scale gives the value
 // (exact, see above).  Two codes per packed f16x2 operation.
 //
-// One CTA of 128 threads per 8 rows, 16 threads per row: thread (r, l)
+// One launch converts both operands (the weight rows first, then the
+// activation rows: one grid, so the two passes share a single ramp-up and
+// tail).  One CTA of 128 threads per 8 rows, 16 threads per row: thread (r, l)
 // takes the 16-byte code chunks l, l + 16, l + 32, ... of row r (a row's 16
 // threads read 256 contiguous bytes per step), issuing the loads of up to
 // eight chunks before it converts any, so that enough bytes are in flight to
@@ -100,11 +102,14 @@ SVDQ_DEV void dequant_word(uint32_t w, uint32_t s2, uint32_t (&o)[4]) {
   o[3] = hmul2_rn(hsub2_rn(prmt(hi, kMagic, 0x4342u), kBias), s2);
 }
 
-__global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Params p) {
+__global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Params pw, DequantInt4Params pa) {
   extern __shared__ float dq_smem[];
+  const int blocks_w = (pw.R + DQ_ROWS - 1) / DQ_ROWS;
+  const bool is_w = (int)blockIdx.x < blocks_w;
+  const DequantInt4Params p = is_w ? pw : pa;
   const int groups = p.K / 64;
   float* sc = dq_smem;                          // [groups][DQ_ROWS]
-  const int r0 = blockIdx.x * DQ_ROWS;
+  const int r0 = ((int)blockIdx.x - (is_w ? 0 : blocks_w)) * DQ_ROWS;
   const int tid = threadIdx.x;
   const int r = tid / DQ_TPR, l = tid % DQ_TPR;
   const int row = r0 + r;
@@ -133,7 +138,7 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
   const float inv = exp2i(-e);
   if (row_ok && l == 0) p.factor[row] = exp2i(e);
 
-  if (row_ok) {
+  if (row_ok && p.out != nullptr) {
     // Codes: 16 bytes (32 codes, all in one 64-group) per chunk.
     const int chunks = p.K / 32;
     const uint4* src = reinterpret_cast<const uint4*>(p.codes + (size_t)row * (p.K / 2));
@@ -162,6 +167,8 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
         }
       }
     }
+  }
+  if (row_ok) {
     // The low-rank operand row, scaled by the same power of two: four
     // values per thread.
     if (p.lora_in != nullptr) {
@@ -181,20 +188,21 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
 
 size_t dequant_int4_smem_bytes(int K) { return (size_t)(K / 64) * DQ_ROWS * sizeof(float); }
 
-cudaError_t launch_dequant_int4(const DequantInt4Params& p, cudaStream_t stream, bool pdl) {
-  const size_t smem = dequant_int4_smem_bytes(p.K);
+cudaError_t launch_dequant_int4(const DequantInt4Params& pw, const DequantInt4Params& pa, cudaStream_t stream,
+                                bool pdl) {
+  const size_t smem = dequant_int4_smem_bytes(pw.K);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(dequant_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((p.R + DQ_ROWS - 1) / DQ_ROWS));
+  cfg.gridDim = dim3((unsigned)((pw.R + DQ_ROWS - 1) / DQ_ROWS + (pa.R + DQ_ROWS - 1) / DQ_ROWS));
   cfg.blockDim = dim3(DQ_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   set_pdl(cfg, attr, pdl);
-  return cudaLaunchKernelEx(&cfg, dequant_int4_kernel, p);
+  return cudaLaunchKernelEx(&cfg, dequant_int4_kernel, pw, pa);
 }
 
 }  // namespace svdq

@@ -169,13 +169,38 @@ struct DequantInt4Params {
   const uint8_t* codes;       // [R, K/2]
   const uint16_t* scales;     // bf16 [K/64][R_pad]
   const uint16_t* lora_in;    // bf16 [R, 64] or null
-  uint16_t* out;              // fp16 [R, K]
+  uint16_t* out;              // fp16 [R, K], or null: only factor and lora_out
   uint16_t* lora_out;         // bf16 [R, 64] (unused when lora_in is null)
   float* factor;              // fp32 [R]
 };
 
 size_t dequant_int4_smem_bytes(int K);
-cudaError_t launch_dequant_int4(const DequantInt4Params& p, cudaStream_t stream, bool pdl);
+// One launch for both operands (pw: weight rows, pa: activation rows; same K).
+cudaError_t launch_dequant_int4(const DequantInt4Params& pw, const DequantInt4Params& pa, cudaStream_t stream,
+                                bool pdl);
+
+// The INT4 layer's product with the fp16 operands built inside the GEMM
+// (gemm_int4_pair.cu): a4 / b4 map the packed codes [M, K/2] / [N, K/2] in
+// 32-byte x 128-row boxes, la / lb the scaled low-rank operands (bf16
+// [rows, 64], 64 x 128 SWIZZLE_128B boxes), y the output (16 x 32 boxes,
+// 32-byte swizzle).
+struct GemmInt4DqParams {
+  int M, N, K, M_pad, N_pad;
+  const uint16_t* act_scales;  // bf16 [K/64][M_pad]
+  const uint16_t* w_scales;    // bf16 [K/64][N_pad]
+  const uint16_t* bias;        // bf16 [N] or null
+  const float* row_factor;     // 2^Ea [M]
+  const float* col_factor;     // 2^Ew [N]
+  int* dev_status;
+  unsigned long long timeout_ns;
+};
+
+struct GemmInt4DqTmaps {
+  CUtensorMap a4, b4, la, lb, y;
+};
+
+cudaError_t launch_gemm_int4_pair(const GemmInt4DqParams& p, const GemmInt4DqTmaps& t, cudaStream_t stream,
+                                  bool pdl);
 
 struct GemmInt4Params {
   int M, N, K, M_pad, N_pad;

@@ -203,15 +203,17 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  * programmatic dependent launch so that its prologue overlaps the quantize
  * kernel's tail.
  *  - INT4: the product runs on the fp16 tensor pipe instead of svdq_w4a4_gemm's
- *    i8 kernel (which has no scratch): both operands are first turned into
- *    fp16 values in the workspace, exactly sa*qa and sw*qw (an 8-bit scale
- *    significand times a code of at most 3 bits fits fp16's 11), each row
- *    scaled by a power of two 2^-E (E = floor(log2 of the row's largest
- *    scale) - 12, clamped to [-100, 100]) and undone in the epilogue; exact
- *    for every group within 2^29 of its row's largest scale.  Same products,
+ *    i8 kernel (which has no scratch): both operands are first written out
+ *    to the workspace as fp16 values, exactly sa*qa and sw*qw (an 8-bit
+ *    scale significand times a code of at most 3 bits fits fp16's 11), each
+ *    row scaled by a power of two 2^-E (E = floor(log2 of the row's largest
+ *    scale) - 12, clamped to [-100, 100]) that the epilogue undoes; exact for
+ *    every group within 2^29 of its row's largest scale.  Same products,
  *    summed in fp32 in another order, so y can differ from quantize + gemm in
- *    its last bits.  SVDQ_INT4_LAYER_GEMM=i8 in the environment (read at
- *    every call) runs svdq_w4a4_gemm's kernel instead.
+ *    its last bits.  SVDQ_INT4_LAYER_GEMM in the environment (read at every
+ *    call) selects "dq" (the GEMM builds the fp16 tiles itself in shared
+ *    memory; the same y bit for bit, slower) or "i8" (svdq_w4a4_gemm's
+ *    kernel).
  *  - With SVDQ_LAYER_KERNEL=fused in the environment (read at every call;
  *    NVFP4 on the CTA-pair GEMM only): ONE kernel, whose epilogue warps
  *    quantize x themselves, 128 rows x K/splits columns at a time (splits =
@@ -235,7 +237,8 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  *   [4]  NVFP4: the one-kernel layer's fp32 low-rank partial sums; INT4: the
  *        fp16 operands of the product (A' [M, K], the scaled lora_act
  *        [M, 2r], the rows' powers of two [M], then W' [N, K], the scaled
- *        lora_up [N, 2r] and [N], each 256-byte aligned);
+ *        lora_up [N, 2r] and [N], each 256-byte aligned; A' and W' are
+ *        not written with SVDQ_INT4_LAYER_GEMM=dq);
  *   [5]  the end (= the size).
  * N (the layer's output width) sizes only the INT4 region; NVFP4 accepts any
  * N >= 0.

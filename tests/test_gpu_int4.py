@@ -1,9 +1,12 @@
 """GPU parity: the CUDA SVDQuant W4A4 INT4 path against the CPU oracle.  S1
-(INT4 quantize): activation codes and bf16 group scales bit-exact.  S3 two
-ways: svdq_w4a4_gemm's i8 tcgen05 kernel, and the layer's product on the fp16
-tensor pipe, whose fp16 operands must be exactly the oracle's dequantized
-values (scaled by the documented power of two per row).  Outputs within the
-layer bound; every output row checked."""
+(INT4 quantize): activation codes and bf16 group scales bit-exact.  S3 three
+ways: svdq_w4a4_gemm's i8 tcgen05 kernel; the layer's default, the fp16
+tensor pipe on fp16 operands written out first, whose values must be exactly
+the oracle's dequantized codes (scaled by the documented power of two per
+row); and the same product with the fp16 operand tiles built inside the
+GEMM.  The two fp16 paths issue the same MMAs on the same values and must
+agree bit for bit.  Outputs within the layer bound; every output row
+checked."""
 import numpy as np
 import pytest
 import torch
@@ -24,6 +27,7 @@ CASES = [
     ("int4_m1024", dict(M=300, N=512)),                 # ragged M
     ("int4_m1024", dict(M=129, N=256, K=1024)),
     ("int4_m1024", dict(M=1, N=128, K=256)),             # one token, one tile
+    ("int4_m1024", dict(M=130, N=384, K=512)),           # half of the last 256-column tile past N
     ("int4_m1024", {}),
     ("int4_m2048", {}),
     ("int4_m4096", {}),
@@ -43,9 +47,11 @@ def test_int4_linear_matches_oracle(name, kw):
     x = B.bits_to_bf16(inp.x_bits, "cuda")
     codes, scales, lora = B.svdq_quantize_act("int4", x, w["inv_smooth"], w["lora_down"], 1.0, 1.0)
     y = B.svdq_w4a4_gemm("int4", codes, scales, lora, w, 1.0)
-    y2 = B.svdq_w4a4_linear("int4", x, w, 1.0)              # fp16-operand product
+    y2 = B.svdq_w4a4_linear("int4", x, w, 1.0)              # fp16 operands written out first
     with _env("SVDQ_INT4_LAYER_GEMM", "i8"):
         y3 = B.svdq_w4a4_linear("int4", x, w, 1.0)          # the i8 kernel
+    with _env("SVDQ_INT4_LAYER_GEMM", "dq"):
+        y4 = B.svdq_w4a4_linear("int4", x, w, 1.0)          # fp16 tiles built in the GEMM
     torch.cuda.synchronize()
     ref_pw = O.pack_weights("int4", inp.W, inp.lam, inp.L1, inp.L2)
     act = O.quantize_activations("int4", inp.x, ref_pw["inv_lam"])
@@ -61,6 +67,7 @@ def test_int4_linear_matches_oracle(name, kw):
     assert_output_close(y.float().cpu().numpy(), y64, f"{c.name} int4")
     assert_output_close(y2.float().cpu().numpy(), y64, f"{c.name} int4 (fp16 operands)")
     assert torch.equal(y, y3)
+    assert torch.equal(y2, y4), "the two fp16 paths differ"
     # Both products sum the same exact terms in fp32, in different orders:
     # they differ by fp32 rounding (a few 2^-24 of the terms' magnitudes, far
     # below 2^-12 of the output's largest) and then by at most one bf16 step.
@@ -120,8 +127,9 @@ def _unpermute(a16):
 def test_int4_fp16_operands_are_the_oracle_values(name, kw, zero_row):
     """The layer's fp16 operands (workspace region [4]) against the oracle's
     codes and scales, bit for bit: A' from the activation quantizer, W' from
-    the weight pack, and the rows' powers of two.  A row of x set to zero
-    checks the zero-row case (factor 1, all values +0)."""
+    the weight pack, and the rows' powers of two (which the "dq" option
+    computes the same way).  A row of
+    x set to zero checks the zero-row case (factor 1, all values +0)."""
     import bit_w4a4_diffusion_b200 as B
     c = wl.SVDQ_CASES[name]
     if kw:
@@ -137,7 +145,10 @@ def test_int4_fp16_operands_are_the_oracle_values(name, kw, zero_row):
     x = B.bits_to_bf16(x_bits, "cuda")
     ws = torch.zeros(B.workspace_bytes("int4", c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
     y = B.svdq_w4a4_linear("int4", x, w, 1.0, workspace=ws)
+    with _env("SVDQ_INT4_LAYER_GEMM", "dq"):
+        y_dq = B.svdq_w4a4_linear("int4", x, w, 1.0)
     torch.cuda.synchronize()
+    assert torch.equal(y, y_dq), "the two fp16 paths differ"
     off = B.workspace_offsets("int4", c.M, c.N, c.K)
     region = ws[off[4]:off[5]].cpu().numpy()
 
