@@ -133,7 +133,14 @@ SVDQ_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-constexpr int S1_PREFETCH = 2;
+// Units whose copies are in flight per warp.  The ring holds PREFETCH x STEP
+// slots of 6 x 16 bytes per thread: 96 KB per CTA for NVFP4 with two units,
+// 96 KB for INT4 (two 32-blocks per unit) with one.  At two units INT4 would
+// take 192 KB, one CTA per SM, and the 256 CTAs of a 4096-row activation two
+// waves; with one, two CTAs fit on every SM and the warps of the other CTA
+// cover a warp's memory round trip.
+template <bool kNvfp4>
+constexpr int s1_prefetch() { return kNvfp4 ? 2 : 1; }
 // Slot contents per 32-wide block: x rows g and g+8 (2 x 16 B), then the four
 // L1^T fragments of the lane (4 x 16 B).
 constexpr int S1_SLOT_U4 = 6;
@@ -141,6 +148,7 @@ constexpr int S1_SLOT_U4 = 6;
 template <bool kNvfp4>
 __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActParams p) {
   constexpr int STEP = kNvfp4 ? 1 : 2;  // 32-blocks per unit (INT4 group = 64)
+  constexpr int S1_PREFETCH = s1_prefetch<kNvfp4>();
   extern __shared__ uint4 s1_ring[];     // [PREFETCH][STEP][SLOT_U4][THREADS]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -361,7 +369,8 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl) {
   const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
   dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS);
-  const size_t ring_bytes = (size_t)S1_PREFETCH * (nvfp4 ? 1 : 2) * S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
+  const size_t ring_bytes = (size_t)(nvfp4 ? s1_prefetch<true>() : s1_prefetch<false>()) * (nvfp4 ? 1 : 2) *
+                            S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(S1_THREADS);
