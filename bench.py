@@ -41,14 +41,18 @@ L2_BYTES = 126 * 2 ** 20
 # SHA-256 of the kernel sources it was taken from: once a source changes the
 # figure no longer applies and the bench reports null.
 GEMM_TRAFFIC = {
-    "bytes": 30466560 + 51553792,
+    "bytes": 30486272 + 52263168,
     "sources": {
         "bit_w4a4_diffusion_b200/csrc/gemm_nvfp4_pair.cu":
-            "d563a192a133c5c5fd1bfebc29eafbbac85b0c05f19dbd55a65ec2ba4ce95bee",
+            "970105a4508e7e73ae94d34360d31df5931e56a058275e65edbaeac82990a07b",
         "bit_w4a4_diffusion_b200/csrc/epilogue.cuh":
             "c18b2678b535744d65b902ff8a6fbea589e0eb0a94e9e56de6a7c73e243609d9",
         "bit_w4a4_diffusion_b200/csrc/ptx.cuh":
-            "184c8282cd62329003ff02d6229c85f8fd484990a2c956a6aaa2e49c17d1a9ee",
+            "d0ae4c9c0226adbd9ca9b7e6557ba21e131287ed65767747f8c97e2702b61e1e",
+        "bit_w4a4_diffusion_b200/csrc/fused_quant.cuh":
+            "f21ab85bdbe311d3d4165dcdeb812572d29a3cf396e766fb4835a66c8d267e4b",
+        "bit_w4a4_diffusion_b200/csrc/svdq_internal.h":
+            "caf820c4f487524424ab25f7913de95e9cc45ec6d451543bdbf6b4bf2183370b",
     },
 }
 

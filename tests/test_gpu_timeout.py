@@ -85,6 +85,40 @@ def test_int4_gemm_wait_timeout_reports_and_recovers():
     assert_output_close(y.float().cpu().numpy(), y64, "INT4 GEMM after a timed-out call")
 
 
+@pytest.mark.parametrize("option", ["default", "dq"])
+def test_int4_layer_wait_timeout_reports_and_recovers(option, monkeypatch):
+    """The INT4 layer's own GEMMs (the pair kernel on fp16 operands, and the
+    one that builds the fp16 tiles itself) report a timed-out wait and leave
+    the library usable."""
+    import bit_w4a4_diffusion_b200 as B
+    if option != "default":
+        monkeypatch.setenv("SVDQ_INT4_LAYER_GEMM", option)
+    c = wl.SVDQ_CASES["int4_m4096"]
+    inp = svdq_inputs(c)
+    pk = B.svdq_pack_weights("int4", inp.W_bits, inp.lam, inp.L1_bits, inp.L2_bits)
+    w = B.to_device(pk)
+    x = B.bits_to_bf16(inp.x_bits, "cuda")
+    ws = torch.zeros(B.workspace_bytes("int4", c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    old = B.get_timeout_ns()
+    try:
+        B.set_timeout_ns(1)
+        B.svdq_w4a4_linear("int4", x, w, 1.0, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+    finally:
+        B.set_timeout_ns(old)
+    assert int(status.item()) in TIMEOUT_CODES, f"no timeout reported (status {int(status.item())})"
+
+    status.zero_()
+    y = B.svdq_w4a4_linear("int4", x, w, 1.0, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_pw = O.pack_weights("int4", inp.W, inp.lam, inp.L1, inp.L2)
+    act = O.quantize_activations("int4", inp.x, ref_pw["inv_lam"])
+    y64 = O.linear_f64("int4", act, ref_pw, inp.L1, inp.L2, inp.bias)
+    assert_output_close(y.float().cpu().numpy(), y64, f"INT4 layer ({option}) after a timed-out call")
+
+
 @pytest.mark.parametrize("kernel", ["single", "pair"])
 def test_gelu_mlp_gemm_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     """The GELU-MLP kernel (eight epilogue warps that stop together)."""
