@@ -130,14 +130,14 @@ def workload_config(M, K, N, world):
 
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_offline(inp):
+def oracle_offline(inp, precision="nvfp4"):
     """The oracle's offline weight pack and weight dequantization (untimed)."""
     from oracle import svdq as O
-    pw = O.pack_weights("nvfp4", inp.W, inp.lam, inp.L1, inp.L2)
-    return pw, O.dequantized_weight("nvfp4", pw)
+    pw = O.pack_weights(precision, inp.W, inp.lam, inp.L1, inp.L2)
+    return pw, O.dequantized_weight(precision, pw)
 
 
-def oracle_step_fn(case, inp, rows_per_step, offline):
+def oracle_step_fn(case, inp, rows_per_step, offline, precision="nvfp4"):
     """Per step: the oracle's activation quantization and fp64 layer output for
     `rows_per_step` rows (cycling through x)."""
     from oracle import svdq as O
@@ -145,13 +145,14 @@ def oracle_step_fn(case, inp, rows_per_step, offline):
     L1 = inp.L1.astype(np.float64)
     L2 = inp.L2.astype(np.float64)
     state = {"r0": 0}
+    s_a = np.float32(inp.act_scale) if precision == "nvfp4" else None
 
     def step():
         r0 = state["r0"]
         rows = (np.arange(rows_per_step) + r0) % case.M
         state["r0"] = (r0 + rows_per_step) % case.M
-        act = O.quantize_activations("nvfp4", inp.x[rows], pw["inv_lam"], np.float32(inp.act_scale))
-        y = O.dequantized_act("nvfp4", act) @ deq_w.T
+        act = O.quantize_activations(precision, inp.x[rows], pw["inv_lam"], s_a)
+        y = O.dequantized_act(precision, act) @ deq_w.T
         y += (act["x_hat"].astype(np.float64) @ L1) @ L2
         if inp.bias is not None:
             y += inp.bias[None, :]
@@ -160,16 +161,16 @@ def oracle_step_fn(case, inp, rows_per_step, offline):
     return step
 
 
-def time_oracle(case, inp, steps, warmup, budget_s):
+def time_oracle(case, inp, steps, warmup, budget_s, precision="nvfp4"):
     """Returns (TFLOPS, seconds per step, rows per step)."""
-    offline = oracle_offline(inp)
-    probe = oracle_step_fn(case, inp, 32, offline)
+    offline = oracle_offline(inp, precision)
+    probe = oracle_step_fn(case, inp, min(32, case.M), offline, precision)
     probe()
     t0 = time.perf_counter()
     probe()
-    t_row = (time.perf_counter() - t0) / 32
+    t_row = (time.perf_counter() - t0) / min(32, case.M)
     rows = int(max(1, min(case.M, budget_s / max(steps + warmup, 1) / max(t_row, 1e-6))))
-    fn = oracle_step_fn(case, inp, rows, offline)
+    fn = oracle_step_fn(case, inp, rows, offline, precision)
     for _ in range(warmup):
         fn()
     t0 = time.perf_counter()
@@ -177,6 +178,44 @@ def time_oracle(case, inp, steps, warmup, budget_s):
         fn()
     dt = (time.perf_counter() - t0) / steps
     return 2.0 * rows * case.N * case.K / dt / 1e12, dt, rows
+
+
+def time_oracle_configs(budget_s):
+    """The CPU oracle on every workload (a bounded sample of rows each, about
+    `budget_s` seconds per config), plus the tiny layer on one thread: the
+    per-config CPU baseline.  Host only."""
+    import workloads as wl
+    from oracle import awq as OA
+    from oracle import calibrate as OC
+    out = {}
+    for name, prec in (("tiny", "nvfp4"), ("qkv", "nvfp4"), ("mlp_up", "nvfp4"), ("mlp_down", "nvfp4"),
+                       ("int4_m4096", "int4")):
+        case = wl.SVDQ_CASES[name]
+        inp = wl.make_svdq_inputs(case, OC.calibrate)
+        tf, dt, rows = time_oracle(case, inp, 2, 1, budget_s, prec)
+        out[name] = {"precision": prec, "TFLOPS": round(tf, 6), "rows_timed": rows, "s_per_step": round(dt, 3)}
+        if name == "tiny":
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    tf1, dt1, rows1 = time_oracle(case, inp, 2, 1, budget_s, prec)
+                out["tiny_1_thread"] = {"precision": prec, "TFLOPS": round(tf1, 6), "rows_timed": rows1,
+                                        "s_per_step": round(dt1, 3)}
+            except ImportError:
+                pass
+    a = wl.make_awq_inputs(1)
+    q, sc, z = OA.awq_quantize(a.W)
+    OA.awq_linear(a.x, q, sc, z)
+    t0 = time.perf_counter()
+    reps = 3
+    for _ in range(reps):
+        OA.awq_linear(a.x, q, sc, z)
+    dt = (time.perf_counter() - t0) / reps
+    wbytes = a.N * a.K // 2 + a.N * a.K // 64 * 2 + a.N * a.K // 128
+    out["awq_m1"] = {"GB/s": round(wbytes / dt / 1e9, 3), "s_per_call": round(dt, 4),
+                     "note": "each timed call dequantizes W and multiplies in fp64"}
+    out["cores"] = _cpu_threads()
+    return out
 
 
 # ------------------------------------------------------------------ clocks
@@ -911,6 +950,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-configs", action="store_true",
+                    help="time the CPU oracle on every workload (host only) and print one JSON line")
     ap.add_argument("--no-rows", action="store_true", help="skip the INT4 / AWQ / MLP row measurements")
     ap.add_argument("--mlp-calls", type=int, default=0,
                     help="only run this many fused DiT MLP calls (untimed; for profiling) and exit")
@@ -929,6 +970,9 @@ def main():
         return
     if args.profile is not None:
         run_profile_calls(args.profile, args.calls)
+        return
+    if args.cpu_configs:
+        print(json.dumps({"cpu_oracle_configs": time_oracle_configs(args.cpu_budget / 2)}), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
