@@ -29,18 +29,9 @@
 // lora_w equals the layer's sum times 2^-(E_a[m] + E_w[n]), undone in its
 // epilogue by f_a[m] f_w[n].
 //
-// Order along K: within every 8-code word the outputs are stored as
-// elements (0, 2, 4, 6, 1, 3, 5, 7) -- the order in which the low and then
-// the high nibbles of the word's four bytes come out of the conversion.  Both
-// operands of the product are stored in this order, so every dot product
-// pairs the same elements as in natural order, and a word never straddles a
-// 64-group.
-//
-// Conversion of a code: the code's bits with bit 3 flipped are q + 8 in
-// 0..15; placed in the low byte of the fp16 pattern 0x6400 (1024, whose unit
-// in the last place is 1) they give 1024 + q + 8, and subtracting 1032 leaves
-// q exactly; one fp16 multiply by the scaled group scale gives the value
-// (exact, see above).  Two codes per packed f16x2 operation.
+// The conversion of a code and the order of the values within every 8 codes,
+// (0, 2, 4, 6, 1, 3, 5, 7) for both operands of the product, are those of
+// int4_fp16.cuh.
 //
 // One launch converts both operands (the weight rows first, then the
 // activation rows: one grid, so the two passes share a single ramp-up and
@@ -54,6 +45,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "int4_fp16.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -64,43 +56,6 @@ constexpr int DQ_ROWS = 8;
 constexpr int DQ_TPR = 16;                         // threads per row
 constexpr int DQ_THREADS = DQ_ROWS * DQ_TPR;
 constexpr int DQ_BATCH = 8;                        // chunk loads in flight per thread
-
-SVDQ_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-SVDQ_DEV uint32_t hsub2_rn(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-SVDQ_DEV uint32_t hmul2_rn(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-SVDQ_DEV uint32_t f32_to_f16x2_dup(float v) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(v));
-  return d;
-}
-// 2^e as an fp32 bit pattern, -126 <= e <= 127.
-SVDQ_DEV float exp2i(int e) { return __int_as_float((e + 127) << 23); }
-
-// Eight codes (one 32-bit word, code 2j in the low nibble of byte j) times
-// the f16x2 scale s2 -> four f16x2 words in the order (0,2), (4,6), (1,3), (5,7).
-SVDQ_DEV void dequant_word(uint32_t w, uint32_t s2, uint32_t (&o)[4]) {
-  w ^= 0x88888888u;                          // q + 8 in every nibble
-  const uint32_t lo = w & 0x0F0F0F0Fu;       // codes 0, 2, 4, 6 (one per byte)
-  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
-  constexpr uint32_t kMagic = 0x64646464u;   // high byte of the fp16 pattern of 1024
-  constexpr uint32_t kBias = 0x64086408u;    // 1032 in both halves
-  o[0] = hmul2_rn(hsub2_rn(prmt(lo, kMagic, 0x4140u), kBias), s2);
-  o[1] = hmul2_rn(hsub2_rn(prmt(lo, kMagic, 0x4342u), kBias), s2);
-  o[2] = hmul2_rn(hsub2_rn(prmt(hi, kMagic, 0x4140u), kBias), s2);
-  o[3] = hmul2_rn(hsub2_rn(prmt(hi, kMagic, 0x4342u), kBias), s2);
-}
 
 __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Params pw, DequantInt4Params pa) {
   extern __shared__ float dq_smem[];
@@ -129,14 +84,9 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
   for (int g = l; g < groups; g += DQ_TPR) mx = fmaxf(mx, sc[g * DQ_ROWS + r]);
 #pragma unroll
   for (int o = DQ_TPR / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  int e = 0;
-  if (mx > 0.f) {
-    const int biased = (__float_as_int(mx) >> 23) & 0xFF;   // 0 for an fp32 subnormal
-    e = (biased == 0 ? -126 : biased - 127) - 12;
-    e = e < -100 ? -100 : (e > 100 ? 100 : e);
-  }
-  const float inv = exp2i(-e);
-  if (row_ok && l == 0) p.factor[row] = exp2i(e);
+  const int e = i4_row_exponent(mx);
+  const float inv = i4_exp2i(-e);
+  if (row_ok && l == 0) p.factor[row] = i4_exp2i(e);
 
   if (row_ok && p.out != nullptr) {
     // Codes: 16 bytes (32 codes, all in one 64-group) per chunk.
@@ -156,14 +106,11 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
         if (j < chunks) {
           // The scaled group scale: exact in fp32 (a power-of-two factor),
           // then in fp16 for every group within 2^29 of the row's largest.
-          const uint32_t s2 = f32_to_f16x2_dup(__fmul_rn(sc[(j >> 1) * DQ_ROWS + r], inv));
-          uint32_t o[4][4];
-          dequant_word(w[b].x, s2, o[0]);
-          dequant_word(w[b].y, s2, o[1]);
-          dequant_word(w[b].z, s2, o[2]);
-          dequant_word(w[b].w, s2, o[3]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[4 * j + q] = make_uint4(o[q][0], o[q][1], o[q][2], o[q][3]);
+          const uint32_t s2 = i4_f16x2_dup(__fmul_rn(sc[(j >> 1) * DQ_ROWS + r], inv));
+          dst[4 * j] = i4_dequant_word(w[b].x, s2);
+          dst[4 * j + 1] = i4_dequant_word(w[b].y, s2);
+          dst[4 * j + 2] = i4_dequant_word(w[b].z, s2);
+          dst[4 * j + 3] = i4_dequant_word(w[b].w, s2);
         }
       }
     }

@@ -60,6 +60,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "int4_fp16.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -119,39 +120,6 @@ SVDQ_DEV uint64_t sw128_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024,
 SVDQ_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 SVDQ_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-SVDQ_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-SVDQ_DEV uint32_t hsub2_rn(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-SVDQ_DEV uint32_t hmul2_rn(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-SVDQ_DEV uint32_t f32_to_f16x2_dup(float v) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(v));
-  return d;
-}
-// Eight codes (one word, code 2j in the low nibble of byte j) times the
-// f16x2 scale s2 -> 16 bytes of fp16 in the order (0,2), (4,6), (1,3), (5,7):
-// the code's bits with bit 3 flipped (q + 8) in the low byte of the fp16
-// pattern of 1024, minus 1032, times the scale.
-SVDQ_DEV uint4 dequant_word(uint32_t w, uint32_t s2) {
-  w ^= 0x88888888u;
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  constexpr uint32_t kMagic = 0x64646464u, kBias = 0x64086408u;
-  return make_uint4(hmul2_rn(hsub2_rn(prmt(lo, kMagic, 0x4140u), kBias), s2),
-                    hmul2_rn(hsub2_rn(prmt(lo, kMagic, 0x4342u), kBias), s2),
-                    hmul2_rn(hsub2_rn(prmt(hi, kMagic, 0x4140u), kBias), s2),
-                    hmul2_rn(hsub2_rn(prmt(hi, kMagic, 0x4342u), kBias), s2));
-}
 SVDQ_DEV uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -182,7 +150,7 @@ SVDQ_DEV void dequant_row(uint32_t codes, uint32_t s2, uint32_t tile, int r) {
   const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
   const uint32_t row = tile + (uint32_t)r * 128u;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) sts_v4(row + (uint32_t)((c ^ (r & 7)) << 4), dequant_word(w[c], s2));
+  for (int c = 0; c < 8; ++c) sts_v4(row + (uint32_t)((c ^ (r & 7)) << 4), i4_dequant_word(w[c], s2));
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -362,8 +330,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t sc = smem_u32(scl(stage));
             const float sa = __uint_as_float(lds_u16(sc + 2 * t) << 16);
             const float sb = __uint_as_float(lds_u16(sc + 256 + 2 * t) << 16);
-            dequant_row(smem_u32(a4(stage)) + 32 * t, f32_to_f16x2_dup(__fmul_rn(sa, inv_a)), smem_u32(a16(stage)), t);
-            dequant_row(smem_u32(b4(stage)) + 32 * t, f32_to_f16x2_dup(__fmul_rn(sb, inv_b)), smem_u32(b16(stage)), t);
+            dequant_row(smem_u32(a4(stage)) + 32 * t, i4_f16x2_dup(__fmul_rn(sa, inv_a)), smem_u32(a16(stage)), t);
+            dequant_row(smem_u32(b4(stage)) + 32 * t, i4_f16x2_dup(__fmul_rn(sb, inv_b)), smem_u32(b16(stage)), t);
             // The generic-proxy writes, before the tensor core reads them.
             fence_proxy_async_smem();
           }
