@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -305,9 +306,12 @@ static bool use_copy_quantizer() {
   return v && strcmp(v, "copy") == 0;
 }
 
+// w_side (INT4 only, or null): the layer's weight rows to convert to fp16
+// operands in extra blocks of the quantizer's launch (int4_dequant_rows.cuh).
 static int quantize_act_impl(int precision, int M, int K, int rank, const void* x, const float* inv_smooth,
                              const void* lora_down, float act_scale, float weight_scale, void* act_codes,
-                             void* act_scales, void* lora_act, int* dev_status, void* stream) {
+                             void* act_scales, void* lora_act, int* dev_status, void* stream,
+                             const DequantInt4Params* w_side = nullptr) {
   if (precision != SVDQ_NVFP4 && precision != SVDQ_INT4)
     return fail(SVDQ_ERR_INVALID_ARG, "precision %d is not SVDQ_NVFP4 or SVDQ_INT4", precision);
   if (M <= 0 || K <= 0) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M=%d K=%d must be positive", M, K);
@@ -349,6 +353,13 @@ static int quantize_act_impl(int precision, int M, int K, int rank, const void* 
   p.act_codes = static_cast<uint8_t*>(act_codes);
   p.act_scales = static_cast<uint8_t*>(act_scales);
   p.lora_act = static_cast<uint16_t*>(lora_act);
+  p.s1_blocks = p.M_pad / 16;
+  if (w_side != nullptr && precision == SVDQ_INT4 && w_side->R > 0) {
+    // One conversion block per 32 weight rows (the caller checked that they
+    // fit beside the quantizer's own CTAs, two of which fit per SM).
+    p.w_side = *w_side;
+    p.w_blocks = (w_side->R + 31) / 32;
+  }
   if (precision == SVDQ_NVFP4 && !use_copy_quantizer()) {
     // TMA-fed kernel: x [M, K] bf16 and L1^T [32, K] fp16 in 64 x 32 boxes.
     CUtensorMap tx, tl;
@@ -514,7 +525,7 @@ static Int4LayerGemm int4_layer_gemm() {
 static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const void* act_scales,
                               const void* lora_act, const void* w_codes, const void* w_scales, const void* lora_up,
                               const void* bias, void* y, uint8_t* region, int* dev_status, cudaStream_t stream,
-                              bool pdl, bool in_gemm) {
+                              bool pdl, bool in_gemm, bool weights_done = false) {
   long long o[7];
   int4_operand_offsets(M, N, K, o);
   uint16_t* a16 = reinterpret_cast<uint16_t*>(region + o[0]);
@@ -576,9 +587,11 @@ static int gemm_int4_f16_impl(int M, int N, int K, const void* act_codes, const 
   if (!ok) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the fp16-operand INT4 GEMM");
   u.sfa = u.a;   // not read
   u.sfb = u.a;
+  // The weight side is converted here unless the quantizer's launch already
+  // did it (int4_w_side): then this launch covers the activation rows only.
   DequantInt4Params da{M, K, (int)round_up(M, 256), static_cast<const uint8_t*>(act_codes),
                        static_cast<const uint16_t*>(act_scales), static_cast<const uint16_t*>(lora_act), a16, la, fa};
-  DequantInt4Params dw{N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
+  DequantInt4Params dw{weights_done ? 0 : N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
                        static_cast<const uint16_t*>(w_scales), static_cast<const uint16_t*>(lora_up), w16, lb, fw};
   if (int s = check_cuda(launch_dequant_int4(dw, da, stream, pdl), "dequant_int4 launch")) return s;
   GemmNvfp4Params p{};
@@ -729,17 +742,36 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
     return layer_nvfp4_impl(M, N, K, x, inv_smooth, lora_down, act_scale, w_codes, w_scales, weight_scale, lora_up,
                             bias, y, ws, off, dev_status, static_cast<cudaStream_t>(stream), pdl_on());
   }
+  const Int4LayerGemm g4 = int4_layer_gemm();
+  // INT4 on fp16 operands written out first: when one block per 32 weight
+  // rows fits in the SM slots the quantizer leaves free (it runs two 512-
+  // thread CTAs per SM, one per 16 rows), extra blocks of the quantizer's
+  // launch convert the weight rows beside it; otherwise the operand pass
+  // converts both sides after it.  Measured at K = N = 3072: 48.5 against
+  // 51.8 us at M = 1024; with too few free slots (M = 4096) the extra blocks
+  // lengthen the quantizer's tail instead (115 against 100 us).
+  const bool int4_w_side = precision == SVDQ_INT4 && g4 == Int4LayerGemm::kF16Operands &&
+                           2 * sms - (int)(round_up(M, 256) / 16) >= (N + 31) / 32;
+  DequantInt4Params w_side{};
+  if (int4_w_side) {
+    long long o[7];
+    int4_operand_offsets(M, N, K, o);
+    w_side = DequantInt4Params{N, K, (int)round_up(N, 256), static_cast<const uint8_t*>(w_codes),
+                               static_cast<const uint16_t*>(w_scales), static_cast<const uint16_t*>(lora_up),
+                               reinterpret_cast<uint16_t*>(ws + off[4] + o[3]),
+                               reinterpret_cast<uint16_t*>(ws + off[4] + o[4]),
+                               reinterpret_cast<float*>(ws + off[4] + o[5])};
+  }
   if (int s = quantize_act_impl(precision, M, K, rank, x, inv_smooth, lora_down, act_scale, weight_scale, codes,
-                                scales, lora, dev_status, stream))
+                                scales, lora, dev_status, stream, int4_w_side ? &w_side : nullptr))
     return s;
   if (precision == SVDQ_INT4) {
-    const Int4LayerGemm g = int4_layer_gemm();
-    if (g == Int4LayerGemm::kI8)
+    if (g4 == Int4LayerGemm::kI8)
       return gemm_int4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, dev_status,
                             static_cast<cudaStream_t>(stream), pdl_on(), sms);
     return gemm_int4_f16_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, y, ws + off[4],
                               dev_status, static_cast<cudaStream_t>(stream), pdl_on(),
-                              g == Int4LayerGemm::kDequantInGemm);
+                              g4 == Int4LayerGemm::kDequantInGemm, int4_w_side);
   }
   return gemm_nvfp4_impl(M, N, K, codes, scales, lora, w_codes, w_scales, lora_up, bias, act_scale * weight_scale,
                          y, dev_status, static_cast<cudaStream_t>(stream), pdl_on(), sms);

@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "int4_dequant_rows.cuh"
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -157,6 +158,18 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
   const bool ok0 = row0 < p.M, ok1 = row1 < p.M;
   const int K = p.K;
   pdl_wait();  // x and the weights of the previous kernel's making
+  if constexpr (!kNvfp4) {
+    // The blocks past the quantizer's convert the layer's weight rows (they
+    // depend on nothing this kernel writes), on the SM slots the quantizer
+    // leaves free.
+    if (p.w_side.R > 0 && (int)blockIdx.x >= p.s1_blocks) {
+      pdl_launch_dependents();
+      float* sc = reinterpret_cast<float*>(s1_ring);
+      for (int r0 = ((int)blockIdx.x - p.s1_blocks) * 32; r0 < p.w_side.R; r0 += p.w_blocks * 32)
+        int4_dequant_rows<32>(p.w_side, r0, sc);
+      return;
+    }
+  }
   const int nunits = K / (32 * STEP);
 
   const uint16_t* __restrict__ x = p.x;
@@ -368,7 +381,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
 
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl) {
   const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
-  dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS);
+  dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS + (!nvfp4 && p.w_side.R > 0 ? p.w_blocks : 0));
   const size_t ring_bytes = (size_t)(nvfp4 ? s1_prefetch<true>() : s1_prefetch<false>()) * (nvfp4 ? 1 : 2) *
                             S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
   cudaLaunchConfig_t cfg = {};

@@ -26,6 +26,20 @@ enum DeviceStatus : int {
   kDevTimeoutDrain = 4,
 };
 
+// INT4 rows -> exact fp16 operands for the fp16 tensor pipe (dequant_int4.cu):
+// out[r, k] = fp16(s[r, k/64] 2^-E[r] q[r, k]) with K permuted within every
+// 8-code word as (0, 2, 4, 6, 1, 3, 5, 7), lora_out = lora_in 2^-E[r],
+// factor[r] = 2^E[r].
+struct DequantInt4Params {
+  int R, K, R_pad;
+  const uint8_t* codes;       // [R, K/2]
+  const uint16_t* scales;     // bf16 [K/64][R_pad]
+  const uint16_t* lora_in;    // bf16 [R, 64] or null
+  uint16_t* out;              // fp16 [R, K], or null: only factor and lora_out
+  uint16_t* lora_out;         // bf16 [R, 64] (unused when lora_in is null)
+  float* factor;              // fp32 [R]
+};
+
 struct QuantActParams {
   int M, K, M_pad;            // M_pad: rows of the scale buffer (multiple of 256)
   const uint16_t* x;          // bf16 [M, K]
@@ -37,6 +51,12 @@ struct QuantActParams {
   uint8_t* act_codes;         // [M, K/2]
   uint8_t* act_scales;        // NVFP4: tiled e4m3; INT4: bf16 [K/64][M_pad]
   uint16_t* lora_act;         // bf16 [M, 2r]  (hi | lo)
+  // INT4: blocks s1_blocks .. s1_blocks + w_blocks - 1 of the launch convert
+  // the rows of w_side (the layer's weight operand, int4_dequant_rows.cuh)
+  // beside the quantizer, 32 rows at a time; w_side.R = 0: none.
+  DequantInt4Params w_side;
+  int s1_blocks;
+  int w_blocks;
 };
 
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl);
@@ -159,20 +179,6 @@ cudaError_t launch_gemm_f16_pair(const GemmNvfp4Params& p, const GemmPairTmaps& 
 // both in 64 x 128 / 64 x 32 SWIZZLE_128B boxes (the quantizer's chunks).
 cudaError_t launch_layer_nvfp4_pair(const GemmNvfp4Params& p, const GemmPairTmaps& t, const CUtensorMap& tm_x,
                                     const CUtensorMap& tm_l1, cudaStream_t stream, bool pdl);
-
-// INT4 rows -> exact fp16 operands for the fp16 tensor pipe (dequant_int4.cu):
-// out[r, k] = fp16(s[r, k/64] 2^-E[r] q[r, k]) with K permuted within every
-// 8-code word as (0, 2, 4, 6, 1, 3, 5, 7), lora_out = lora_in 2^-E[r],
-// factor[r] = 2^E[r].
-struct DequantInt4Params {
-  int R, K, R_pad;
-  const uint8_t* codes;       // [R, K/2]
-  const uint16_t* scales;     // bf16 [K/64][R_pad]
-  const uint16_t* lora_in;    // bf16 [R, 64] or null
-  uint16_t* out;              // fp16 [R, K], or null: only factor and lora_out
-  uint16_t* lora_out;         // bf16 [R, 64] (unused when lora_in is null)
-  float* factor;              // fp32 [R]
-};
 
 size_t dequant_int4_smem_bytes(int K);
 // One launch for both operands (pw: weight rows, pa: activation rows; same K).

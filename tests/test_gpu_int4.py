@@ -123,7 +123,8 @@ def _unpermute(a16):
 
 @pytest.mark.parametrize("name,kw,zero_row", [("int4_m1024", dict(M=300, N=512), 7),
                                               ("int4_m1024", dict(M=129, N=256, K=1024), None),
-                                              ("int4_m2048", {}, 1000)])
+                                              ("int4_m2048", {}, 1000),   # weight rows in the quantizer's launch
+                                              ("int4_m4096", {}, None)])  # both sides in the operand pass
 def test_int4_fp16_operands_are_the_oracle_values(name, kw, zero_row):
     """The layer's fp16 operands (workspace region [4]) against the oracle's
     codes and scales, bit for bit: A' from the activation quantizer, W' from
