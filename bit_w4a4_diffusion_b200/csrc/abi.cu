@@ -749,9 +749,11 @@ int svdq_w4a4_linear(int precision, int M, int N, int K, int rank, const void* x
   // launch convert the weight rows beside it; otherwise the operand pass
   // converts both sides after it.  Measured at K = N = 3072: 48.5 against
   // 51.8 us at M = 1024; with too few free slots (M = 4096) the extra blocks
-  // lengthen the quantizer's tail instead (115 against 100 us).
+  // lengthen the quantizer's tail instead (115 against 100 us).  The extra
+  // blocks stage their rows in the quantizer's 96 KB ring, which bounds K
+  // (23552 at most).
   const bool int4_w_side = precision == SVDQ_INT4 && g4 == Int4LayerGemm::kF16Operands &&
-                           2 * sms - (int)(round_up(M, 256) / 16) >= (N + 31) / 32;
+                           2 * sms - (int)(round_up(M, 256) / 16) >= (N + 31) / 32 && int4_weight_side_fits(K);
   DequantInt4Params w_side{};
   if (int4_w_side) {
     long long o[7];

@@ -50,7 +50,7 @@ constexpr int DQ_ROWS = 8;
 constexpr int DQ_THREADS = DQ_ROWS * kDqThreadsPerRow;
 
 __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Params pw, DequantInt4Params pa) {
-  extern __shared__ float dq_smem[];   // [K/64][DQ_ROWS] scales
+  extern __shared__ float dq_smem[];   // scales, then the code stage (int4_dequant_rows.cuh)
   const int blocks_w = (pw.R + DQ_ROWS - 1) / DQ_ROWS;
   const bool is_w = (int)blockIdx.x < blocks_w;
   const DequantInt4Params p = is_w ? pw : pa;
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(DQ_THREADS) dequant_int4_kernel(DequantInt4Par
 
 }  // namespace
 
-size_t dequant_int4_smem_bytes(int K) { return (size_t)(K / 64) * DQ_ROWS * sizeof(float); }
+size_t dequant_int4_smem_bytes(int K) { return int4_dequant_rows_smem(DQ_ROWS, K); }
 
 cudaError_t launch_dequant_int4(const DequantInt4Params& pw, const DequantInt4Params& pa, cudaStream_t stream,
                                 bool pdl) {

@@ -4,13 +4,17 @@
 // arithmetic).  Used by the operand-pass kernel and by the extra blocks of
 // the INT4 quantizer's launch that convert the weight rows beside it.
 //
-// kRows * 16 threads, 16 per row: thread (r, l) takes the 16-byte code chunks
-// l, l + 16, ... of row r (a row's 16 threads read 256 contiguous bytes per
-// step), issuing the loads of up to eight chunks before it converts any.  The
-// rows' scales are staged in `sc` (shared, (K/64) * kRows floats,
-// group-major so that a group's row scales are one contiguous read) and a
-// row's largest scale is a max over its 16 threads.  Every thread of the
-// block calls it (it contains block barriers).
+// kRows * 16 threads, 16 per row.  The rows' scales are staged in shared
+// memory (group-major, so that a group's row scales are one contiguous read)
+// and a row's largest scale is a max over its 16 threads.  The codes go
+// through shared memory too, kDqChunkWords 4-byte words (8 codes each) of
+// every row at a time: the block loads them with 16-byte loads, then thread
+// (r, l) converts words l, l + 16, ... of row r, so that each store
+// instruction writes 256 contiguous bytes of a row (one 16-byte fp16 group
+// of 8 values per thread).  Converting a whole 16-byte chunk per thread
+// instead leaves every store 64 bytes apart from its neighbour's, which
+// writes each 32-byte sector in two halves.  Every thread of the block calls
+// it (it contains block barriers).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -22,12 +26,20 @@
 namespace svdq {
 
 constexpr int kDqThreadsPerRow = 16;
-constexpr int kDqBatch = 8;   // chunk loads in flight per thread
+constexpr int kDqChunkWords = 384;                      // 3072 codes of a row per staging round
+constexpr int kDqStageStride = kDqChunkWords + 16;      // words; rows r, r + 1 land 16 banks apart
+
+// Shared memory the routine needs for kRows rows of length K.
+__host__ __device__ constexpr size_t int4_dequant_rows_smem(int rows, int K) {
+  return (size_t)(K / 64) * rows * sizeof(float) + (size_t)rows * kDqStageStride * sizeof(uint32_t);
+}
 
 template <int kRows>
-__device__ __forceinline__ void int4_dequant_rows(const DequantInt4Params& p, int r0, float* sc) {
+__device__ __forceinline__ void int4_dequant_rows(const DequantInt4Params& p, int r0, float* smem) {
   constexpr int kThreads = kRows * kDqThreadsPerRow;
   const int groups = p.K / 64;
+  float* sc = smem;                                                   // [groups][kRows]
+  uint32_t* stage = reinterpret_cast<uint32_t*>(smem + groups * kRows);   // [kRows][kDqStageStride]
   const int tid = threadIdx.x;
   const int r = tid / kDqThreadsPerRow, l = tid % kDqThreadsPerRow;
   const int row = r0 + r;
@@ -35,12 +47,15 @@ __device__ __forceinline__ void int4_dequant_rows(const DequantInt4Params& p, in
 
   // Scales of the block's rows (rows past R read the zero padding: R_pad is
   // a multiple of 256 and r0 + kRows <= R_pad).  The first barrier ends the
-  // previous call's reads of `sc`.
+  // previous call's reads of shared memory.
   __syncthreads();
   for (int i = tid; i < groups * kRows; i += kThreads) {
     const int g = i / kRows, rr = i - g * kRows;
     sc[i] = __bfloat162float(__ushort_as_bfloat16(p.scales[(size_t)g * p.R_pad + r0 + rr]));
   }
+  // The low-rank operand row is read now, ahead of the stores below.
+  uint2 lora = make_uint2(0, 0);
+  if (row_ok && p.lora_in != nullptr) lora = __ldg(reinterpret_cast<const uint2*>(p.lora_in + (size_t)row * 64) + l);
   __syncthreads();
   float mx = 0.f;
   for (int g = l; g < groups; g += kDqThreadsPerRow) mx = fmaxf(mx, sc[g * kRows + r]);
@@ -50,29 +65,36 @@ __device__ __forceinline__ void int4_dequant_rows(const DequantInt4Params& p, in
   const float inv = i4_exp2i(-e);
   if (row_ok && l == 0) p.factor[row] = i4_exp2i(e);
 
-  if (row_ok && p.out != nullptr) {
-    // Codes: 16 bytes (32 codes, all in one 64-group) per chunk.
-    const int chunks = p.K / 32;
-    const uint4* src = reinterpret_cast<const uint4*>(p.codes + (size_t)row * (p.K / 2));
-    uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.K);
-    for (int j0 = l; j0 < chunks; j0 += kDqThreadsPerRow * kDqBatch) {
-      uint4 w[kDqBatch];
+  if (p.out != nullptr) {
+    const int words = p.K / 8;   // a multiple of 32 (K % 256 == 0)
+    for (int w0 = 0; w0 < words; w0 += kDqChunkWords) {
+      const int nw = words - w0 < kDqChunkWords ? words - w0 : kDqChunkWords;
+      const int nq = nw / 4;     // 16-byte loads per row
+      // The previous round's readers are done with the stage.
+      __syncthreads();
+      constexpr int kLoads = (kRows * kDqChunkWords / 4 + kThreads - 1) / kThreads;
+      uint4 v[kLoads];
 #pragma unroll
-      for (int b = 0; b < kDqBatch; ++b) {
-        const int j = j0 + kDqThreadsPerRow * b;
-        if (j < chunks) w[b] = __ldg(src + j);
+      for (int b = 0; b < kLoads; ++b) {
+        const int i = tid + b * kThreads;
+        const int rr = i / nq, c = i - rr * nq;
+        if (rr < kRows && r0 + rr < p.R)
+          v[b] = __ldg(reinterpret_cast<const uint4*>(p.codes + (size_t)(r0 + rr) * (p.K / 2) + (size_t)w0 * 4) + c);
       }
 #pragma unroll
-      for (int b = 0; b < kDqBatch; ++b) {
-        const int j = j0 + kDqThreadsPerRow * b;
-        if (j < chunks) {
+      for (int b = 0; b < kLoads; ++b) {
+        const int i = tid + b * kThreads;
+        const int rr = i / nq, c = i - rr * nq;
+        if (rr < kRows && r0 + rr < p.R) *reinterpret_cast<uint4*>(stage + rr * kDqStageStride + 4 * c) = v[b];
+      }
+      __syncthreads();
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.K) + w0;
+        for (int w = l; w < nw; w += kDqThreadsPerRow) {
           // The scaled group scale: exact in fp32 (a power-of-two factor),
           // then in fp16 for every group within 2^29 of the row's largest.
-          const uint32_t s2 = i4_f16x2_dup(__fmul_rn(sc[(j >> 1) * kRows + r], inv));
-          dst[4 * j] = i4_dequant_word(w[b].x, s2);
-          dst[4 * j + 1] = i4_dequant_word(w[b].y, s2);
-          dst[4 * j + 2] = i4_dequant_word(w[b].z, s2);
-          dst[4 * j + 3] = i4_dequant_word(w[b].w, s2);
+          const uint32_t s2 = i4_f16x2_dup(__fmul_rn(sc[((w0 + w) >> 3) * kRows + r], inv));
+          dst[w] = i4_dequant_word(stage[r * kDqStageStride + w], s2);
         }
       }
     }
@@ -80,14 +102,13 @@ __device__ __forceinline__ void int4_dequant_rows(const DequantInt4Params& p, in
   if (row_ok && p.lora_in != nullptr) {
     // The low-rank operand row, scaled by the same power of two: four values
     // per thread.
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.lora_in + (size_t)row * 64) + l);
     auto scale2 = [&](uint32_t b) {
       const float lo = __fmul_rn(__uint_as_float(b << 16), inv);
       const float hi = __fmul_rn(__uint_as_float(b & 0xFFFF0000u), inv);
       return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
     };
-    reinterpret_cast<uint2*>(p.lora_out + (size_t)row * 64)[l] = make_uint2(scale2(v.x), scale2(v.y));
+    reinterpret_cast<uint2*>(p.lora_out + (size_t)row * 64)[l] = make_uint2(scale2(lora.x), scale2(lora.y));
   }
 }
 

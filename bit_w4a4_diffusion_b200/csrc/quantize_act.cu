@@ -379,7 +379,12 @@ __global__ void __launch_bounds__(S1_THREADS, 2) quantize_act_kernel(QuantActPar
 
 }  // namespace
 
+bool int4_weight_side_fits(int K) {
+  return int4_dequant_rows_smem(32, K) <= (size_t)s1_prefetch<false>() * 2 * S1_SLOT_U4 * S1_THREADS * sizeof(uint4);
+}
+
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl) {
+  if (!nvfp4 && p.w_side.R > 0 && !int4_weight_side_fits(p.K)) return cudaErrorInvalidValue;
   const int rows_pad = p.M_pad;  // cover scale padding rows too (they get zero scales)
   dim3 grid((rows_pad + S1_ROWS - 1) / S1_ROWS + (!nvfp4 && p.w_side.R > 0 ? p.w_blocks : 0));
   const size_t ring_bytes = (size_t)(nvfp4 ? s1_prefetch<true>() : s1_prefetch<false>()) * (nvfp4 ? 1 : 2) *

@@ -60,6 +60,9 @@ struct QuantActParams {
 };
 
 cudaError_t launch_quantize_act(const QuantActParams& p, bool nvfp4, cudaStream_t stream, bool pdl);
+// Whether the INT4 quantizer's shared-memory ring holds the staging of its
+// weight-side blocks (32 rows of length K) as well.
+bool int4_weight_side_fits(int K);
 // NVFP4, TMA-fed: x [M, K] bf16 and L1^T [32, K] fp16 as 64 x 32 SWIZZLE_128B boxes.
 cudaError_t launch_quantize_nvfp4(const QuantActParams& p, const CUtensorMap& tm_x, const CUtensorMap& tm_l1t,
                                   int* dev_status, unsigned long long timeout_ns, cudaStream_t stream, bool pdl);
