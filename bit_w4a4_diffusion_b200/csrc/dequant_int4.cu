@@ -21,7 +21,9 @@
 //               the row's largest scale (smaller groups round as fp16
 //               subnormals, an error below 2^-36 of the row's largest value);
 //               the largest is below 8 * 2^13 = 65536, within fp16's 65504
-//               since a scale's significand is at most 255/128
+//               since a scale's significand is at most 255/128.  Both hold
+//               while E is not clamped (largest scale in [2^-88, 2^113));
+//               beyond 2^113, 8 s 2^-100 leaves fp16's range
 //   lora[r,:] = lora_in[r,:] 2^-E[r]        (bf16, exact)
 //   f[r]      = 2^E[r]                       (fp32)
 //

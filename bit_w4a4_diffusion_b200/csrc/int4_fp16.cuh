@@ -11,7 +11,9 @@
 //          row whose scales are all zero),
 //
 // and then exact for every group within 2^29 of the row's largest scale
-// (smaller groups round as fp16 subnormals).  Within every 8-code word the
+// (smaller groups round as fp16 subnormals), as long as the clamp is not
+// reached: a row whose largest scale is 2^113 or more keeps E = 100 and its
+// largest values leave fp16's range.  Within every 8-code word the
 // values come out in the order (0, 2, 4, 6, 1, 3, 5, 7); every kernel that
 // writes an operand uses this order for both operands of the product.
 #pragma once

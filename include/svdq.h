@@ -208,7 +208,10 @@ int svdq_w4a4_gemm(int precision, int M, int N, int K, int rank, const void* act
  *    scale significand times a code of at most 3 bits fits fp16's 11), each
  *    row scaled by a power of two 2^-E (E = floor(log2 of the row's largest
  *    scale) - 12, clamped to [-100, 100]) that the epilogue undoes; exact for
- *    every group within 2^29 of its row's largest scale.  Same products,
+ *    every group within 2^29 of its row's largest scale while that scale
+ *    lies in [2^-88, 2^113) (E not clamped).  A row whose largest scale is
+ *    2^113 or more (values near 10^34) overflows the fp16 operand: use
+ *    SVDQ_INT4_LAYER_GEMM=i8 for such data.  Same products,
  *    summed in fp32 in another order, so y can differ from quantize + gemm in
  *    its last bits.  SVDQ_INT4_LAYER_GEMM in the environment (read at every
  *    call) selects "dq" (the GEMM builds the fp16 tiles itself in shared
